@@ -1,0 +1,228 @@
+"""Seeded synthetic inputs for exact tiled attention (prefill and paged split-KV decode).
+
+This module is shared by the parity tests, the bench and the oracle driver. It holds no
+attention arithmetic: it draws numbers (SplitMix64 + Box-Muller, see gen.c), rounds them to
+the storage dtype and lays them out in the shapes the workloads use. The 16-bit bit patterns
+it returns are the inputs; the CUDA path uploads them unchanged and the oracle widens them
+exactly to fp64.
+
+Stream numbering per workload: q=0, k=1, v=2, sequence lengths=3, page permutation=4.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass, field
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SO = os.path.join(_HERE, "libmfa_inputs.so")
+_SRC = os.path.join(_HERE, "gen.c")
+
+FP16, BF16 = 0, 1
+DTYPE_NAMES = {FP16: "fp16", BF16: "bf16"}
+STREAM_Q, STREAM_K, STREAM_V, STREAM_LENS, STREAM_PERM = 0, 1, 2, 3, 4
+PAGE_SIZE = 16
+
+
+def build() -> str:
+    """Compile gen.c into libmfa_inputs.so (gcc, OpenMP)."""
+    if (not os.path.exists(_SO)) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", _SO, _SRC, "-lm"])
+    return _SO
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_SO)
+        lib.mfa_gen_draw.restype = ctypes.c_uint64
+        lib.mfa_gen_draw.argtypes = [ctypes.c_uint64] * 3
+        lib.mfa_gen_u64.restype = None
+        lib.mfa_gen_u64.argtypes = [ctypes.c_uint64, ctypes.c_uint64, ctypes.c_uint64,
+                                    ctypes.c_int64, ctypes.c_void_p]
+        lib.mfa_gen_normal.restype = None
+        lib.mfa_gen_normal.argtypes = [ctypes.c_uint64, ctypes.c_uint64, ctypes.c_uint64,
+                                       ctypes.c_int64, ctypes.c_double, ctypes.c_int,
+                                       ctypes.c_void_p, ctypes.c_void_p]
+        lib.mfa_gen_widen.restype = None
+        lib.mfa_gen_widen.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p]
+        _lib = lib
+    return _lib
+
+
+def draws_u64(seed: int, stream: int, n: int, offset: int = 0) -> np.ndarray:
+    out = np.empty(n, dtype=np.uint64)
+    if n:
+        _load().mfa_gen_u64(seed, stream, offset, n, out.ctypes.data)
+    return out
+
+
+def normal_bits(seed: int, stream: int, shape, dtype: int, mul: float = 1.0,
+                offset: int = 0) -> np.ndarray:
+    """N(0,1)*mul values rounded to fp16/bf16, returned as uint16 bit patterns of `shape`."""
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.uint16)
+    if n:
+        _load().mfa_gen_normal(seed, stream, offset, n, mul, dtype, out.ctypes.data, None)
+    return out.reshape(shape)
+
+
+def normal_f64(seed: int, stream: int, n: int, offset: int = 0) -> np.ndarray:
+    """The unrounded fp64 normals (used to check the generator's distribution)."""
+    out = np.empty(n, dtype=np.float64)
+    if n:
+        _load().mfa_gen_normal(seed, stream, offset, n, 1.0, 2, None, out.ctypes.data)
+    return out
+
+
+def widen(bits: np.ndarray, dtype: int) -> np.ndarray:
+    """Exact fp64 values of fp16/bf16 bit patterns."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    out = np.empty(bits.shape, dtype=np.float64)
+    if bits.size:
+        _load().mfa_gen_widen(bits.ctypes.data, bits.size, dtype, out.ctypes.data)
+    return out
+
+
+def uniform_ints(seed: int, stream: int, n: int, lo: int, hi: int) -> np.ndarray:
+    """n integers uniform on [lo, hi] inclusive (multiply-high of the top 32 bits)."""
+    d = draws_u64(seed, stream, n) >> np.uint64(32)
+    span = np.uint64(hi - lo + 1)
+    return (np.int64(lo) + ((d * span) >> np.uint64(32)).astype(np.int64)).astype(np.int64)
+
+
+def permutation(seed: int, stream: int, n: int) -> np.ndarray:
+    """Fisher-Yates shuffle of [0, n): step k (k = 0..n-2) swaps i = n-1-k with j uniform on [0, i]."""
+    perm = np.arange(n, dtype=np.int64)
+    if n < 2:
+        return perm
+    d = draws_u64(seed, stream, n - 1) >> np.uint64(32)
+    i_vals = np.arange(n - 1, 0, -1, dtype=np.uint64)
+    j_vals = ((d * (i_vals + np.uint64(1))) >> np.uint64(32)).astype(np.int64)
+    for k in range(n - 1):
+        i = n - 1 - k
+        j = j_vals[k]
+        perm[i], perm[j] = perm[j], perm[i]
+    return perm
+
+
+NAN_BITS = {FP16: 0x7E00, BF16: 0x7FC0}
+
+
+@dataclass
+class PrefillCase:
+    """Shapes and flags of one dense forward workload; q [B,Hq,Nq,D], k/v [B,Hkv,Nk,D]."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Nq: int
+    Nk: int
+    D: int
+    dtype: int
+    causal: bool
+    win_l: int = -1
+    win_r: int = -1
+    softcap: float = 0.0
+    mul: float = 1.0
+    seed: int = 1
+    scale: float | None = None
+
+    def scale_f32(self) -> float:
+        s = self.scale if self.scale is not None else 1.0 / np.sqrt(self.D)
+        return float(np.float32(s))
+
+    def tensors(self):
+        """(q, k, v) as uint16 bit patterns."""
+        q = normal_bits(self.seed, STREAM_Q, (self.B, self.Hq, self.Nq, self.D), self.dtype, self.mul)
+        k = normal_bits(self.seed, STREAM_K, (self.B, self.Hkv, self.Nk, self.D), self.dtype, self.mul)
+        v = normal_bits(self.seed, STREAM_V, (self.B, self.Hkv, self.Nk, self.D), self.dtype, self.mul)
+        return q, k, v
+
+
+@dataclass
+class DecodeCase:
+    """Paged split-KV decode workload.
+
+    q [B,Hq,Nq,D]; k/v pages [num_pages, 16, Hkv, D]; block_table int32 [B, max_pages];
+    seq_lens int32 [B]. Pages are handed out in the order of a seeded permutation of
+    [0, num_pages); table entries past a sequence's last page are -1; page slots at or past
+    the sequence length are filled with NaN so that any read of them shows up in the output.
+    """
+    name: str
+    B: int
+    Nq: int
+    Hq: int
+    Hkv: int
+    D: int
+    dtype: int
+    len_lo: int
+    len_hi: int
+    causal: bool = True
+    softcap: float = 0.0
+    seed: int = 1
+    max_pages: int | None = None
+    fixed_lens: list | None = None
+    scale: float | None = None
+    extra_pages: int = 0
+    permute: bool = True
+    _cache: dict = field(default_factory=dict, repr=False)
+
+    def scale_f32(self) -> float:
+        s = self.scale if self.scale is not None else 1.0 / np.sqrt(self.D)
+        return float(np.float32(s))
+
+    def seq_lens(self) -> np.ndarray:
+        if self.fixed_lens is not None:
+            return np.asarray(self.fixed_lens, dtype=np.int32)
+        return uniform_ints(self.seed, STREAM_LENS, self.B, self.len_lo, self.len_hi).astype(np.int32)
+
+    def max_pages_per_seq(self) -> int:
+        if self.max_pages is not None:
+            return self.max_pages
+        return max(1, -(-self.len_hi // PAGE_SIZE))
+
+    def layout(self):
+        """(seq_lens, block_table, num_pages)."""
+        lens = self.seq_lens()
+        npg = [-(-int(L) // PAGE_SIZE) for L in lens]
+        num_pages = int(sum(npg)) + self.extra_pages
+        if self.permute:
+            perm = permutation(self.seed, STREAM_PERM, num_pages)
+        else:
+            perm = np.arange(num_pages, dtype=np.int64)
+        mp = self.max_pages_per_seq()
+        table = np.full((self.B, mp), -1, dtype=np.int32)
+        off = 0
+        for b in range(self.B):
+            table[b, :npg[b]] = perm[off:off + npg[b]]
+            off += npg[b]
+        return lens, table, max(num_pages, 1)
+
+    def tensors(self):
+        """(q, k_pages, v_pages, block_table, seq_lens) with q/k/v as uint16 bit patterns."""
+        lens, table, num_pages = self.layout()
+        q = normal_bits(self.seed, STREAM_Q, (self.B, self.Hq, self.Nq, self.D), self.dtype)
+        shape = (num_pages, PAGE_SIZE, self.Hkv, self.D)
+        k = normal_bits(self.seed, STREAM_K, shape, self.dtype)
+        v = normal_bits(self.seed, STREAM_V, shape, self.dtype)
+        nan = np.uint16(NAN_BITS[self.dtype])
+        used = np.zeros(num_pages, dtype=bool)
+        for b in range(self.B):
+            L = int(lens[b])
+            n = -(-L // PAGE_SIZE)
+            used[table[b, :n]] = True
+            if L % PAGE_SIZE:
+                last = table[b, n - 1]
+                k[last, L % PAGE_SIZE:] = nan
+                v[last, L % PAGE_SIZE:] = nan
+        k[~used] = nan
+        v[~used] = nan
+        return q, k, v, table, lens

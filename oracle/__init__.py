@@ -1,0 +1,158 @@
+"""fp64 CPU oracle for exact scaled-dot-product attention.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path imports this package: only the tests,
+the smoke check and the bench's CPU-baseline / reference arm may call it. It shares no code
+with the CUDA library and never reads anything the CUDA path produced.
+
+What it computes is the plain definition that the tiled online-softmax forward reaches exactly
+(up to rounding order): for every query row an explicit score vector over all keys, a
+visibility mask, a softmax and a weighted sum of value rows, all in fp64.
+
+Sources (web pages, cited by title and section):
+  * "mlx-bun 0.4.0 -> 1.0.0, src/model/flash-attention.ts" (diffend): the file header states
+    the forward is FlashAttention-2 that never materialises the [.,L,L] score matrix; its
+    forward shader defines the score as scale * q.k, the key-to-head map kv_head = head / reps,
+    and the saved statistic m + log(l); its manualSdpa helper is a materialised
+    matmul -> mask -> softmax -> matmul reference with GQA by grouping.
+  * "mlx-mfa 2.5.2" (pypi.org), Features and Usage: sliding window as a (left, right) tuple
+    with -1 meaning unbounded, native GQA without repeating K/V, tanh softcap (softcap=50.0),
+    paged KV with a block_table, two-phase split-KV decode for N_q <= 4.
+  * "mxflashattn 1.4.0 -> 1.5.0" (diffend), README: paged decode reads a paged KV cache with
+    page size 16 and GQA 4.
+
+Readings where the pages are silent or ambiguous (each restated in the design doc):
+  * window: key j is visible from absolute query position a iff a - win_l <= j <= a + win_r
+    (inclusive; -1 = unbounded on that side), ANDed with causality when both are given;
+  * causal with Nq != Nk is bottom-right aligned: query i sits at absolute position
+    a = i + (Nk - Nq);
+  * softcap: s <- cap * tanh(s / cap) applied to the scaled score before masking/softmax,
+    disabled when cap <= 0; the LSE uses the capped scores;
+  * LSE is the natural log-sum-exp of the final visible scores;
+  * a row with no visible key has output 0 and LSE = -inf;
+  * GQA groups are contiguous: query head h uses kv head h // (Hq // Hkv).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = ["visible", "attention", "attention_rows", "paged_gather", "decode"]
+
+
+def visible(Nq: int, Nk: int, causal: bool, win_l: int = -1, win_r: int = -1) -> np.ndarray:
+    """Boolean [Nq, Nk]: may query row i attend to key j.
+
+    Causal masking (mlx-bun forward shader masks keys after the query; mlx-mfa 2.5.2 Features,
+    "Causal tile-skip") is aligned bottom-right; the window tuple follows mlx-mfa 2.5.2 Usage,
+    window_size=(left, right) with -1 unbounded.
+    """
+    i = np.arange(Nq, dtype=np.int64)[:, None]
+    j = np.arange(Nk, dtype=np.int64)[None, :]
+    a = i + (Nk - Nq)
+    vis = np.ones((Nq, Nk), dtype=bool)
+    if causal:
+        vis &= j <= a
+    if win_l >= 0:
+        vis &= j >= a - win_l
+    if win_r >= 0:
+        vis &= j <= a + win_r
+    return vis
+
+
+def _rows_for_head(qh, kh, vh, vis_rows, scale, softcap):
+    """Attention for a block of query rows of one head.
+
+    qh [r, D], kh/vh [Nk, D] fp64; vis_rows [r, Nk] bool. Returns (o [r, D], lse [r]).
+    """
+    s = (qh @ kh.T) * float(scale)                      # scaled scores (mlx-bun forward shader)
+    if softcap > 0.0:                                   # mlx-mfa 2.5.2 Features: tanh softcap
+        s = float(softcap) * np.tanh(s / float(softcap))
+    s = np.where(vis_rows, s, -np.inf)
+    has = vis_rows.any(axis=1)
+    m = np.where(has, s.max(axis=1, initial=-np.inf), 0.0)
+    w = np.exp(s - m[:, None])                          # exp(-inf) = 0 for masked keys
+    l = w.sum(axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        o = np.where(has[:, None], (w @ vh) / np.where(has, l, 1.0)[:, None], 0.0)
+        lse = np.where(has, m + np.log(np.where(has, l, 1.0)), -np.inf)
+    return o, lse
+
+
+def attention(q, k, v, scale, causal=False, win_l=-1, win_r=-1, softcap=0.0, row_block=512):
+    """Full forward. q [B,Hq,Nq,D], k/v [B,Hkv,Nk,D] (fp64). Returns (o [B,Hq,Nq,D], lse [B,Hq,Nq])."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, Hq, Nq, D = q.shape
+    _, Hkv, Nk, _ = k.shape
+    assert Hq % Hkv == 0, "Hkv must divide Hq"
+    G = Hq // Hkv
+    vis = visible(Nq, Nk, causal, win_l, win_r)
+    o = np.zeros((B, Hq, Nq, D))
+    lse = np.full((B, Hq, Nq), -np.inf)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G                                   # mlx-bun forward shader: kv_head = head / reps
+            for r0 in range(0, Nq, row_block):
+                r1 = min(Nq, r0 + row_block)
+                o[b, h, r0:r1], lse[b, h, r0:r1] = _rows_for_head(
+                    q[b, h, r0:r1], k[b, g], v[b, g], vis[r0:r1], scale, softcap)
+    return o, lse
+
+
+def attention_rows(q, k, v, rows, scale, causal=False, win_l=-1, win_r=-1, softcap=0.0):
+    """Selected rows only. rows: int array [n, 3] of (b, h, i). Returns (o [n, D], lse [n])."""
+    q = np.asarray(q)
+    B, Hq, Nq, D = q.shape
+    _, Hkv, Nk, _ = k.shape
+    G = Hq // Hkv
+    rows = np.asarray(rows, dtype=np.int64).reshape(-1, 3)
+    o = np.zeros((len(rows), D))
+    lse = np.full(len(rows), -np.inf)
+    j = np.arange(Nk, dtype=np.int64)
+    for n, (b, h, i) in enumerate(rows):
+        g = h // G
+        a = i + (Nk - Nq)
+        vis = np.ones(Nk, dtype=bool)
+        if causal:
+            vis &= j <= a
+        if win_l >= 0:
+            vis &= j >= a - win_l
+        if win_r >= 0:
+            vis &= j <= a + win_r
+        qi = np.asarray(q[b, h, i:i + 1], dtype=np.float64)
+        oi, li = _rows_for_head(qi, np.asarray(k[b, g], dtype=np.float64),
+                                np.asarray(v[b, g], dtype=np.float64), vis[None, :], scale, softcap)
+        o[n], lse[n] = oi[0], li[0]
+    return o, lse
+
+
+def paged_gather(k_pages, v_pages, block_table, seq_len: int, b: int, page_size: int = 16):
+    """Logical K/V of sequence b: token t lives in page block_table[b][t // page_size], slot
+    t % page_size (mlx-mfa 2.5.2 Features, "Paged KV ... with block_table"; page size 16 as in
+    the mxflashattn 1.5.0 README). Pages are [num_pages, page_size, Hkv, D]. Returns [Hkv, len, D]."""
+    t = np.arange(int(seq_len), dtype=np.int64)
+    pages = np.asarray(block_table[b], dtype=np.int64)[t // page_size]
+    slots = t % page_size
+    kb = np.asarray(k_pages[pages, slots], dtype=np.float64)   # [len, Hkv, D]
+    vb = np.asarray(v_pages[pages, slots], dtype=np.float64)
+    return kb.transpose(1, 0, 2), vb.transpose(1, 0, 2)
+
+
+def decode(q, k_pages, v_pages, block_table, seq_lens, scale, causal=True, softcap=0.0,
+           page_size: int = 16):
+    """Decode over a paged cache: each sequence is gathered, then the dense definition applies
+    with Nk = len_b (query t of Nq sits at position len_b - Nq + t). Split-KV is a schedule of the
+    same sum (mlx-mfa 2.5.2 Features, "Flash Decode -- two-phase split-KV"), so the oracle does
+    not split. q [B,Hq,Nq,D]. Returns (o [B,Hq,Nq,D], lse [B,Hq,Nq])."""
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, Nq, D = q.shape
+    o = np.zeros((B, Hq, Nq, D))
+    lse = np.full((B, Hq, Nq), -np.inf)
+    for b in range(B):
+        L = int(seq_lens[b])
+        if L == 0:
+            continue
+        kb, vb = paged_gather(k_pages, v_pages, block_table, L, b, page_size)
+        ob, lb = attention(q[b:b + 1], kb[None], vb[None], scale, causal=causal, softcap=softcap)
+        o[b], lse[b] = ob[0], lb[0]
+    return o, lse

@@ -1,0 +1,296 @@
+"""Pins for the fp64 oracle, independent of the oracle's own code.
+
+Each check below uses something other than the oracle's arithmetic: torch's fp64 SDPA with a
+mask built from torch's band routines, closed forms (Q = 0 gives LSE = ln(#visible keys)),
+hand-computed two-key cases, and the invariants of exact attention (one visible key, identical
+value rows, key permutation, GQA == MHA on repeated heads, cap -> infinity). A dropped scale,
+a wrong mask index or sign, log2 instead of ln, or h % G instead of h // G fails at least one.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+rng = np.random.default_rng(7)
+
+
+def band_mask_torch(Nq, Nk, causal, win_l, win_r):
+    """Visibility built from torch.tril / torch.triu diagonals (bottom-right alignment:
+    query i sits at i + Nk - Nq)."""
+    off = Nk - Nq
+    m = torch.ones(Nq, Nk, dtype=torch.bool)
+    if causal:
+        m &= torch.tril(torch.ones(Nq, Nk, dtype=torch.bool), diagonal=off)
+    if win_r >= 0:
+        m &= torch.tril(torch.ones(Nq, Nk, dtype=torch.bool), diagonal=off + win_r)
+    if win_l >= 0:
+        m &= torch.triu(torch.ones(Nq, Nk, dtype=torch.bool), diagonal=off - win_l)
+    return m
+
+
+def sdpa_ref(q, k, v, scale, mask):
+    G = q.shape[1] // k.shape[1]
+    kt = torch.from_numpy(k).repeat_interleave(G, dim=1)
+    vt = torch.from_numpy(v).repeat_interleave(G, dim=1)
+    return torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), kt, vt, attn_mask=mask, scale=scale).numpy()
+
+
+CASES = [
+    # B, Hq, Hkv, Nq, Nk, D, causal, win_l, win_r
+    (2, 4, 2, 37, 53, 16, False, -1, -1),
+    (2, 4, 2, 37, 53, 16, True, -1, -1),
+    (1, 6, 3, 40, 40, 8, True, 5, -1),
+    (1, 4, 4, 33, 33, 8, False, 3, 2),
+    (1, 4, 1, 20, 64, 8, True, 11, 0),
+    (1, 2, 2, 64, 29, 8, False, 7, 7),
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_output_matches_torch_sdpa(case):
+    B, Hq, Hkv, Nq, Nk, D, causal, wl, wr = case
+    q = rng.standard_normal((B, Hq, Nq, D))
+    k = rng.standard_normal((B, Hkv, Nk, D))
+    v = rng.standard_normal((B, Hkv, Nk, D))
+    scale = 0.37
+    o, lse = oracle.attention(q, k, v, scale, causal, wl, wr)
+    mask = band_mask_torch(Nq, Nk, causal, wl, wr)
+    has = mask.any(dim=1).numpy()
+    ref = sdpa_ref(q, k, v, scale, mask)
+    np.testing.assert_allclose(o[:, :, has], ref[:, :, has], rtol=0, atol=1e-12)
+    assert np.all(o[:, :, ~has] == 0.0)
+    assert np.all(np.isneginf(lse[:, :, ~has]))
+    assert np.all(np.isfinite(lse[:, :, has]))
+
+
+def closed_form_count(Nq, Nk, causal, wl, wr):
+    """Number of visible keys for each row, written as interval arithmetic."""
+    out = []
+    for i in range(Nq):
+        a = i + Nk - Nq
+        lo = 0 if wl < 0 else max(0, a - wl)
+        hi = Nk - 1
+        if causal:
+            hi = min(hi, a)
+        if wr >= 0:
+            hi = min(hi, a + wr)
+        out.append(max(0, hi - lo + 1))
+    return np.array(out)
+
+
+@pytest.mark.parametrize("case", CASES + [(1, 2, 2, 300, 300, 4, True, 128, 0)])
+def test_zero_query_lse_is_log_count(case):
+    """Q = 0: every visible score is 0, so LSE = ln(#visible) and O = mean of visible V rows."""
+    B, Hq, Hkv, Nq, Nk, D, causal, wl, wr = case
+    q = np.zeros((B, Hq, Nq, D))
+    k = rng.standard_normal((B, Hkv, Nk, D))
+    v = rng.standard_normal((B, Hkv, Nk, D))
+    o, lse = oracle.attention(q, k, v, 0.5, causal, wl, wr, softcap=3.0)
+    cnt = closed_form_count(Nq, Nk, causal, wl, wr)
+    G = Hq // Hkv
+    csum = np.concatenate([np.zeros((B, Hkv, 1, D)), np.cumsum(v, axis=2)], axis=2)
+    for i in range(Nq):
+        if cnt[i] == 0:
+            assert np.all(np.isneginf(lse[:, :, i]))
+            continue
+        np.testing.assert_allclose(lse[:, :, i], math.log(cnt[i]), rtol=0, atol=1e-13)
+        a = i + Nk - Nq
+        lo = 0 if wl < 0 else max(0, a - wl)
+        mean = (csum[:, :, lo + cnt[i]] - csum[:, :, lo]) / cnt[i]
+        for h in range(Hq):
+            np.testing.assert_allclose(o[:, h, i], mean[:, h // G], rtol=0, atol=1e-12)
+
+
+def test_sliding_window_512_closed_form():
+    """Causal + window (512, 0): LSE_i = ln(min(i + 1, 513)) when Q = 0."""
+    N = 1100
+    q = np.zeros((1, 1, N, 2))
+    k = rng.standard_normal((1, 1, N, 2))
+    v = rng.standard_normal((1, 1, N, 2))
+    _, lse = oracle.attention(q, k, v, 0.1, True, 512, 0)
+    want = np.log(np.minimum(np.arange(N) + 1, 513))
+    np.testing.assert_allclose(lse[0, 0], want, rtol=0, atol=1e-13)
+
+
+def test_one_visible_key_gives_its_value_row_and_score():
+    """Window (0, 0), non-causal, Nq = Nk: row i sees key i only."""
+    N, D = 9, 4
+    q = rng.integers(-3, 4, (1, 2, N, D)).astype(float)
+    k = rng.integers(-3, 4, (1, 2, N, D)).astype(float)
+    v = rng.standard_normal((1, 2, N, D))
+    for cap in (0.0, 2.5):
+        o, lse = oracle.attention(q, k, v, 0.5, False, 0, 0, softcap=cap)
+        np.testing.assert_array_equal(o, v)
+        for h in range(2):
+            for i in range(N):
+                s = 0.5 * sum(q[0, h, i, d] * k[0, h, i, d] for d in range(D))
+                if cap > 0:
+                    s = cap * math.tanh(s / cap)
+                assert lse[0, h, i] == pytest.approx(s, abs=1e-14)
+
+
+def test_causal_row_zero_equals_first_value_row():
+    q = rng.standard_normal((1, 3, 16, 8))
+    k = rng.standard_normal((1, 3, 16, 8))
+    v = rng.standard_normal((1, 3, 16, 8))
+    o, lse = oracle.attention(q, k, v, 0.3, True)
+    np.testing.assert_allclose(o[0, :, 0], v[0, :, 0], rtol=0, atol=1e-15)
+    for h in range(3):
+        assert lse[0, h, 0] == pytest.approx(0.3 * float(q[0, h, 0] @ k[0, h, 0]), abs=1e-13)
+
+
+def test_identical_value_rows():
+    v = np.tile(rng.standard_normal((1, 2, 1, 8)), (1, 1, 30, 1))
+    q = rng.standard_normal((1, 4, 30, 8)) * 3
+    k = rng.standard_normal((1, 2, 30, 8)) * 3
+    o, _ = oracle.attention(q, k, v, 0.7, True, 6, -1, softcap=5.0)
+    for h in range(4):
+        np.testing.assert_allclose(o[0, h], np.broadcast_to(v[0, h // 2, 0], (30, 8)), rtol=0, atol=1e-12)
+
+
+def test_two_key_hand_case():
+    """q = (1, 0), k0 = (2, 0), k1 = (0, 1), scale 1: weights e^2/(e^2+1) and 1/(e^2+1)."""
+    q = np.array([[[[1.0, 0.0]]]])
+    k = np.array([[[[2.0, 0.0], [0.0, 1.0]]]])
+    v = np.array([[[[1.0, -1.0], [3.0, 5.0]]]])
+    o, lse = oracle.attention(q, k, v, 1.0)
+    w0 = math.exp(2) / (math.exp(2) + 1)
+    w1 = 1 / (math.exp(2) + 1)
+    assert o[0, 0, 0, 0] == pytest.approx(w0 * 1 + w1 * 3, abs=1e-15)
+    assert o[0, 0, 0, 1] == pytest.approx(-w0 + 5 * w1, abs=1e-15)
+    assert lse[0, 0, 0] == pytest.approx(math.log(math.exp(2) + 1), abs=1e-15)
+    # with softcap 1: scores become tanh(2) and tanh(0) = 0
+    o, lse = oracle.attention(q, k, v, 1.0, softcap=1.0)
+    t = math.tanh(2.0)
+    assert lse[0, 0, 0] == pytest.approx(math.log(math.exp(t) + 1), abs=1e-15)
+    assert o[0, 0, 0, 0] == pytest.approx((math.exp(t) * 1 + 3) / (math.exp(t) + 1), abs=1e-15)
+
+
+def test_key_permutation_invariance_unmasked():
+    q = rng.standard_normal((1, 2, 11, 8))
+    k = rng.standard_normal((1, 2, 23, 8))
+    v = rng.standard_normal((1, 2, 23, 8))
+    p = rng.permutation(23)
+    o1, l1 = oracle.attention(q, k, v, 0.4)
+    o2, l2 = oracle.attention(q, k[:, :, p], v[:, :, p], 0.4)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-13)
+
+
+def test_gqa_equals_mha_on_repeated_heads():
+    q = rng.standard_normal((2, 8, 19, 8))
+    k = rng.standard_normal((2, 2, 19, 8))
+    v = rng.standard_normal((2, 2, 19, 8))
+    o1, l1 = oracle.attention(q, k, v, 0.3, True, 4, -1, softcap=2.0)
+    o2, l2 = oracle.attention(q, np.repeat(k, 4, axis=1), np.repeat(v, 4, axis=1), 0.3, True, 4, -1,
+                              softcap=2.0)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+
+
+def test_softcap_limits():
+    q = rng.standard_normal((1, 2, 17, 8)) * 4
+    k = rng.standard_normal((1, 2, 17, 8)) * 4
+    v = rng.standard_normal((1, 2, 17, 8))
+    o0, l0 = oracle.attention(q, k, v, 0.5, True)
+    o1, l1 = oracle.attention(q, k, v, 0.5, True, softcap=1e9)  # s - cap*tanh(s/cap) ~ s^3/(3 cap^2)
+    np.testing.assert_allclose(o1, o0, rtol=0, atol=1e-9)
+    np.testing.assert_allclose(l1, l0, rtol=0, atol=1e-9)
+    # with a tiny cap every score is squeezed into (-cap, cap): LSE <= cap + ln(#visible)
+    _, l2 = oracle.attention(q, k, v, 0.5, True, softcap=0.25)
+    n = np.arange(1, 18)
+    assert np.all(l2[0] <= 0.25 + np.log(n)[None, :] + 1e-12)
+    assert np.all(l2[0] >= -0.25 + np.log(n)[None, :] - 1e-12)
+
+
+def test_window_special_cases():
+    q = rng.standard_normal((1, 2, 25, 8))
+    k = rng.standard_normal((1, 2, 25, 8))
+    v = rng.standard_normal((1, 2, 25, 8))
+    full = oracle.attention(q, k, v, 0.3, False)
+    unb = oracle.attention(q, k, v, 0.3, False, -1, -1)
+    np.testing.assert_array_equal(full[0], unb[0])
+    causal = oracle.attention(q, k, v, 0.3, True)
+    wide = oracle.attention(q, k, v, 0.3, False, 25, 0)
+    np.testing.assert_array_equal(causal[0], wide[0])
+    np.testing.assert_array_equal(causal[1], wide[1])
+
+
+def test_empty_rows_when_queries_precede_all_keys():
+    """Bottom-right causal with Nq > Nk: the first Nq - Nk rows see no key."""
+    q = rng.standard_normal((1, 1, 6, 4))
+    k = rng.standard_normal((1, 1, 4, 4))
+    v = rng.standard_normal((1, 1, 4, 4))
+    o, lse = oracle.attention(q, k, v, 1.0, True)
+    assert np.all(o[0, 0, :2] == 0) and np.all(np.isneginf(lse[0, 0, :2]))
+    np.testing.assert_allclose(o[0, 0, 2], v[0, 0, 0], atol=1e-15)
+
+
+def test_rows_helper_matches_full():
+    q = rng.standard_normal((2, 4, 30, 8))
+    k = rng.standard_normal((2, 2, 41, 8))
+    v = rng.standard_normal((2, 2, 41, 8))
+    o, lse = oracle.attention(q, k, v, 0.2, True, 9, 3, softcap=4.0)
+    rows = np.array([[0, 0, 0], [1, 3, 29], [0, 2, 17], [1, 1, 5]])
+    o2, l2 = oracle.attention_rows(q, k, v, rows, 0.2, True, 9, 3, softcap=4.0)
+    for n, (b, h, i) in enumerate(rows):
+        np.testing.assert_allclose(o2[n], o[b, h, i], rtol=0, atol=1e-14)
+        assert l2[n] == pytest.approx(lse[b, h, i], abs=1e-14)
+
+
+def _paged_from_contiguous(kc, vc, lens, page=16, perm_seed=3):
+    """Scatter contiguous [B, Hkv, N, D] caches into a permuted page pool."""
+    B, Hkv, N, D = kc.shape
+    npg = [-(-L // page) for L in lens]
+    total = sum(npg)
+    perm = np.random.default_rng(perm_seed).permutation(total)
+    kp = np.full((total, page, Hkv, D), np.nan)
+    vp = np.full((total, page, Hkv, D), np.nan)
+    table = np.full((B, max(npg) + 2), -1, dtype=np.int64)
+    off = 0
+    for b in range(B):
+        for p in range(npg[b]):
+            pid = perm[off + p]
+            table[b, p] = pid
+            for s in range(page):
+                t = p * page + s
+                if t < lens[b]:
+                    kp[pid, s] = kc[b, :, t]
+                    vp[pid, s] = vc[b, :, t]
+        off += npg[b]
+    return kp, vp, table
+
+
+@pytest.mark.parametrize("Nq", [1, 3, 4])
+def test_decode_gather_matches_sdpa_on_contiguous_cache(Nq):
+    B, Hq, Hkv, D = 3, 8, 2, 8
+    lens = [37, 16, 70]
+    N = max(lens)
+    kc = rng.standard_normal((B, Hkv, N, D))
+    vc = rng.standard_normal((B, Hkv, N, D))
+    q = rng.standard_normal((B, Hq, Nq, D))
+    kp, vp, table = _paged_from_contiguous(kc, vc, lens)
+    o, lse = oracle.decode(q, kp, vp, table, lens, 0.3, causal=True)
+    for b in range(B):
+        L = lens[b]
+        mask = band_mask_torch(Nq, L, True, -1, -1)
+        ref = sdpa_ref(q[b:b + 1], kc[b:b + 1, :, :L], vc[b:b + 1, :, :L], 0.3, mask)
+        np.testing.assert_allclose(o[b], ref[0], rtol=0, atol=1e-12)
+    assert np.all(np.isfinite(o))
+
+
+def test_decode_page_permutation_and_empty_sequence():
+    B, Hq, Hkv, D = 2, 4, 2, 8
+    lens = [50, 0]
+    kc = rng.standard_normal((B, Hkv, 50, D))
+    vc = rng.standard_normal((B, Hkv, 50, D))
+    q = rng.standard_normal((B, Hq, 1, D))
+    a = oracle.decode(q, *_paged_from_contiguous(kc, vc, [50, 1], perm_seed=1), [50, 0], 0.3)
+    b = oracle.decode(q, *_paged_from_contiguous(kc, vc, [50, 1], perm_seed=2), [50, 0], 0.3)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+    assert np.all(a[0][1] == 0) and np.all(np.isneginf(a[1][1]))
