@@ -1,0 +1,186 @@
+/*
+ * mfa.h -- C ABI of libmfa.so: exact tiled scaled-dot-product attention on B200 (sm_100a).
+ *
+ * Two operations:
+ *   mfa_fwd            dense forward with online softmax: causal and sliding-window tile skip,
+ *                      native GQA, optional tanh softcap, optional fp32 log-sum-exp output.
+ *   mfa_decode_splitkv two-phase split-KV decode (N_q <= 4) over a paged KV cache.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [MLXBUN]  "mlx-bun 0.4.0 -> 1.0.0, src/model/flash-attention.ts" (diffend): forward shader
+ *             (online softmax over K/V tiles, fp32 accumulation, saved m + log(l), kv_head =
+ *             head / reps) and flashForward (q [B,Hq,Tq,D], k/v [B,Hkv,Tkv,D], o like q,
+ *             log-sum-exp [B,Hq,Tq] fp32).
+ *   [MFA252]  "mlx-mfa 2.5.2" (pypi.org): Features (causal tile-skip, window_size=(left,right)
+ *             tile-skip, native GQA, tanh softcap, Flash Decode two-phase split-KV for N_q <= 4,
+ *             paged KV with block_table), Usage (window (512,-1), softcap=50.0), Supported
+ *             Configurations ([B,H,N,D] row-major, float16 / bfloat16).
+ *   [MXFA15]  "mxflashattn 1.4.0 -> 1.5.0" (diffend), README: split-KV paged decode reading a
+ *             paged KV cache, page_size 16, GQA 4; per-split (m, l) slots merged by a combine
+ *             step; explicit errors instead of silent fallbacks.
+ *   [MFA261]  "mlx-mfa 2.61.0" (PyPI package metadata): raw entry points carry the same guards
+ *             as the wrappers (contiguity, paged capacity, zero-KV, GQA geometry).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers to contiguous row-major buffers owned by the
+ *     caller. The library allocates nothing per call, never synchronises, and launches only on
+ *     the stream it is given (a cudaStream_t passed as void*; NULL = legacy default stream).
+ *   - Every tensor pointer must be 16-byte aligned.
+ *   - Malformed arguments are rejected BEFORE any launch with a negative status; nothing is
+ *     written then. There is no fallback path: an unsupported case is an error, never a slower
+ *     or approximate answer.
+ *   - Kernels bound every internal wait; a wait that runs out, or an out-of-range block_table
+ *     entry, records a device status that mfa_device_status() returns.
+ */
+#ifndef MFA_H_
+#define MFA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element types of q, k, v, out (and of the page pools). */
+#define MFA_DTYPE_FP16 0
+#define MFA_DTYPE_BF16 1
+
+/* Status codes. */
+#define MFA_OK                       0
+#define MFA_ERR_NULL_POINTER        -1   /* a required pointer is NULL */
+#define MFA_ERR_MISALIGNED          -2   /* a tensor pointer is not 16-byte aligned */
+#define MFA_ERR_BAD_DTYPE           -3   /* dtype not MFA_DTYPE_FP16 / MFA_DTYPE_BF16 */
+#define MFA_ERR_BAD_HEAD_DIM        -4   /* D not in {64, 128} */
+#define MFA_ERR_BAD_SHAPE           -5   /* negative size, or a size whose element count overflows */
+#define MFA_ERR_GQA_GEOMETRY        -6   /* Hkv < 1 or Hq not a multiple of Hkv */
+#define MFA_ERR_BAD_WINDOW          -7   /* window bound below -1 */
+#define MFA_ERR_BAD_SOFTCAP         -8   /* softcap negative or not finite */
+#define MFA_ERR_BAD_SCALE           -9   /* scale not finite or not > 0 */
+#define MFA_ERR_NQ_TOO_LARGE       -10   /* decode with N_q > 4 */
+#define MFA_ERR_PAGE_SIZE          -11   /* page_size != 16 */
+#define MFA_ERR_WORKSPACE          -12   /* workspace NULL, misaligned or smaller than required */
+#define MFA_ERR_UNSUPPORTED        -13   /* decode with (Hq / Hkv) * N_q > 16 query rows per kv head */
+#define MFA_ERR_CUDA               -20   /* a CUDA runtime/driver call or a launch failed */
+#define MFA_ERR_DEVICE_TIMEOUT     -21   /* device status: a bounded wait inside a kernel ran out */
+#define MFA_ERR_DEVICE_BAD_PAGE    -22   /* device status: a block_table entry was outside [0, num_pages) */
+
+/*
+ * mfa_fwd -- exact attention forward (prefill).
+ *
+ * Computes, for every batch b, query head h, query row i:
+ *   g      = h / (Hq / Hkv)                          (contiguous GQA groups [MLXBUN] kv_head = head / reps)
+ *   a      = i + (Nk - Nq)                           (bottom-right alignment of the query rows)
+ *   vis(j) = (!causal || j <= a) && (win_l < 0 || j >= a - win_l) && (win_r < 0 || j <= a + win_r)
+ *   s_j    = scale * <q[b,h,i,:], k[b,g,j,:]>;  if softcap > 0: s_j = softcap * tanh(s_j / softcap)
+ *   out[b,h,i,:] = sum_{vis j} exp(s_j - m) v[b,g,j,:] / sum_{vis j} exp(s_j - m),  m = max_{vis j} s_j
+ *   lse[b,h,i]   = m + ln(sum_{vis j} exp(s_j - m))
+ * without materialising the score matrix ([MLXBUN] forward shader; [MFA252] Features). A row
+ * with no visible key gets out = 0 and lse = -inf. Key tiles that no row of a block can see are
+ * never loaded (causal and window tile skip, [MFA252] Features).
+ *
+ * Arguments
+ *   q    [B, Hq,  Nq, D]  dtype        k, v [B, Hkv, Nk, D]  dtype       (read only)
+ *   out  [B, Hq,  Nq, D]  dtype        lse  [B, Hq, Nq] float32, or NULL to skip it
+ *   D in {64, 128}; Hq % Hkv == 0; win_l, win_r >= -1 (-1 = unbounded on that side);
+ *   causal != 0 enables the causal predicate; softcap == 0 disables the cap;
+ *   scale: the caller's float, used as given (typically 1/sqrt(D)).
+ *   Sizes of 0 for B, Hq or Nq are a no-op; Nk == 0 gives out = 0, lse = -inf.
+ * Returns MFA_OK after the launch was queued, or a negative status (nothing launched).
+ */
+int mfa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+            int B, int Hq, int Hkv, int Nq, int Nk, int D, float scale,
+            int causal, int win_l, int win_r, float softcap, int dtype, void* stream);
+
+/*
+ * mfa_decode_workspace_size -- bytes of scratch mfa_decode_splitkv needs for this shape.
+ * The split plan is a function of these arguments only (not of seq_lens), so one workspace
+ * serves every call with the same shape. Returns 0 for invalid arguments.
+ */
+size_t mfa_decode_workspace_size(int B, int Nq, int Hq, int Hkv, int D,
+                                 int max_pages_per_seq, int page_size);
+
+/*
+ * mfa_decode_splitkv -- two-phase split-KV decode over a paged KV cache
+ * ([MFA252] Features "Flash Decode -- two-phase split-KV for N_q <= 4" and "Paged KV";
+ *  [MXFA15] README: paged decode with per-split (m, l) slots and a combine step).
+ *
+ * Sequence b holds seq_lens[b] tokens; its token t is stored in page block_table[b][t / 16],
+ * slot t % 16. Query token t (of Nq) sits at position seq_lens[b] - Nq + t; with causal != 0 it
+ * sees keys at positions <= its own. Phase 1 splits each sequence into runs of pages and
+ * computes, per run, unnormalised partial outputs with their running max and sum; phase 2
+ * merges the runs with max-rescaling. The result equals mfa_fwd's definition on the gathered
+ * K/V (up to fp32 rounding order).
+ *
+ * Arguments
+ *   q            [B, Hq, Nq, D] dtype, Nq in [1, 4]          (device)
+ *   k_pages      [num_pages, 16, Hkv, D] dtype                (device)
+ *   v_pages      [num_pages, 16, Hkv, D] dtype                (device)
+ *   block_table  int32 [B, max_pages_per_seq]; entries for pages t < ceil(len/16) must lie in
+ *                [0, num_pages); later entries are never read    (device)
+ *   seq_lens     int32 [B], each in [0, max_pages_per_seq * 16]  (device)
+ *   out          [B, Hq, Nq, D] dtype; lse float32 [B, Hq, Nq] or NULL   (device)
+ *   page_size must be 16; (Hq / Hkv) * Nq <= 16; D in {64, 128};
+ *   workspace: device scratch of at least mfa_decode_workspace_size(...) bytes, 256-byte
+ *   aligned, owned by the caller; its contents need no initialisation and are overwritten.
+ * Page slots at or past a sequence's length are never used in the arithmetic, so they may hold
+ * any bit pattern (NaN included). Returns MFA_OK after both launches were queued.
+ */
+int mfa_decode_splitkv(const void* q, const void* k_pages, const void* v_pages,
+                       const int32_t* block_table, const int32_t* seq_lens,
+                       void* out, float* lse,
+                       int B, int Nq, int Hq, int Hkv, int D, int page_size,
+                       int max_pages_per_seq, int num_pages,
+                       float scale, int causal, float softcap, int dtype,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* Human-readable text for a status code (static storage). */
+const char* mfa_status_string(int code);
+
+/*
+ * Launch record of the last successful call on this host thread: which kernel ran and with
+ * what schedule ([MXFA15] README keeps a per-dispatch record; this is the same idea).
+ */
+typedef struct mfa_launch_info {
+    int kernel;                 /* 1 = prefill forward, 2 = decode phase 1 + combine, 3 = empty-key fill */
+    int grid_x, grid_y, grid_z; /* grid of the main kernel */
+    int block_threads;          /* threads per CTA of the main kernel */
+    int smem_bytes;             /* dynamic shared memory per CTA of the main kernel */
+    int tile_m, tile_n;         /* prefill: query rows per Q tile, keys per K/V tile */
+    int q_tiles_per_cta;        /* prefill: Q tiles per CTA */
+    int pages_per_split;        /* decode: pages per split */
+    int max_splits;             /* decode: splits per sequence at max_pages_per_seq */
+    int kv_heads_per_cta;       /* decode: kv heads handled by one CTA */
+} mfa_launch_info;
+
+int mfa_last_launch_info(mfa_launch_info* info);
+
+/*
+ * Device status: copies the kernels' status word to *code (MFA_OK or MFA_ERR_DEVICE_*) and
+ * *detail (where it happened), then clears it. Synchronises `stream`. For tests and debugging.
+ */
+int mfa_device_status(void* stream, int* code, int* detail);
+
+/*
+ * Debug switches (process-wide; default 0). Bit 0: the forward visits every key tile and masks
+ * element-wise instead of skipping tiles. Bit 1: count the key tiles each forward CTA visits
+ * into a device counter read by mfa_debug_tiles_visited. Returns the previous flags.
+ */
+#define MFA_DEBUG_NO_TILE_SKIP 1
+#define MFA_DEBUG_COUNT_TILES  2
+int mfa_debug_set_flags(int flags);
+
+/* Reads and resets the tile counter (synchronises `stream`). */
+int mfa_debug_tiles_visited(void* stream, unsigned long long* count);
+
+/*
+ * Decode split size override in pages (0 = automatic). It changes the split plan, and with it
+ * mfa_decode_workspace_size. Returns the previous value.
+ */
+int mfa_debug_set_decode_split_pages(int pages);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MFA_H_ */

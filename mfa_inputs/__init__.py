@@ -226,3 +226,27 @@ class DecodeCase:
         k[~used] = nan
         v[~used] = nan
         return q, k, v, table, lens
+
+
+def workloads():
+    """The named full-size workloads (shapes, flags, seeds and value scales)."""
+    return {
+        "causal_b1_h2_n128_d64_fp16": PrefillCase(
+            "causal_b1_h2_n128_d64_fp16", 1, 2, 2, 128, 128, 64, FP16, True, seed=1001),
+        "causal_b2_h8_n4096_d128_fp16": PrefillCase(
+            "causal_b2_h8_n4096_d128_fp16", 2, 8, 8, 4096, 4096, 128, FP16, True, seed=1002),
+        "noncausal_b2_h8_n4096_d128_fp16": PrefillCase(
+            "noncausal_b2_h8_n4096_d128_fp16", 2, 8, 8, 4096, 4096, 128, FP16, False, seed=1002),
+        "window512_b2_h8_n8192_d128_fp16": PrefillCase(
+            "window512_b2_h8_n8192_d128_fp16", 2, 8, 8, 8192, 8192, 128, FP16, True, 512, 0,
+            seed=1003),
+        "window256_b2_h8_n8192_d128_fp16": PrefillCase(
+            "window256_b2_h8_n8192_d128_fp16", 2, 8, 8, 8192, 8192, 128, FP16, True, 256, 0,
+            seed=1003),
+        "gqa_causal_b1_hq32_hkv8_n16384_d128_bf16_cap50": PrefillCase(
+            "gqa_causal_b1_hq32_hkv8_n16384_d128_bf16_cap50", 1, 32, 8, 16384, 16384, 128, BF16,
+            True, softcap=50.0, mul=0.5, seed=1004),
+        "decode_b8_hq32_hkv8_d128_bf16_len8k_128k": DecodeCase(
+            "decode_b8_hq32_hkv8_d128_bf16_len8k_128k", 8, 1, 32, 8, 128, BF16, 8192, 131072,
+            seed=1005),
+    }

@@ -35,7 +35,7 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["visible", "attention", "attention_rows", "paged_gather", "decode"]
+__all__ = ["visible", "attention", "attention_rows", "paged_gather", "decode", "decode_rows"]
 
 
 def visible(Nq: int, Nk: int, causal: bool, win_l: int = -1, win_r: int = -1) -> np.ndarray:
@@ -155,4 +155,37 @@ def decode(q, k_pages, v_pages, block_table, seq_lens, scale, causal=True, softc
         kb, vb = paged_gather(k_pages, v_pages, block_table, L, b, page_size)
         ob, lb = attention(q[b:b + 1], kb[None], vb[None], scale, causal=causal, softcap=softcap)
         o[b], lse[b] = ob[0], lb[0]
+    return o, lse
+
+
+def decode_rows(q, k_pages, v_pages, block_table, seq_lens, rows, scale, causal=True,
+                softcap=0.0, page_size: int = 16, to_f64=None):
+    """Decode outputs for selected rows only, gathering just the kv head each row needs.
+
+    rows: int array [n, 3] of (b, h, t). to_f64 converts a gathered slice of the pools to fp64
+    (default: numpy conversion). Returns (o [n, D], lse [n])."""
+    conv = to_f64 if to_f64 is not None else (lambda a: np.asarray(a, dtype=np.float64))
+    B, Hq, Nq, D = np.asarray(q).shape
+    Hkv = k_pages.shape[2]
+    G = Hq // Hkv
+    rows = np.asarray(rows, dtype=np.int64).reshape(-1, 3)
+    o = np.zeros((len(rows), D))
+    lse = np.full(len(rows), -np.inf)
+    for n, (b, h, t) in enumerate(rows):
+        L = int(seq_lens[b])
+        if L == 0:
+            continue
+        g = h // G
+        tok = np.arange(L, dtype=np.int64)
+        pages = np.asarray(block_table[b], dtype=np.int64)[tok // page_size]
+        slots = tok % page_size
+        kb = conv(k_pages[pages, slots, g])           # [L, D]
+        vb = conv(v_pages[pages, slots, g])
+        a = L - Nq + t                               # position of query token t
+        vis = np.ones(L, dtype=bool)
+        if causal:
+            vis &= tok <= a
+        qi = conv(np.asarray(q)[b, h, t:t + 1])
+        oi, li = _rows_for_head(qi, kb, vb, vis[None, :], scale, softcap)
+        o[n], lse[n] = oi[0], li[0]
     return o, lse

@@ -1,0 +1,121 @@
+"""The C-ABI boundary without a GPU: the library loads, exports every symbol include/mfa.h
+declares, and rejects malformed arguments before touching the device.
+
+Pointers passed here are fake (aligned integers) and every call has exactly one thing wrong,
+so each returns its status during validation; no call reaches a CUDA API.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import tiled_exact_attention_mfa_b200 as mfa
+from conftest import gpu_available
+
+# The rejection tests hand fake addresses to the library; they only run where no GPU is
+# reachable, so that a mistake in a case can never turn into a launch on bad pointers.
+no_device = pytest.mark.skipif(gpu_available(), reason="fake pointers are used only without a GPU")
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mfa.h")
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(mfa_\w+)\s*\(", text, flags=re.M)))
+
+
+def header_defines():
+    return dict(re.findall(r"#define\s+(MFA_\w+)\s+(-?\d+)", open(HEADER).read()))
+
+
+def test_every_declared_symbol_is_exported():
+    names = header_functions()
+    assert "mfa_fwd" in names and "mfa_decode_splitkv" in names
+    lib = ctypes.CDLL(mfa.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(mfa.EXPORTED)
+
+
+def test_status_strings_cover_codes():
+    d = header_defines()
+    codes = [int(v) for k, v in d.items() if k.startswith("MFA_ERR_") or k == "MFA_OK"]
+    for c in codes:
+        assert mfa.mfa_status_string(c) != "unknown status", c
+    assert mfa.mfa_status_string(12345) == "unknown status"
+    assert int(d["MFA_DTYPE_BF16"]) == mfa.MFA_DTYPE_BF16
+
+
+A = 0x10000  # fake, 16-byte aligned device addresses (never dereferenced)
+
+
+def fwd(**kw):
+    args = dict(q=A, k=A, v=A, out=A, lse=A, B=2, Hq=8, Hkv=2, Nq=64, Nk=64, D=128, scale=0.125,
+                causal=1, win_l=-1, win_r=-1, softcap=0.0, dtype=1, stream=None)
+    args.update(kw)
+    return mfa.lib.mfa_fwd(*args.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=2), -3), (dict(D=96), -4), (dict(D=256), -4), (dict(B=-1), -5), (dict(Nk=-3), -5),
+    (dict(Hkv=3), -6), (dict(Hkv=0), -6), (dict(win_l=-2), -7), (dict(win_r=-5), -7),
+    (dict(softcap=-1.0), -8), (dict(softcap=float("inf")), -8), (dict(softcap=float("nan")), -8),
+    (dict(scale=0.0), -9), (dict(scale=float("nan")), -9), (dict(scale=-0.1), -9),
+    (dict(q=None), -1), (dict(out=None), -1), (dict(k=None), -1),
+    (dict(q=A + 8), -2), (dict(v=A + 4), -2), (dict(lse=A + 2), -2),
+])
+@no_device
+def test_fwd_rejects_malformed(kw, code):
+    assert fwd(**kw) == code
+
+
+@no_device
+def test_fwd_empty_problem_is_noop():
+    # nothing to compute: OK without any launch, even with NULL pointers
+    assert fwd(B=0, q=None, k=None, v=None, out=None) == 0
+    assert fwd(Nq=0, q=None, k=None, v=None, out=None) == 0
+
+
+def dec(**kw):
+    ws = kw.pop("ws_bytes", 1 << 30)
+    args = dict(q=A, k=A, v=A, table=A, lens=A, out=A, lse=A, B=8, Nq=1, Hq=32, Hkv=8, D=128,
+                page=16, max_pages=8192, num_pages=40000, scale=0.088, causal=1, softcap=0.0,
+                dtype=1, ws=A, ws_bytes=ws, stream=None)
+    args.update(kw)
+    return mfa.lib.mfa_decode_splitkv(*args.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=5), -3), (dict(D=80), -4), (dict(Nq=5), -10), (dict(Nq=0), -5), (dict(Hkv=5), -6),
+    (dict(page=32), -11), (dict(max_pages=0), -5), (dict(num_pages=0), -5),
+    (dict(Hq=64, Hkv=2), -13), (dict(Nq=3, Hq=64, Hkv=8), -13), (dict(softcap=-2.0), -8),
+    (dict(scale=float("inf")), -9), (dict(table=None), -1), (dict(lens=None), -1),
+    (dict(k=A + 2), -2), (dict(table=A + 4), -2), (dict(ws=None), -12), (dict(ws=A + 16), -12),
+    (dict(ws_bytes=1024), -12),
+])
+@no_device
+def test_decode_rejects_malformed(kw, code):
+    assert dec(**kw) == code
+
+
+def test_decode_workspace_size_is_shape_only():
+    n = mfa.mfa_decode_workspace_size(8, 1, 32, 8, 128, 8192)
+    # 8 sequences x 256 splits of 32 pages x 32 rows x (128 + 2) floats
+    assert n == 8 * 256 * 32 * 128 * 4 + 8 * 256 * 32 * 2 * 4
+    assert mfa.mfa_decode_workspace_size(8, 5, 32, 8, 128, 8192) == 0
+    assert mfa.mfa_decode_workspace_size(8, 1, 32, 8, 128, 8192, 8) == 0
+    # small grids get smaller splits (more CTAs): 1 sequence of 64 pages -> 4-page splits
+    assert mfa.mfa_decode_workspace_size(1, 1, 32, 8, 128, 64) == 16 * 32 * 128 * 4 + 16 * 32 * 2 * 4
+    old = mfa.mfa_debug_set_decode_split_pages(8)
+    try:
+        assert mfa.mfa_decode_workspace_size(1, 1, 32, 8, 128, 64) == 8 * 32 * 128 * 4 + 8 * 32 * 2 * 4
+    finally:
+        mfa.mfa_debug_set_decode_split_pages(old)
+
+
+def test_debug_flags_roundtrip():
+    old = mfa.mfa_debug_set_flags(3)
+    assert mfa.mfa_debug_set_flags(old) == 3

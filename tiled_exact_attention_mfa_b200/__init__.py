@@ -1,0 +1,195 @@
+"""Python binding of libmfa.so: exact tiled attention (prefill + paged split-KV decode) on B200.
+
+Argument marshalling only: every step of the computation runs in the CUDA kernels behind the C
+ABI declared in include/mfa.h. PyTorch provides device memory and the stream. There is no CPU
+or library fallback: importing this package fails if libmfa.so has not been built, and every
+call raises if the library rejects its arguments.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmfa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it first (python -m tiled_exact_attention_mfa_b200.build "
+        "or __graft_entry__.build()). There is no fallback implementation.")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+MFA_DTYPE_FP16 = 0
+MFA_DTYPE_BF16 = 1
+MFA_DEBUG_NO_TILE_SKIP = 1
+MFA_DEBUG_COUNT_TILES = 2
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+
+lib.mfa_fwd.restype = _i
+lib.mfa_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _i, _f, _i, _vp]
+lib.mfa_decode_workspace_size.restype = ctypes.c_size_t
+lib.mfa_decode_workspace_size.argtypes = [_i] * 7
+lib.mfa_decode_splitkv.restype = _i
+lib.mfa_decode_splitkv.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
+                                   _f, _i, _f, _i, _vp, ctypes.c_size_t, _vp]
+lib.mfa_status_string.restype = ctypes.c_char_p
+lib.mfa_status_string.argtypes = [_i]
+
+
+class LaunchInfo(ctypes.Structure):
+    _fields_ = [(n, _i) for n in (
+        "kernel", "grid_x", "grid_y", "grid_z", "block_threads", "smem_bytes", "tile_m", "tile_n",
+        "q_tiles_per_cta", "pages_per_split", "max_splits", "kv_heads_per_cta")]
+
+    def as_dict(self):
+        return {n: getattr(self, n) for n, _ in self._fields_}
+
+
+lib.mfa_last_launch_info.restype = _i
+lib.mfa_last_launch_info.argtypes = [ctypes.POINTER(LaunchInfo)]
+lib.mfa_device_status.restype = _i
+lib.mfa_device_status.argtypes = [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i)]
+lib.mfa_debug_set_flags.restype = _i
+lib.mfa_debug_set_flags.argtypes = [_i]
+lib.mfa_debug_tiles_visited.restype = _i
+lib.mfa_debug_tiles_visited.argtypes = [_vp, ctypes.POINTER(ctypes.c_ulonglong)]
+lib.mfa_debug_set_decode_split_pages.restype = _i
+lib.mfa_debug_set_decode_split_pages.argtypes = [_i]
+
+EXPORTED = ("mfa_fwd", "mfa_decode_workspace_size", "mfa_decode_splitkv", "mfa_status_string",
+            "mfa_last_launch_info", "mfa_device_status", "mfa_debug_set_flags",
+            "mfa_debug_tiles_visited", "mfa_debug_set_decode_split_pages")
+
+
+class MFAError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {mfa_status_string(code)} (status {code})")
+
+
+def mfa_status_string(code: int) -> str:
+    return lib.mfa_status_string(code).decode()
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise MFAError(rc, where)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float16:
+        return MFA_DTYPE_FP16
+    if t.dtype == torch.bfloat16:
+        return MFA_DTYPE_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; use float16 or bfloat16")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def mfa_fwd(q, k, v, out=None, lse=None, *, scale=None, causal=False, window=(-1, -1),
+            softcap=0.0, return_lse=True, stream=None):
+    """Attention forward. q [B,Hq,Nq,D], k/v [B,Hkv,Nk,D]; returns (out, lse or None)."""
+    torch = _torch()
+    B, Hq, Nq, D = q.shape
+    _, Hkv, Nk, _ = k.shape
+    if k.shape != v.shape or k.shape[0] != B or k.shape[3] != D:
+        raise ValueError("k and v must be [B, Hkv, Nk, D] matching q")
+    if q.dtype != k.dtype or q.dtype != v.dtype:
+        raise TypeError("q, k and v must share one dtype")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    wl, wr = window
+    rc = lib.mfa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Nq, Nk, D,
+                     float(scale), int(bool(causal)), int(wl), int(wr), float(softcap),
+                     _dtype_code(q), _stream(stream))
+    _check(rc, "mfa_fwd")
+    return out, lse
+
+
+def mfa_decode_workspace_size(B, Nq, Hq, Hkv, D, max_pages_per_seq, page_size=16) -> int:
+    return int(lib.mfa_decode_workspace_size(B, Nq, Hq, Hkv, D, max_pages_per_seq, page_size))
+
+
+def mfa_decode_splitkv(q, k_pages, v_pages, block_table, seq_lens, out=None, lse=None, *,
+                       scale=None, causal=True, softcap=0.0, workspace=None, return_lse=True,
+                       stream=None):
+    """Paged split-KV decode. q [B,Hq,Nq,D]; pages [num_pages,16,Hkv,D]; block_table int32
+    [B,max_pages]; seq_lens int32 [B]. Returns (out, lse or None)."""
+    torch = _torch()
+    B, Hq, Nq, D = q.shape
+    num_pages, page, Hkv, _ = k_pages.shape
+    max_pages = block_table.shape[1]
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("block_table and seq_lens must be int32")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    need = mfa_decode_workspace_size(B, Nq, Hq, Hkv, D, max_pages, page)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    rc = lib.mfa_decode_splitkv(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
+                                _ptr(seq_lens), _ptr(out), _ptr(lse), B, Nq, Hq, Hkv, D, page,
+                                max_pages, num_pages, float(scale), int(bool(causal)),
+                                float(softcap), _dtype_code(q), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "mfa_decode_splitkv")
+    return out, lse
+
+
+def mfa_last_launch_info() -> dict:
+    info = LaunchInfo()
+    _check(lib.mfa_last_launch_info(ctypes.byref(info)), "mfa_last_launch_info")
+    return info.as_dict()
+
+
+def mfa_device_status(stream=None):
+    code, detail = _i(0), _i(0)
+    _check(lib.mfa_device_status(_stream(stream), ctypes.byref(code), ctypes.byref(detail)),
+           "mfa_device_status")
+    return code.value, detail.value
+
+
+def mfa_debug_set_flags(flags: int) -> int:
+    return lib.mfa_debug_set_flags(flags)
+
+
+def mfa_debug_tiles_visited(stream=None) -> int:
+    n = ctypes.c_ulonglong(0)
+    _check(lib.mfa_debug_tiles_visited(_stream(stream), ctypes.byref(n)), "mfa_debug_tiles_visited")
+    return n.value
+
+
+def mfa_debug_set_decode_split_pages(pages: int) -> int:
+    return lib.mfa_debug_set_decode_split_pages(pages)

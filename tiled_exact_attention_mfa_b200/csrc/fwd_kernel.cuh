@@ -1,0 +1,416 @@
+// fwd_kernel.cuh -- exact attention forward (prefill) for sm_100a.
+//
+// Algorithm: FlashAttention-2 style single pass over K/V tiles with an online softmax (running
+// row max m, running sum l, fp32 accumulator O), as in the forward shader of "mlx-bun 0.4.0 ->
+// 1.0.0, src/model/flash-attention.ts": S = scale * Q K^T per tile, m_new = max(m, rowmax(S)),
+// alpha = exp(m - m_new), P = exp(S - m_new), l = alpha l + rowsum(P), O = alpha O + P V, and at
+// the end O / l and LSE = m + ln l. A tile whose every score of a row is masked leaves that
+// row untouched (the shader's m_new = -inf guard).
+//
+// B200 mapping (one CTA per SM, 320 threads, 2 Q tiles of 128 rows per CTA):
+//   warp 8      TMA producer: Q tiles once, then K and V tiles through 2-stage rings (128-byte
+//               swizzled smem, 3-D tensor maps so tails are zero-filled per head).
+//   warp 9      TMEM owner and single-thread tcgen05.mma issuer:
+//                 S_t = Q_t K^T   (M=128, N=128, K=D; A and B K-major from smem)
+//                 O_t += P_t V    (M=128, N=D, K=128; P_t from TMEM, V MN-major from smem)
+//   warps 0-3   softmax for Q tile 0, warps 4-7 for Q tile 1: one TMEM lane = one query row =
+//               one thread, so row max / row sum are thread-local. Scores are kept in the log2
+//               domain (scale * log2 e folded into one FFMA). The running max is only moved when
+//               it grows by more than 2^8 (rescaling is exact for any reference max; a stale one
+//               only bounds P by 2^8), and then O is rescaled in TMEM by the owning warp.
+//   TMEM columns: S_0 [0,128) S_1 [128,256) O_0 [256,256+D) O_1 [256+D, 256+2D);
+//                 P_t (16-bit, 2 per column) overwrites the first 64 columns of S_t.
+// Ordering: QK for tile j+1 of Q tile t is issued only after PV for tile j of Q tile t has
+// completed (its P lives in S_t's columns), so when the softmax of tile j+1 starts, the previous
+// PV is done and O_t can be rescaled in place.
+//
+// Tile skip ("mlx-mfa 2.5.2", Features: causal tile-skip, window_size=(left,right) tile skip):
+// each CTA visits only key tiles that intersect the union of its rows' visible ranges; inside,
+// masking is applied per element only on tiles that are not fully visible to all 128 rows.
+#pragma once
+#include "sm100.cuh"
+
+namespace mfa {
+
+constexpr int kFwdBM = 128;       // query rows per Q tile (= TMEM lanes)
+constexpr int kFwdBN = 128;       // keys per K/V tile
+constexpr int kFwdQT = 2;         // Q tiles per CTA
+constexpr int kFwdStages = 2;     // K ring and V ring depth
+constexpr int kFwdThreads = 320;  // 8 softmax warps + producer + MMA
+constexpr float kRescaleLog2 = 8.0f;
+
+struct FwdParams {
+  CUtensorMap tm_q;  // [B*Hq][Nq][D]
+  CUtensorMap tm_k;  // [B*Hkv][Nk][D]
+  CUtensorMap tm_v;
+  void* out;
+  float* lse;
+  unsigned long long* tile_counter;
+  int B, Hq, Hkv, Nq, Nk, G;
+  int causal, win_l, win_r;
+  int n_qblk;       // number of 256-row query blocks per head
+  int flags;        // bit 0: no tile skip; bit 1: count tiles
+  float c_log2;     // factor taking the stored score to the log2 domain
+  float softcap;    // 0 = off
+  float cap_in;     // scale / softcap
+  float lse_mul;    // ln 2
+};
+
+template <int D>
+struct FwdSmem {
+  static constexpr int kTileBytes = kFwdBM * D * 2;  // one 128 x D tile of 16-bit values
+  static constexpr int kSlabBytes = 128 * 128;       // 128 rows x 64 columns (128 B) slab
+  uint8_t q[kFwdQT][kTileBytes];
+  uint8_t k[kFwdStages][kTileBytes];
+  uint8_t v[kFwdStages][kTileBytes];
+  uint64_t bar_q;
+  uint64_t bar_k_full[kFwdStages], bar_k_empty[kFwdStages];
+  uint64_t bar_v_full[kFwdStages], bar_v_empty[kFwdStages];
+  uint64_t bar_s_full[kFwdQT], bar_p_full[kFwdQT], bar_o_done[kFwdQT];
+  uint64_t bar_final;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int D>
+constexpr int fwd_smem_bytes() {
+  return (int)sizeof(FwdSmem<D>) + 1024;  // + alignment slack for the 1024-byte swizzle atoms
+}
+
+// Visible key range [lo, hi) of absolute query positions [a0, a1] (inclusive).
+__device__ __forceinline__ void key_range(const FwdParams& p, int a0, int a1, int& lo, int& hi) {
+  lo = 0;
+  hi = p.Nk;
+  if (p.causal) hi = min(hi, a1 + 1);
+  if (p.win_r >= 0) hi = min(hi, a1 + p.win_r + 1);
+  if (p.win_l >= 0) lo = max(lo, a0 - p.win_l);
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_constant__ FwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  FwdSmem<D>& sm = *reinterpret_cast<FwdSmem<D>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: heavy query blocks first (causal blocks near the end see the most keys)
+  const int BH = p.B * p.Hq;
+  const int qb = p.n_qblk - 1 - (int)(blockIdx.x / BH);
+  const int bh = blockIdx.x % BH;
+  const int b = bh / p.Hq;
+  const int h = bh % p.Hq;
+  const int g = h / p.G;
+  const int q0 = qb * (kFwdBM * kFwdQT);
+  const int off = p.Nk - p.Nq;
+  const int q_last = min(q0 + kFwdBM * kFwdQT, p.Nq) - 1;
+
+  int lo, hi;
+  key_range(p, q0 + off, q_last + off, lo, hi);
+  if (p.flags & 1) {
+    lo = 0;
+    hi = p.Nk;
+  }
+  const int kt_lo = lo / kFwdBN;
+  const int n_tiles = (hi > lo) ? ((hi + kFwdBN - 1) / kFwdBN - kt_lo) : 0;
+
+  // ---- setup
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&sm.bar_q), 1);
+    for (int s = 0; s < kFwdStages; ++s) {
+      mbar_init(smem_u32(&sm.bar_k_full[s]), 1);
+      mbar_init(smem_u32(&sm.bar_k_empty[s]), 1);
+      mbar_init(smem_u32(&sm.bar_v_full[s]), 1);
+      mbar_init(smem_u32(&sm.bar_v_empty[s]), 1);
+    }
+    for (int t = 0; t < kFwdQT; ++t) {
+      mbar_init(smem_u32(&sm.bar_s_full[t]), 1);
+      mbar_init(smem_u32(&sm.bar_p_full[t]), kFwdBM);
+      mbar_init(smem_u32(&sm.bar_o_done[t]), 1);
+    }
+    mbar_init(smem_u32(&sm.bar_final), 1);
+    sm.abort = 0;
+    fence_barrier_init();
+    if ((p.flags & 2) && n_tiles > 0) atomicAdd(p.tile_counter, (unsigned long long)n_tiles);
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(&sm.tmem_base), 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+
+  constexpr int kSlabs = D / 64;
+  constexpr uint32_t kTileBytes = FwdSmem<D>::kTileBytes;
+  constexpr int kSlab = FwdSmem<D>::kSlabBytes;
+
+  if (warp == 8) {
+    // ================================================================ TMA producer
+    if (lane == 0 && n_tiles > 0) {
+      const uint32_t bq = smem_u32(&sm.bar_q);
+      mbar_expect_tx(bq, kFwdQT * kTileBytes);
+      for (int t = 0; t < kFwdQT; ++t)
+        for (int sl = 0; sl < kSlabs; ++sl)
+          tma_load_3d(smem_u32(sm.q[t]) + sl * kSlab, &p.tm_q, bq, sl * 64, q0 + t * kFwdBM,
+                      b * p.Hq + h);
+      int issued_k[kFwdStages] = {0, 0}, issued_v[kFwdStages] = {0, 0};
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % kFwdStages;
+        const int use = j / kFwdStages;
+        const int row = (kt_lo + j) * kFwdBN;
+        if (use > 0 && !mbar_wait(smem_u32(&sm.bar_k_empty[s]), (use - 1) & 1, abort, 801)) break;
+        const uint32_t bk = smem_u32(&sm.bar_k_full[s]);
+        mbar_expect_tx(bk, kTileBytes);
+        for (int sl = 0; sl < kSlabs; ++sl)
+          tma_load_3d(smem_u32(sm.k[s]) + sl * kSlab, &p.tm_k, bk, sl * 64, row, b * p.Hkv + g);
+        issued_k[s] = use + 1;
+        if (use > 0 && !mbar_wait(smem_u32(&sm.bar_v_empty[s]), (use - 1) & 1, abort, 802)) break;
+        const uint32_t bv = smem_u32(&sm.bar_v_full[s]);
+        mbar_expect_tx(bv, kTileBytes);
+        for (int sl = 0; sl < kSlabs; ++sl)
+          tma_load_3d(smem_u32(sm.v[s]) + sl * kSlab, &p.tm_v, bv, sl * 64, row, b * p.Hkv + g);
+        issued_v[s] = use + 1;
+      }
+      // Make sure no copy into this CTA's shared memory is still in flight when it exits.
+      volatile int no_abort = 0;
+      mbar_wait(bq, 0, &no_abort, 803);
+      for (int s = 0; s < kFwdStages; ++s) {
+        if (issued_k[s] > 0) mbar_wait(smem_u32(&sm.bar_k_full[s]), (issued_k[s] - 1) & 1, &no_abort, 804);
+        if (issued_v[s] > 0) mbar_wait(smem_u32(&sm.bar_v_full[s]), (issued_v[s] - 1) & 1, &no_abort, 805);
+      }
+    }
+  } else if (warp == 9) {
+    // ================================================================ MMA issuer
+    if (lane == 0 && n_tiles > 0) {
+      const uint32_t idesc_qk = idesc_f16(BF16 ? 1 : 0, kFwdBM, kFwdBN, 0);
+      const uint32_t idesc_pv = idesc_f16(BF16 ? 1 : 0, kFwdBM, D, 1);
+      auto issue_qk = [&](int t, int s) {
+        const uint32_t qa = smem_u32(sm.q[t]);
+        const uint32_t ka = smem_u32(sm.k[s]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * kSlab + (kk & 3) * 32;
+          tc_mma_ss(tmem + t * kFwdBN, smem_desc_sw128(qa + koff, 16, 1024),
+                    smem_desc_sw128(ka + koff, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int s, bool acc) {
+        const uint32_t va = smem_u32(sm.v[s]);
+#pragma unroll
+        for (int kk = 0; kk < kFwdBN / 16; ++kk) {
+          tc_mma_ts(tmem + 256 + t * D, tmem + t * kFwdBN + kk * 8,
+                    smem_desc_sw128(va + kk * 16 * 128, kSlab, 1024), idesc_pv,
+                    (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(smem_u32(&sm.bar_q), 0, abort, 901);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int s = j % kFwdStages;
+        const uint32_t ph = (j / kFwdStages) & 1;
+        const int s1 = (j + 1) % kFwdStages;
+        const uint32_t ph1 = ((j + 1) / kFwdStages) & 1;
+        const bool more = j + 1 < n_tiles;
+        if (j == 0) {
+          if (!(ok = mbar_wait(smem_u32(&sm.bar_k_full[s]), ph, abort, 902))) break;
+          tc_fence_after();
+          issue_qk(0, s);
+          tc_commit(smem_u32(&sm.bar_s_full[0]));
+          issue_qk(1, s);
+          tc_commit(smem_u32(&sm.bar_s_full[1]));
+          tc_commit(smem_u32(&sm.bar_k_empty[s]));
+        }
+        // Q tile 0: PV(j), then QK(j+1) once PV(j) is done (P_0 lives in S_0's columns)
+        if (!(ok = mbar_wait(smem_u32(&sm.bar_v_full[s]), ph, abort, 903))) break;
+        if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[0]), j & 1, abort, 904))) break;
+        tc_fence_after();
+        issue_pv(0, s, j > 0);
+        tc_commit(smem_u32(&sm.bar_o_done[0]));
+        if (more) {
+          if (!(ok = mbar_wait(smem_u32(&sm.bar_k_full[s1]), ph1, abort, 905))) break;
+          if (!(ok = mbar_wait(smem_u32(&sm.bar_o_done[0]), j & 1, abort, 906))) break;
+          tc_fence_after();
+          issue_qk(0, s1);
+          tc_commit(smem_u32(&sm.bar_s_full[0]));
+        }
+        // Q tile 1
+        if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[1]), j & 1, abort, 907))) break;
+        tc_fence_after();
+        issue_pv(1, s, j > 0);
+        tc_commit(smem_u32(&sm.bar_o_done[1]));
+        tc_commit(smem_u32(&sm.bar_v_empty[s]));
+        if (more) {
+          if (!(ok = mbar_wait(smem_u32(&sm.bar_o_done[1]), j & 1, abort, 908))) break;
+          tc_fence_after();
+          issue_qk(1, s1);
+          tc_commit(smem_u32(&sm.bar_s_full[1]));
+          tc_commit(smem_u32(&sm.bar_k_empty[s1]));
+        }
+      }
+      // Drain: every MMA issued above has completed before TMEM is released.
+      tc_commit(smem_u32(&sm.bar_final));
+      volatile int no_abort = 0;
+      mbar_wait(smem_u32(&sm.bar_final), 0, &no_abort, 909);
+    }
+  } else {
+    // ================================================================ softmax warps
+    const int t = warp >> 2;                  // Q tile of this warpgroup
+    const int quarter = warp & 3;             // TMEM lane quarter of this warp
+    const int r = quarter * 32 + lane;        // row within the Q tile
+    const int row = q0 + t * kFwdBM + r;      // query row
+    const int a = row + off;                  // absolute position of the row
+    const int a_lo = q0 + t * kFwdBM + off;   // first / last absolute position of the Q tile
+    const int a_hi = a_lo + kFwdBM - 1;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const uint32_t t_s = tmem + lane_base + t * kFwdBN;
+    const uint32_t t_o = tmem + lane_base + 256 + t * D;
+    const float c = p.c_log2;
+    float m_run = -INFINITY;  // running max of the stored (scaled, capped) score
+    float l_run = 0.f;
+
+    for (int j = 0; j < n_tiles; ++j) {
+      const bool got = mbar_wait(smem_u32(&sm.bar_s_full[t]), j & 1, abort, 1001 + t);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      uint32_t sraw[128];
+      tmem_ld32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&sraw[0]));
+      tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sraw[32]));
+      tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&sraw[64]));
+      tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&sraw[96]));
+      tmem_wait_ld();
+      float* s = reinterpret_cast<float*>(sraw);
+
+      const int k0 = (kt_lo + j) * kFwdBN;
+      if (p.softcap > 0.f) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) s[i] = p.softcap * tanh_from_exp(s[i] * p.cap_in);
+      }
+      // Element masks only where some row of this Q tile may not see some key of the tile.
+      bool interior = (k0 + kFwdBN <= p.Nk);
+      if (p.causal) interior = interior && (k0 + kFwdBN - 1 <= a_lo);
+      if (p.win_r >= 0) interior = interior && (k0 + kFwdBN - 1 <= a_lo + p.win_r);
+      if (p.win_l >= 0) interior = interior && (k0 >= a_hi - p.win_l);
+      if (p.flags & 1) interior = false;
+      if (!interior) {
+        int jhi = p.Nk - k0;                                   // keys >= Nk
+        if (p.causal) jhi = min(jhi, a - k0 + 1);
+        if (p.win_r >= 0) jhi = min(jhi, a + p.win_r - k0 + 1);
+        const int jlo = (p.win_l >= 0) ? (a - p.win_l - k0) : -1;
+#pragma unroll
+        for (int i = 0; i < 128; ++i) s[i] = (i < jhi && i >= jlo) ? s[i] : -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+
+      // Lazy rescale: move the reference max only when it grew by more than 2^8 in exp2 terms.
+      const float m_new = fmaxf(m_run, mx);
+      const bool need = (m_new > -INFINITY) && (m_run == -INFINITY || (m_new - m_run) * c > kRescaleLog2);
+      float alpha = 1.f;
+      const bool warp_rescale = __any_sync(0xffffffffu, need);
+      if (warp_rescale) {
+        if (m_new > m_run) {
+          alpha = (m_run == -INFINITY) ? 0.f : fast_exp2((m_run - m_new) * c);
+          m_run = m_new;
+        }
+      }
+      const float neg_mc = (m_run == -INFINITY) ? 0.f : -m_run * c;
+      float sum = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const float p0 = fast_exp2(fmaf(s[2 * i], c, neg_mc));
+        const float p1 = fast_exp2(fmaf(s[2 * i + 1], c, neg_mc));
+        sum += p0 + p1;
+        pk[i] = pack2<BF16>(p0, p1);
+      }
+      l_run = l_run * alpha + sum;
+      tmem_st32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      // O rescale (only after the first tile: before it O holds nothing).
+      if (warp_rescale && j > 0) {
+#pragma unroll
+        for (int cb = 0; cb < D; cb += 32) {
+          uint32_t o[32];
+          tmem_ld32(t_o + cb, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(t_o + cb, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&sm.bar_p_full[t]));
+    }
+
+    // ---- epilogue: O / l, LSE
+    bool have_o = false;
+    if (n_tiles > 0 && !*abort) {
+      have_o = mbar_wait(smem_u32(&sm.bar_o_done[t]), (n_tiles - 1) & 1, abort, 1003 + t);
+      tc_fence_after();
+    }
+    have_o = __all_sync(0xffffffffu, have_o);
+    {
+    }
+    const bool valid = row < p.Nq;
+    const size_t obase = ((size_t)(b * p.Hq + h) * p.Nq + (size_t)row) * D;
+    const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+#pragma unroll
+    for (int cb = 0; cb < D; cb += 32) {
+      uint32_t o[32];
+      if (have_o) {
+        tmem_ld32(t_o + cb, o);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0u;
+      }
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + obase + cb);
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) {
+          uint4 w;
+          w.x = pack2<BF16>(__uint_as_float(o[v4 * 8 + 0]) * inv_l, __uint_as_float(o[v4 * 8 + 1]) * inv_l);
+          w.y = pack2<BF16>(__uint_as_float(o[v4 * 8 + 2]) * inv_l, __uint_as_float(o[v4 * 8 + 3]) * inv_l);
+          w.z = pack2<BF16>(__uint_as_float(o[v4 * 8 + 4]) * inv_l, __uint_as_float(o[v4 * 8 + 5]) * inv_l);
+          w.w = pack2<BF16>(__uint_as_float(o[v4 * 8 + 6]) * inv_l, __uint_as_float(o[v4 * 8 + 7]) * inv_l);
+          dst[v4] = w;
+        }
+      }
+    }
+    if (valid && p.lse != nullptr) {
+      p.lse[(size_t)(b * p.Hq + h) * p.Nq + row] =
+          (l_run > 0.f) ? (m_run * c + log2f(l_run)) * p.lse_mul : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Nk == 0: every row sees no key.
+template <bool BF16>
+__global__ void mfa_fill_empty_kernel(void* out, float* lse, size_t rows, int D) {
+  const size_t n = rows * (size_t)D;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    reinterpret_cast<uint16_t*>(out)[i] = 0;
+  if (lse)
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < rows; i += (size_t)gridDim.x * blockDim.x)
+      lse[i] = -INFINITY;
+}
+
+}  // namespace mfa

@@ -1,0 +1,399 @@
+// mfa_api.cu -- the C ABI of libmfa.so (declared in include/mfa.h): argument validation, the
+// split plan, TMA tensor maps and kernel launches. All kernels live in this translation unit so
+// that the device status word is one symbol.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "decode_kernel.cuh"
+#include "fwd_kernel.cuh"
+#include "mfa.h"
+
+namespace {
+
+thread_local mfa_launch_info g_last = {};
+int g_debug_flags = 0;
+int g_split_pages_override = 0;
+std::mutex g_mutex;
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
+// ------------------------------------------------------------------ driver entry point
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D map over a [rows_outer][n][D] 16-bit tensor, box 64 x 128 x 1, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int dtype, long long outer, long long n, int D) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)n, (cuuint64_t)outer};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)n * D * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dtype == MFA_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Opt a kernel into its dynamic shared memory size once per device.
+template <typename K>
+bool ensure_smem(K kernel, int bytes, bool (&done)[kMaxDevices]) {
+  int dev = current_device();
+  if (dev < 0) return false;
+  if (done[dev]) return true;
+  std::lock_guard<std::mutex> lk(g_mutex);
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+      return false;
+    done[dev] = true;
+  }
+  return true;
+}
+
+// ------------------------------------------------------------------ decode split plan
+struct DecodePlan {
+  int pages_per_split;
+  int max_splits;
+  int heads_per_cta;
+  int groups;
+};
+
+DecodePlan decode_plan(int B, int Hkv, int max_pages) {
+  DecodePlan pl;
+  pl.heads_per_cta = 1;
+  for (int h = 8; h >= 1; --h)
+    if (Hkv % h == 0) {
+      pl.heads_per_cta = h;
+      break;
+    }
+  pl.groups = Hkv / pl.heads_per_cta;
+  int s = 32;
+  if (g_split_pages_override > 0) {
+    s = g_split_pages_override > 32 ? 32 : g_split_pages_override;
+  } else {
+    // halve the split while the grid would hold fewer than two CTAs per SM (148 SMs)
+    while (s > 4 && (long long)B * ((max_pages + s - 1) / s) * pl.groups < 296) s /= 2;
+  }
+  pl.pages_per_split = s;
+  pl.max_splits = (max_pages + s - 1) / s;
+  return pl;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int check_sizes(long long a, long long b, long long c, long long d) {
+  // element counts must fit comfortably in 63 bits and TMA coordinates in 31 bits
+  if (a < 0 || b < 0 || c < 0 || d < 0) return MFA_ERR_BAD_SHAPE;
+  long double n = (long double)a * b * c * d;
+  if (n > 4.0e18L) return MFA_ERR_BAD_SHAPE;
+  return MFA_OK;
+}
+
+template <int D, bool BF16>
+int launch_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+               int Hkv, int Nq, int Nk, float scale, int causal, int win_l, int win_r,
+               float softcap, int dtype, cudaStream_t st) {
+  static bool smem_done[kMaxDevices] = {};
+  constexpr int smem = mfa::fwd_smem_bytes<D>();
+  auto kernel = mfa::mfa_fwd_kernel<D, BF16>;
+  if (!ensure_smem(kernel, smem, smem_done)) return MFA_ERR_CUDA;
+  mfa::FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (!make_map(&p.tm_q, q, dtype, (long long)B * Hq, Nq, D)) return MFA_ERR_CUDA;
+  if (!make_map(&p.tm_k, k, dtype, (long long)B * Hkv, Nk, D)) return MFA_ERR_CUDA;
+  if (!make_map(&p.tm_v, v, dtype, (long long)B * Hkv, Nk, D)) return MFA_ERR_CUDA;
+  p.out = out;
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.G = Hq / Hkv;
+  p.causal = causal ? 1 : 0;
+  p.win_l = win_l;
+  p.win_r = win_r;
+  const int rows_per_cta = mfa::kFwdBM * mfa::kFwdQT;
+  p.n_qblk = (Nq + rows_per_cta - 1) / rows_per_cta;
+  p.flags = g_debug_flags;
+  if (p.flags & MFA_DEBUG_COUNT_TILES) {
+    void* ctr = nullptr;
+    if (cudaGetSymbolAddress(&ctr, mfa::g_tile_counter) != cudaSuccess) return MFA_ERR_CUDA;
+    p.tile_counter = static_cast<unsigned long long*>(ctr);
+  }
+  const float log2e = 1.4426950408889634f;
+  if (softcap > 0.f) {
+    p.softcap = softcap;
+    p.cap_in = scale / softcap;
+    p.c_log2 = log2e;
+  } else {
+    p.softcap = 0.f;
+    p.cap_in = 0.f;
+    p.c_log2 = scale * log2e;
+  }
+  p.lse_mul = 0.69314718055994531f;
+  const long long grid = (long long)p.n_qblk * B * Hq;
+  if (grid > 0x7FFFFFFFLL) return MFA_ERR_BAD_SHAPE;
+  kernel<<<(unsigned)grid, mfa::kFwdThreads, smem, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
+  mfa_launch_info li = {};
+  li.kernel = 1;
+  li.grid_x = (int)grid;
+  li.grid_y = li.grid_z = 1;
+  li.block_threads = mfa::kFwdThreads;
+  li.smem_bytes = smem;
+  li.tile_m = mfa::kFwdBM;
+  li.tile_n = mfa::kFwdBN;
+  li.q_tiles_per_cta = mfa::kFwdQT;
+  g_last = li;
+  return MFA_OK;
+}
+
+template <int D, bool BF16>
+int launch_decode(const mfa::DecodeParams& p, const DecodePlan& pl, cudaStream_t st) {
+  static bool smem_done[kMaxDevices] = {};
+  const int smem = mfa::dec_smem_bytes<D>(pl.heads_per_cta);
+  // the largest plan (8 heads per CTA) sets the attribute for all
+  auto k1 = mfa::mfa_decode_phase1_kernel<D, BF16>;
+  if (!ensure_smem(k1, mfa::dec_smem_bytes<D>(8), smem_done)) return MFA_ERR_CUDA;
+  dim3 g1(pl.max_splits, p.B, pl.groups);
+  k1<<<g1, (pl.heads_per_cta + 1) * 32, smem, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
+  dim3 g2(p.Hq * p.Nq, p.B, 1);
+  mfa::mfa_decode_combine_kernel<D, BF16><<<g2, D, 0, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
+  mfa_launch_info li = {};
+  li.kernel = 2;
+  li.grid_x = g1.x;
+  li.grid_y = g1.y;
+  li.grid_z = g1.z;
+  li.block_threads = (pl.heads_per_cta + 1) * 32;
+  li.smem_bytes = smem;
+  li.pages_per_split = pl.pages_per_split;
+  li.max_splits = pl.max_splits;
+  li.kv_heads_per_cta = pl.heads_per_cta;
+  g_last = li;
+  return MFA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mfa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+            int Hkv, int Nq, int Nk, int D, float scale, int causal, int win_l, int win_r,
+            float softcap, int dtype, void* stream) {
+  if (dtype != MFA_DTYPE_FP16 && dtype != MFA_DTYPE_BF16) return MFA_ERR_BAD_DTYPE;
+  if (D != 64 && D != 128) return MFA_ERR_BAD_HEAD_DIM;
+  if (B < 0 || Hq < 0 || Nq < 0 || Nk < 0) return MFA_ERR_BAD_SHAPE;
+  if (Hkv < 1 || Hq % Hkv != 0) return MFA_ERR_GQA_GEOMETRY;
+  if (win_l < -1 || win_r < -1) return MFA_ERR_BAD_WINDOW;
+  if (!std::isfinite(softcap) || softcap < 0.f) return MFA_ERR_BAD_SOFTCAP;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return MFA_ERR_BAD_SCALE;
+  int rc;
+  if ((rc = check_sizes(B, Hq, Nq, D)) != MFA_OK) return rc;
+  if ((rc = check_sizes(B, Hkv, Nk, D)) != MFA_OK) return rc;
+  if ((long long)B * Hq > 0x7FFFFFFFLL || (long long)B * Hkv > 0x7FFFFFFFLL) return MFA_ERR_BAD_SHAPE;
+  if (B == 0 || Hq == 0 || Nq == 0) return MFA_OK;
+  if (!q || !out || (Nk > 0 && (!k || !v))) return MFA_ERR_NULL_POINTER;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(lse) || (Nk > 0 && (!aligned16(k) || !aligned16(v))))
+    return MFA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (Nk == 0) {
+    const size_t rows = (size_t)B * Hq * Nq;
+    if (dtype == MFA_DTYPE_BF16)
+      mfa::mfa_fill_empty_kernel<true><<<148, 256, 0, st>>>(out, lse, rows, D);
+    else
+      mfa::mfa_fill_empty_kernel<false><<<148, 256, 0, st>>>(out, lse, rows, D);
+    if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
+    mfa_launch_info li = {};
+    li.kernel = 3;
+    li.grid_x = 148;
+    li.grid_y = li.grid_z = 1;
+    li.block_threads = 256;
+    g_last = li;
+    return MFA_OK;
+  }
+  const bool bf = dtype == MFA_DTYPE_BF16;
+  if (D == 128)
+    return bf ? launch_fwd<128, true>(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, scale, causal, win_l, win_r, softcap, dtype, st)
+              : launch_fwd<128, false>(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, scale, causal, win_l, win_r, softcap, dtype, st);
+  return bf ? launch_fwd<64, true>(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, scale, causal, win_l, win_r, softcap, dtype, st)
+            : launch_fwd<64, false>(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, scale, causal, win_l, win_r, softcap, dtype, st);
+}
+
+static int validate_decode(int B, int Nq, int Hq, int Hkv, int D, int page_size, int max_pages) {
+  if (D != 64 && D != 128) return MFA_ERR_BAD_HEAD_DIM;
+  if (B < 0 || Hq < 0) return MFA_ERR_BAD_SHAPE;
+  if (Nq < 1 || Nq > 4) return Nq < 1 ? MFA_ERR_BAD_SHAPE : MFA_ERR_NQ_TOO_LARGE;
+  if (Hkv < 1 || Hq % Hkv != 0 || Hq < 1) return MFA_ERR_GQA_GEOMETRY;
+  if (page_size != mfa::kDecPage) return MFA_ERR_PAGE_SIZE;
+  if (max_pages < 1) return MFA_ERR_BAD_SHAPE;
+  if ((Hq / Hkv) * Nq > 16) return MFA_ERR_UNSUPPORTED;
+  if ((long long)max_pages * mfa::kDecPage > 0x7FFFFFFFLL) return MFA_ERR_BAD_SHAPE;
+  return MFA_OK;
+}
+
+size_t mfa_decode_workspace_size(int B, int Nq, int Hq, int Hkv, int D, int max_pages_per_seq,
+                                 int page_size) {
+  if (validate_decode(B, Nq, Hq, Hkv, D, page_size, max_pages_per_seq) != MFA_OK) return 0;
+  DecodePlan pl = decode_plan(B, Hkv, max_pages_per_seq);
+  const size_t rows = (size_t)B * pl.max_splits * Hq * Nq;
+  return align256(rows * D * sizeof(float)) + align256(rows * 2 * sizeof(float));
+}
+
+int mfa_decode_splitkv(const void* q, const void* k_pages, const void* v_pages,
+                       const int32_t* block_table, const int32_t* seq_lens, void* out, float* lse,
+                       int B, int Nq, int Hq, int Hkv, int D, int page_size, int max_pages_per_seq,
+                       int num_pages, float scale, int causal, float softcap, int dtype,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  if (dtype != MFA_DTYPE_FP16 && dtype != MFA_DTYPE_BF16) return MFA_ERR_BAD_DTYPE;
+  int rc = validate_decode(B, Nq, Hq, Hkv, D, page_size, max_pages_per_seq);
+  if (rc != MFA_OK) return rc;
+  if (num_pages < 1) return MFA_ERR_BAD_SHAPE;
+  if (!std::isfinite(softcap) || softcap < 0.f) return MFA_ERR_BAD_SOFTCAP;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return MFA_ERR_BAD_SCALE;
+  if ((rc = check_sizes(num_pages, page_size, Hkv, D)) != MFA_OK) return rc;
+  if ((rc = check_sizes(B, Hq, Nq, D)) != MFA_OK) return rc;
+  if (B == 0) return MFA_OK;
+  if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !out) return MFA_ERR_NULL_POINTER;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(block_table) ||
+      !aligned16(seq_lens) || !aligned16(out) || !aligned16(lse))
+    return MFA_ERR_MISALIGNED;
+  const size_t need = mfa_decode_workspace_size(B, Nq, Hq, Hkv, D, max_pages_per_seq, page_size);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
+    return MFA_ERR_WORKSPACE;
+  DecodePlan pl = decode_plan(B, Hkv, max_pages_per_seq);
+  mfa::DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = static_cast<const uint16_t*>(q);
+  p.k_pages = static_cast<const uint16_t*>(k_pages);
+  p.v_pages = static_cast<const uint16_t*>(v_pages);
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.out = out;
+  p.lse = lse;
+  const size_t rows = (size_t)B * pl.max_splits * Hq * Nq;
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(rows * D * sizeof(float)));
+  p.B = B;
+  p.Nq = Nq;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.max_pages = max_pages_per_seq;
+  p.num_pages = num_pages;
+  p.pages_per_split = pl.pages_per_split;
+  p.max_splits = pl.max_splits;
+  p.heads_per_cta = pl.heads_per_cta;
+  p.causal = causal ? 1 : 0;
+  const float log2e = 1.4426950408889634f;
+  if (softcap > 0.f) {
+    p.softcap = softcap;
+    p.cap_in = scale / softcap;
+    p.c_log2 = log2e;
+  } else {
+    p.c_log2 = scale * log2e;
+  }
+  if (pl.max_splits > 0x7FFFFFFF || B > 65535 || pl.groups > 65535) return MFA_ERR_BAD_SHAPE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool bf = dtype == MFA_DTYPE_BF16;
+  if (D == 128) return bf ? launch_decode<128, true>(p, pl, st) : launch_decode<128, false>(p, pl, st);
+  return bf ? launch_decode<64, true>(p, pl, st) : launch_decode<64, false>(p, pl, st);
+}
+
+const char* mfa_status_string(int code) {
+  switch (code) {
+    case MFA_OK: return "ok";
+    case MFA_ERR_NULL_POINTER: return "a required pointer is NULL";
+    case MFA_ERR_MISALIGNED: return "a tensor pointer is not 16-byte aligned";
+    case MFA_ERR_BAD_DTYPE: return "dtype must be MFA_DTYPE_FP16 or MFA_DTYPE_BF16";
+    case MFA_ERR_BAD_HEAD_DIM: return "head dim D must be 64 or 128";
+    case MFA_ERR_BAD_SHAPE: return "invalid or overflowing size";
+    case MFA_ERR_GQA_GEOMETRY: return "Hkv must be >= 1 and divide Hq";
+    case MFA_ERR_BAD_WINDOW: return "window bounds must be >= -1";
+    case MFA_ERR_BAD_SOFTCAP: return "softcap must be finite and >= 0";
+    case MFA_ERR_BAD_SCALE: return "scale must be finite and > 0";
+    case MFA_ERR_NQ_TOO_LARGE: return "split-KV decode takes at most 4 query tokens";
+    case MFA_ERR_PAGE_SIZE: return "page_size must be 16";
+    case MFA_ERR_WORKSPACE: return "workspace is NULL, not 256-byte aligned or too small";
+    case MFA_ERR_UNSUPPORTED: return "decode supports at most 16 query rows ((Hq/Hkv)*Nq) per kv head";
+    case MFA_ERR_CUDA: return "a CUDA call or kernel launch failed";
+    case MFA_ERR_DEVICE_TIMEOUT: return "device: a bounded wait inside a kernel ran out";
+    case MFA_ERR_DEVICE_BAD_PAGE: return "device: block_table or seq_lens entry out of range";
+    default: return "unknown status";
+  }
+}
+
+int mfa_last_launch_info(mfa_launch_info* info) {
+  if (!info) return MFA_ERR_NULL_POINTER;
+  *info = g_last;
+  return MFA_OK;
+}
+
+int mfa_device_status(void* stream, int* code, int* detail) {
+  if (!code || !detail) return MFA_ERR_NULL_POINTER;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int h[2] = {0, 0};
+  if (cudaMemcpyFromSymbolAsync(h, mfa::g_status, sizeof(h), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return MFA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MFA_ERR_CUDA;
+  int zero[2] = {0, 0};
+  if (cudaMemcpyToSymbolAsync(mfa::g_status, zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return MFA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MFA_ERR_CUDA;
+  *code = h[0];
+  *detail = h[1];
+  return MFA_OK;
+}
+
+int mfa_debug_set_flags(int flags) {
+  int old = g_debug_flags;
+  g_debug_flags = flags;
+  return old;
+}
+
+int mfa_debug_tiles_visited(void* stream, unsigned long long* count) {
+  if (!count) return MFA_ERR_NULL_POINTER;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned long long h = 0, zero = 0;
+  if (cudaMemcpyFromSymbolAsync(&h, mfa::g_tile_counter, sizeof(h), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return MFA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MFA_ERR_CUDA;
+  if (cudaMemcpyToSymbolAsync(mfa::g_tile_counter, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return MFA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MFA_ERR_CUDA;
+  *count = h;
+  return MFA_OK;
+}
+
+int mfa_debug_set_decode_split_pages(int pages) {
+  int old = g_split_pages_override;
+  g_split_pages_override = pages < 0 ? 0 : pages;
+  return old;
+}
+
+}  // extern "C"
