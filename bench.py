@@ -1,0 +1,443 @@
+"""Throughput of exact tiled attention on B200: prefill TFLOP/s and split-KV decode KV GB/s.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mfa|reference] [--workload NAME]
+
+One step = one pass of the hot path over one batch: the prefill forward of the named workload
+(default: causal, B=2, H=8, N=4096, D=128, fp16). The same JSON line also carries the other
+workloads (non-causal, sliding window, GQA + softcap prefill, paged split-KV decode), each timed
+the same way. Inputs are seeded synthetic tensors resident in HBM; L2 is flushed (a 256 MiB
+write) before every timed step, outside the timed kernel. Times are CUDA events on the launching
+stream; with N > 1 (torchrun) every rank runs its own copy of the workload (weak scaling) and the
+max over ranks is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import mfa_inputs as mi  # noqa: E402
+
+MAIN = "causal_b2_h8_n4096_d128_fp16"
+METRIC = "attention TFLOP/s (prefill) and KV GB/s (split-KV decode) vs B200 peak"
+NOMINAL_TFLOPS = 2250.0
+NOMINAL_GBS = 8000.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+# --------------------------------------------------------------------------- work accounting
+def visible_pairs(case) -> int:
+    """Visible (query, key) pairs of one head, summed row by row from the interval form."""
+    i = np.arange(case.Nq, dtype=np.int64)
+    a = i + (case.Nk - case.Nq)
+    lo = np.zeros_like(a) if case.win_l < 0 else np.maximum(0, a - case.win_l)
+    hi = np.full_like(a, case.Nk - 1)
+    if case.causal:
+        hi = np.minimum(hi, a)
+    if case.win_r >= 0:
+        hi = np.minimum(hi, a + case.win_r)
+    return int(np.maximum(0, hi - lo + 1).sum())
+
+
+def prefill_flops(case) -> float:
+    return 4.0 * case.D * case.B * case.Hq * visible_pairs(case)
+
+
+def prefill_bytes(case) -> float:
+    e = 2
+    return (e * case.B * case.Hq * case.Nq * case.D * 2 + e * 2 * case.B * case.Hkv * case.Nk * case.D
+            + 4 * case.B * case.Hq * case.Nq)
+
+
+def decode_bytes(case, lens) -> float:
+    kv = float(np.sum(lens)) * case.Hkv * case.D * 2 * 2
+    return kv + case.B * case.Hq * case.Nq * case.D * 2 * 2 + 4 * case.B * case.Hq * case.Nq
+
+
+def decode_flops(case, lens) -> float:
+    return 4.0 * case.D * case.Hq * case.Nq * float(np.sum(lens))
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"tflops": d["bf16_tflops"], "tflops_sustained": d["bf16_tflops_sustained"],
+                "gbs": d["hbm_gbs"], "source": "measured"}
+    return {"tflops": 1590.0, "tflops_sustained": 1400.0, "gbs": 6650.0, "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "tiled_exact_attention_mfa_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the kernel sources
+    changed since that capture."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    cur = kernel_source_hash()
+    for line in open(path):
+        parts = line.split()
+        if len(parts) == 4 and not line.startswith("#") and parts[0] == workload and parts[1] == kernel:
+            return float(parts[3]) if parts[2] == cur else None
+    return None
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------------- GPU arm
+def upload(bits, dtype, dev):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return t.view(torch.float16 if dtype == mi.FP16 else torch.bfloat16).to(dev)
+
+
+def time_steps(fn, steps, warmup, flush, stream):
+    """Run warmup untimed steps, then `steps` timed ones with an L2 flush before each.
+    Returns per-step kernel milliseconds (CUDA events on `stream`) and the bracketed total."""
+    import torch
+    for _ in range(warmup):
+        flush()
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b0.record(stream)
+    for s, e in ev:
+        flush()
+        s.record(stream)
+        fn()
+        e.record(stream)
+    b1.record(stream)
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in ev], b0.elapsed_time(b1)
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def bench_prefill(case, steps, warmup, flush, stream, with_e2e, world):
+    import torch
+    import tiled_exact_attention_mfa_b200 as mfa
+    dev = torch.device("cuda")
+    q, k, v = case.tensors()
+    qt, kt, vt = (upload(x, case.dtype, dev) for x in (q, k, v))
+    out = torch.empty_like(qt)
+    lse = torch.empty(case.B, case.Hq, case.Nq, dtype=torch.float32, device=dev)
+    scale = case.scale_f32()
+    win = (case.win_l, case.win_r)
+
+    def step():
+        mfa.mfa_fwd(qt, kt, vt, out, lse, scale=scale, causal=case.causal, window=win,
+                    softcap=case.softcap, stream=stream)
+
+    with torch.cuda.stream(stream):
+        ms, bracket = time_steps(step, steps, warmup, flush, stream)
+    res = {"ms": statistics.mean(ms), "ms_min": min(ms), "bracket_ms": bracket,
+           "flops": prefill_flops(case), "bytes": prefill_bytes(case)}
+    res["ms"] = max_over_ranks(res["ms"], world)
+    if with_e2e:
+        # public API with host buffers: pinned H2D of q, k, v, the kernel, D2H of out and lse
+        hq = torch.from_numpy(q.view(np.int16)).pin_memory()
+        hk = torch.from_numpy(k.view(np.int16)).pin_memory()
+        hv = torch.from_numpy(v.view(np.int16)).pin_memory()
+        ho = torch.empty(out.shape, dtype=torch.int16).pin_memory()
+        hl = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+        qi, ki, vi, oi = (x.view(torch.int16) for x in (qt, kt, vt, out))
+
+        def e2e_step():
+            qi.copy_(hq, non_blocking=True)
+            ki.copy_(hk, non_blocking=True)
+            vi.copy_(hv, non_blocking=True)
+            step()
+            ho.copy_(oi, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            ems, _ = time_steps(e2e_step, max(3, steps // 2), 2, flush, stream)
+        res["e2e_ms"] = max_over_ranks(statistics.mean(ems), world)
+        res["h2d"] = int(q.nbytes + k.nbytes + v.nbytes)
+        res["d2h"] = int(ho.numel() * 2 + hl.numel() * 4)
+    return res
+
+
+def bench_decode(case, steps, warmup, flush, stream, world):
+    import torch
+    import tiled_exact_attention_mfa_b200 as mfa
+    dev = torch.device("cuda")
+    q, kp, vp, table, lens = case.tensors()
+    qt, kt, vt = (upload(x, case.dtype, dev) for x in (q, kp, vp))
+    tt = torch.from_numpy(table).to(dev)
+    lt = torch.from_numpy(lens).to(dev)
+    out = torch.empty_like(qt)
+    lse = torch.empty(case.B, case.Hq, case.Nq, dtype=torch.float32, device=dev)
+    ws_bytes = mfa.mfa_decode_workspace_size(case.B, case.Nq, case.Hq, case.Hkv, case.D, table.shape[1])
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    scale = case.scale_f32()
+
+    def step():
+        mfa.mfa_decode_splitkv(qt, kt, vt, tt, lt, out, lse, scale=scale, causal=case.causal,
+                               softcap=case.softcap, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        ms, bracket = time_steps(step, steps, warmup, flush, stream)
+    return {"ms": max_over_ranks(statistics.mean(ms), world), "ms_min": min(ms),
+            "bracket_ms": bracket, "bytes": decode_bytes(case, lens),
+            "flops": decode_flops(case, lens), "seq_len_sum": int(np.sum(lens))}
+
+
+def run_gpu(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        dist.barrier()
+    import tiled_exact_attention_mfa_b200 as mfa
+    pk = peaks()
+    stream = torch.cuda.Stream()
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def flush():
+        flush_buf.fill_(1)
+
+    W = mi.workloads()
+    clocks = ClockSampler(local)
+    clocks.start()
+    main_case = W[args.workload]
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    main = bench_prefill(main_case, args.steps, args.warmup, flush, stream, not args.no_e2e, world)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    others = []
+    if not args.only_main:
+        for name, case in W.items():
+            if name == args.workload:
+                continue
+            sk, wu = max(3, min(args.steps, 10)), max(3, args.warmup)
+            if isinstance(case, mi.DecodeCase):
+                r = bench_decode(case, sk, wu, flush, stream, world)
+                tb = r["bytes"] * world / (r["ms"] * 1e-3) / 1e9
+                others.append({"workload": name, "ms": round(r["ms"], 4), "unit": "GB/s",
+                               "value": round(tb, 1), "bound": "hbm",
+                               "frac_of_measured_peak": round(tb / pk["gbs"], 4),
+                               "frac_of_nominal_peak": round(tb / NOMINAL_GBS, 4),
+                               "seq_len_sum": r["seq_len_sum"],
+                               "tflops": round(r["flops"] * world / (r["ms"] * 1e-3) / 1e12, 2)})
+            else:
+                r = bench_prefill(case, sk, wu, flush, stream, False, world)
+                tf = r["flops"] * world / (r["ms"] * 1e-3) / 1e12
+                gbs = r["bytes"] * world / (r["ms"] * 1e-3) / 1e9
+                t_floor = max(r["flops"] / (pk["tflops"] * 1e12), r["bytes"] / (pk["gbs"] * 1e9))
+                others.append({"workload": name, "ms": round(r["ms"], 4), "unit": "TFLOP/s",
+                               "value": round(tf, 1), "GB/s": round(gbs, 1),
+                               "frac_of_measured_tensor_peak": round(tf / pk["tflops"], 4),
+                               "frac_of_nominal_tensor_peak": round(tf / NOMINAL_TFLOPS, 4),
+                               "frac_of_roofline": round(t_floor / (r["ms"] * 1e-3), 4)})
+    clk = clocks.stop()
+    tflops = main["flops"] * world / (main["ms"] * 1e-3) / 1e12
+    per_gpu_tflops = main["flops"] / (main["ms"] * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": round(tflops, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(main["ms"], 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": mi.DTYPE_NAMES[main_case.dtype],
+        "data": "synthetic (seeded N(0,1) Q/K/V, SplitMix64 + Box-Muller)",
+        "config": {"workload": args.workload, "B": main_case.B, "Hq": main_case.Hq,
+                   "Hkv": main_case.Hkv, "N": main_case.Nq, "D": main_case.D,
+                   "causal": main_case.causal, "l2": "flushed before every timed step (256 MiB write)",
+                   "parallelism": f"replica per GPU x{world}"},
+        "roofline": {"bound": "tensor", "achieved": round(per_gpu_tflops, 2),
+                     "peak": pk["tflops"], "unit": "TFLOP/s",
+                     "frac": round(per_gpu_tflops / pk["tflops"], 4),
+                     "peak_source": f"{pk['source']} bf16 burst (fp16 dense rate is the same)",
+                     "frac_of_nominal": round(per_gpu_tflops / NOMINAL_TFLOPS, 4),
+                     "kernel": "mfa_fwd_kernel",
+                     "traffic": ncu_traffic(args.workload, "mfa_fwd_kernel")},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+        "workloads": others,
+    }
+    if "e2e_ms" in main:
+        line["e2e"] = {"value": round(main["flops"] * world / (main["e2e_ms"] * 1e-3) / 1e12, 3),
+                       "unit": "TFLOP/s", "ms_per_step": round(main["e2e_ms"], 4),
+                       "h2d_bytes_per_step": main["h2d"], "d2h_bytes_per_step": main["d2h"]}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(main_case, budget_s=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------- oracle timing
+def oracle_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(case, budget_s: float = 15.0):
+    """The fp64 oracle as it stands, on whole (b, h) heads of the workload until ~budget_s."""
+    import oracle
+    q, k, v = case.tensors()
+    w = lambda x: mi.widen(x, case.dtype)
+    qd, kd, vd = w(q), w(k), w(v)
+    G = case.Hq // case.Hkv
+    pairs = visible_pairs(case)
+    t0 = time.perf_counter()
+    heads = 0
+    for b in range(case.B):
+        for h in range(case.Hq):
+            oracle.attention(qd[b:b + 1, h:h + 1], kd[b:b + 1, h // G:h // G + 1],
+                             vd[b:b + 1, h // G:h // G + 1], case.scale_f32(), case.causal,
+                             case.win_l, case.win_r, case.softcap)
+            heads += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    flops = 4.0 * case.D * pairs * heads
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle_threads(),
+            "kind": "oracle", "sample": f"{heads} of {case.B * case.Hq} (b,h) heads of {case.name}, "
+                                        f"all {case.Nq} rows each, fp64 numpy, {dt:.1f} s"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    case = mi.workloads()[args.workload]
+    budget = max(1.0, min(20.0, args.cpu_seconds / max(1, args.steps)))
+    for _ in range(args.warmup):
+        cpu_baseline(case, budget_s=0.1)
+    vals = []
+    last = None
+    for _ in range(args.steps):
+        last = cpu_baseline(case, budget_s=budget)
+        vals.append(last["value"])
+    value = statistics.mean(vals)
+    ms = 4.0 * case.D * visible_pairs(case) * case.B * case.Hq / (value * 1e12) * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": last["cores"],
+                             "kind": "oracle", "sample": last["sample"]},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["mfa", "reference"], default="mfa")
+    ap.add_argument("--workload", default=MAIN,
+                    choices=sorted(n for n, c in mi.workloads().items() if isinstance(c, mi.PrefillCase)))
+    ap.add_argument("--only-main", action="store_true", help="skip the other workloads")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()
