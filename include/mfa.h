@@ -64,6 +64,7 @@ extern "C" {
 #define MFA_ERR_CUDA               -20   /* a CUDA runtime/driver call or a launch failed */
 #define MFA_ERR_DEVICE_TIMEOUT     -21   /* device status: a bounded wait inside a kernel ran out */
 #define MFA_ERR_DEVICE_BAD_PAGE    -22   /* device status: a block_table entry was outside [0, num_pages) */
+#define MFA_ERR_SCRATCH_TOO_SMALL  -23   /* mfa_decode_splitkv_noalloc: shape needs more than its fixed scratch */
 
 /*
  * mfa_fwd -- exact attention forward (prefill).
@@ -178,6 +179,40 @@ int mfa_debug_tiles_visited(void* stream, unsigned long long* count);
  * mfa_decode_workspace_size. Returns the previous value.
  */
 int mfa_debug_set_decode_split_pages(int pages);
+
+/*
+ * mfa_decode_splitkv_noalloc -- mfa_decode_splitkv for callers that cannot allocate device
+ * memory. The paper has no counterpart of this entry point; it exists for this library's users.
+ *
+ * Some callers cannot call cudaMalloc when decode runs: a serving engine that reserves all of
+ * HBM for its KV page pool up front and hands out nothing else, code running inside an
+ * allocator or memory-pool callback (where re-entering the allocator is not allowed), and
+ * latency-critical decode loops that cannot afford cudaMalloc's implicit device
+ * synchronisation. They cannot provide mfa_decode_splitkv's workspace. This variant keeps that workspace in a fixed
+ * device array inside the library instead of taking one from the caller; every other argument
+ * has the meaning given for mfa_decode_splitkv, and the computation and result are the same.
+ *
+ *   - The array holds MFA_NOALLOC_SCRATCH_BYTES (64 MiB). Every GPU on which the library is
+ *     loaded holds it until the process exits. A shape whose workspace
+ *     (mfa_decode_workspace_size) is larger is rejected with MFA_ERR_SCRATCH_TOO_SMALL before
+ *     anything runs; the paged decode of 8 sequences x 131072 tokens with 32 query heads, 8 kv
+ *     heads and D = 128 needs about 34 MB.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress with
+ *     that device current) and remembers it; make that first call before any stream capture.
+ *   - No call allocates or frees memory.
+ *   - All calls on a device share the one array and leave their partial results in it. Calls
+ *     whose kernels overlap on the GPU (different streams without ordering, or concurrent
+ *     host threads) race on it and give wrong results; order them on one stream. Nothing in the
+ *     array needs to start at zero: each call writes every entry it later reads.
+ * Returns MFA_OK after both launches were queued, or a negative status.
+ */
+#define MFA_NOALLOC_SCRATCH_BYTES (64u << 20)
+int mfa_decode_splitkv_noalloc(const void* q, const void* k_pages, const void* v_pages,
+                               const int32_t* block_table, const int32_t* seq_lens,
+                               void* out, float* lse,
+                               int B, int Nq, int Hq, int Hkv, int D, int page_size,
+                               int max_pages_per_seq, int num_pages,
+                               float scale, int causal, float softcap, int dtype, void* stream);
 
 #ifdef __cplusplus
 }

@@ -37,6 +37,10 @@ lib.mfa_decode_workspace_size.argtypes = [_i] * 7
 lib.mfa_decode_splitkv.restype = _i
 lib.mfa_decode_splitkv.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
                                    _f, _i, _f, _i, _vp, ctypes.c_size_t, _vp]
+lib.mfa_decode_splitkv_noalloc.restype = _i
+lib.mfa_decode_splitkv_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                           _i, _i, _f, _i, _f, _i, _vp]
+MFA_NOALLOC_SCRATCH_BYTES = 64 << 20
 lib.mfa_status_string.restype = ctypes.c_char_p
 lib.mfa_status_string.argtypes = [_i]
 
@@ -63,7 +67,8 @@ lib.mfa_debug_set_decode_split_pages.argtypes = [_i]
 
 EXPORTED = ("mfa_fwd", "mfa_decode_workspace_size", "mfa_decode_splitkv", "mfa_status_string",
             "mfa_last_launch_info", "mfa_device_status", "mfa_debug_set_flags",
-            "mfa_debug_tiles_visited", "mfa_debug_set_decode_split_pages")
+            "mfa_debug_tiles_visited", "mfa_debug_set_decode_split_pages",
+            "mfa_decode_splitkv_noalloc")
 
 
 class MFAError(RuntimeError):
@@ -165,6 +170,33 @@ def mfa_decode_splitkv(q, k_pages, v_pages, block_table, seq_lens, out=None, lse
                                 float(softcap), _dtype_code(q), _ptr(workspace),
                                 workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "mfa_decode_splitkv")
+    return out, lse
+
+
+def mfa_decode_splitkv_noalloc(q, k_pages, v_pages, block_table, seq_lens, out=None, lse=None, *,
+                               scale=None, causal=True, softcap=0.0, return_lse=True, stream=None):
+    """mfa_decode_splitkv without a caller workspace, for callers that cannot allocate device
+    memory when decode runs (see include/mfa.h). The workspace is the library's fixed 64 MiB
+    device array; calls that overlap on the GPU race on it, so keep them on one stream.
+    Returns (out, lse or None)."""
+    torch = _torch()
+    B, Hq, Nq, D = q.shape
+    num_pages, page, Hkv, _ = k_pages.shape
+    max_pages = block_table.shape[1]
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("block_table and seq_lens must be int32")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    rc = lib.mfa_decode_splitkv_noalloc(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
+                                        _ptr(seq_lens), _ptr(out), _ptr(lse), B, Nq, Hq, Hkv, D,
+                                        page, max_pages, num_pages, float(scale),
+                                        int(bool(causal)), float(softcap), _dtype_code(q),
+                                        _stream(stream))
+    _check(rc, "mfa_decode_splitkv_noalloc")
     return out, lse
 
 

@@ -344,6 +344,7 @@ const char* mfa_status_string(int code) {
     case MFA_ERR_CUDA: return "a CUDA call or kernel launch failed";
     case MFA_ERR_DEVICE_TIMEOUT: return "device: a bounded wait inside a kernel ran out";
     case MFA_ERR_DEVICE_BAD_PAGE: return "device: block_table or seq_lens entry out of range";
+    case MFA_ERR_SCRATCH_TOO_SMALL: return "decode shape needs more workspace than the fixed 64 MiB scratch of mfa_decode_splitkv_noalloc";
     default: return "unknown status";
   }
 }
@@ -397,3 +398,50 @@ int mfa_debug_set_decode_split_pages(int pages) {
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------------------------
+// Allocation-free decode: the workspace lives in a fixed device array of this file.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = MFA_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch per device. In host code the array's name only stands in
+// for the device symbol; kernels must be given the address cudaGetSymbolAddress returns.
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+void* noalloc_scratch(int dev) {
+  std::lock_guard<std::mutex> lk(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" int mfa_decode_splitkv_noalloc(const void* q, const void* k_pages, const void* v_pages,
+                                          const int32_t* block_table, const int32_t* seq_lens,
+                                          void* out, float* lse, int B, int Nq, int Hq, int Hkv,
+                                          int D, int page_size, int max_pages_per_seq,
+                                          int num_pages, float scale, int causal, float softcap,
+                                          int dtype, void* stream) {
+  // Every argument check of mfa_decode_splitkv runs first; with no workspace it returns before
+  // any launch, and MFA_ERR_WORKSPACE then means that everything else is valid.
+  int rc = mfa_decode_splitkv(q, k_pages, v_pages, block_table, seq_lens, out, lse, B, Nq, Hq,
+                              Hkv, D, page_size, max_pages_per_seq, num_pages, scale, causal,
+                              softcap, dtype, nullptr, 0, stream);
+  if (rc != MFA_ERR_WORKSPACE) return rc;
+  const size_t need = mfa_decode_workspace_size(B, Nq, Hq, Hkv, D, max_pages_per_seq, page_size);
+  if (need > kNoAllocScratchBytes) return MFA_ERR_SCRATCH_TOO_SMALL;
+  const int dev = current_device();
+  if (dev < 0) return MFA_ERR_CUDA;
+  void* scratch = noalloc_scratch(dev);
+  if (scratch == nullptr) return MFA_ERR_CUDA;
+  return mfa_decode_splitkv(q, k_pages, v_pages, block_table, seq_lens, out, lse, B, Nq, Hq, Hkv,
+                            D, page_size, max_pages_per_seq, num_pages, scale, causal, softcap,
+                            dtype, scratch, kNoAllocScratchBytes, stream);
+}
