@@ -172,14 +172,21 @@ def time_steps(fn, steps, warmup, flush, stream):
     return [s.elapsed_time(e) for s, e in ev], b0.elapsed_time(b1)
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """Largest per-rank time: every rank runs its own copy of the workload (weak scaling), so the
+    job takes as long as its slowest rank."""
     if world <= 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job rate: the units all ranks processed divided by the slowest rank's time (per s)."""
+    return units_per_rank * world / (max_ms * 1e-3)
 
 
 def bench_prefill(case, steps, warmup, flush, stream, with_e2e, world):
@@ -309,7 +316,7 @@ def run_gpu(args):
                                "frac_of_nominal_tensor_peak": round(tf / NOMINAL_TFLOPS, 4),
                                "frac_of_roofline": round(t_floor / (r["ms"] * 1e-3), 4)})
     clk = clocks.stop()
-    tflops = main["flops"] * world / (main["ms"] * 1e-3) / 1e12
+    tflops = job_throughput(main["flops"], world, main["ms"]) / 1e12
     per_gpu_tflops = main["flops"] / (main["ms"] * 1e-3) / 1e12
     line = {
         "metric": METRIC,

@@ -294,3 +294,18 @@ def test_decode_page_permutation_and_empty_sequence():
     np.testing.assert_array_equal(a[0], b[0])
     np.testing.assert_array_equal(a[1], b[1])
     assert np.all(a[0][1] == 0) and np.all(np.isneginf(a[1][1]))
+
+
+def test_decode_rows_helper_matches_pinned_decode():
+    B, Hq, Hkv, D, Nq = 3, 8, 2, 8, 2
+    lens = [37, 16, 70]
+    kc = rng.standard_normal((B, Hkv, 70, D))
+    vc = rng.standard_normal((B, Hkv, 70, D))
+    q = rng.standard_normal((B, Hq, Nq, D))
+    kp, vp, table = _paged_from_contiguous(kc, vc, lens)
+    o, lse = oracle.decode(q, kp, vp, table, lens, 0.3, causal=True, softcap=4.0)
+    rows = np.array([[0, 0, 0], [1, 7, 1], [2, 3, 0], [2, 4, 1]])
+    o2, l2 = oracle.decode_rows(q, kp, vp, table, lens, rows, 0.3, True, 4.0)
+    for n, (b, h, t) in enumerate(rows):
+        np.testing.assert_allclose(o2[n], o[b, h, t], rtol=0, atol=1e-14)
+        assert l2[n] == pytest.approx(lse[b, h, t], abs=1e-14)
