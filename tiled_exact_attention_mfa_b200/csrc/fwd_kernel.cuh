@@ -7,7 +7,8 @@
 // the end O / l and LSE = m + ln l. A tile whose every score of a row is masked leaves that
 // row untouched (the shader's m_new = -inf guard).
 //
-// B200 mapping (one CTA per SM, 320 threads, 2 Q tiles of 128 rows per CTA):
+// B200 mapping (one CTA per SM, 384 threads, 2 Q tiles of 128 rows per CTA; setmaxnreg gives
+// the softmax warpgroups 200 registers per thread and the producer / MMA warpgroup 104):
 //   warp 8      TMA producer: Q tiles once, then K and V tiles through 2-stage rings (128-byte
 //               swizzled smem, 3-D tensor maps so tails are zero-filled per head).
 //   warp 9      TMEM owner and single-thread tcgen05.mma issuer:
@@ -20,9 +21,12 @@
 //               only bounds P by 2^8), and then O is rescaled in TMEM by the owning warp.
 //   TMEM columns: S_0 [0,128) S_1 [128,256) O_0 [256,256+D) O_1 [256+D, 256+2D);
 //                 P_t (16-bit, 2 per column) overwrites the first 64 columns of S_t.
-// Ordering: QK for tile j+1 of Q tile t is issued only after PV for tile j of Q tile t has
-// completed (its P lives in S_t's columns), so when the softmax of tile j+1 starts, the previous
-// PV is done and O_t can be rescaled in place.
+// Ordering: QK for tile j+1 of Q tile t overwrites S_t's columns, where PV for tile j reads P_t
+// from. tcgen05 only orders MMAs that share an accumulator, so the MMA thread waits for that PV
+// to complete before issuing the QK (kQKBehindPV = 0; issuing it right behind the PV and relying
+// on in-order execution measured ~2 % faster and is not used). The commit that signals S_t
+// ready covers every earlier MMA, so when the softmax of tile j+1 starts, PV of tile j is done
+// and O_t can be rescaled in place.
 //
 // Tile skip ("mlx-mfa 2.5.2", Features: causal tile-skip, window_size=(left,right) tile skip):
 // each CTA visits only key tiles that intersect the union of its rows' visible ranges; inside,
@@ -36,7 +40,11 @@ constexpr int kFwdBM = 128;       // query rows per Q tile (= TMEM lanes)
 constexpr int kFwdBN = 128;       // keys per K/V tile
 constexpr int kFwdQT = 2;         // Q tiles per CTA
 constexpr int kFwdStages = 2;     // K ring and V ring depth
-constexpr int kFwdThreads = 320;  // 8 softmax warps + producer + MMA
+constexpr int kFwdThreads = 384;  // 8 softmax warps + producer + MMA + 2 idle
+#ifndef MFA_QK_BEHIND_PV
+#define MFA_QK_BEHIND_PV 0
+#endif
+constexpr bool kQKBehindPV = MFA_QK_BEHIND_PV != 0;
 constexpr float kRescaleLog2 = 8.0f;
 
 struct FwdParams {
@@ -126,7 +134,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     }
     for (int t = 0; t < kFwdQT; ++t) {
       mbar_init(smem_u32(&sm.bar_s_full[t]), 1);
-      mbar_init(smem_u32(&sm.bar_p_full[t]), kFwdBM);
+      mbar_init(smem_u32(&sm.bar_p_full[t]), kFwdBM / 32);  // one arrival per softmax warp
       mbar_init(smem_u32(&sm.bar_o_done[t]), 1);
     }
     mbar_init(smem_u32(&sm.bar_final), 1);
@@ -153,7 +161,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
   constexpr uint32_t kTileBytes = FwdSmem<D>::kTileBytes;
   constexpr int kSlab = FwdSmem<D>::kSlabBytes;
 
-  if (warp == 8) {
+  if (warp >= 8) {
+   regs_control();
+   if (warp == 8) {
     // ================================================================ TMA producer
     if (lane == 0 && n_tiles > 0) {
       const uint32_t bq = smem_u32(&sm.bar_q);
@@ -236,7 +246,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         tc_commit(smem_u32(&sm.bar_o_done[0]));
         if (more) {
           if (!(ok = mbar_wait(smem_u32(&sm.bar_k_full[s1]), ph1, abort, 905))) break;
-          if (!(ok = mbar_wait(smem_u32(&sm.bar_o_done[0]), j & 1, abort, 906))) break;
+          if (!kQKBehindPV && !(ok = mbar_wait(smem_u32(&sm.bar_o_done[0]), j & 1, abort, 906))) break;
           tc_fence_after();
           issue_qk(0, s1);
           tc_commit(smem_u32(&sm.bar_s_full[0]));
@@ -248,7 +258,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         tc_commit(smem_u32(&sm.bar_o_done[1]));
         tc_commit(smem_u32(&sm.bar_v_empty[s]));
         if (more) {
-          if (!(ok = mbar_wait(smem_u32(&sm.bar_o_done[1]), j & 1, abort, 908))) break;
+          if (!kQKBehindPV && !(ok = mbar_wait(smem_u32(&sm.bar_o_done[1]), j & 1, abort, 908))) break;
           tc_fence_after();
           issue_qk(1, s1);
           tc_commit(smem_u32(&sm.bar_s_full[1]));
@@ -260,7 +270,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       volatile int no_abort = 0;
       mbar_wait(smem_u32(&sm.bar_final), 0, &no_abort, 909);
     }
+   }
   } else {
+    regs_softmax();
     // ================================================================ softmax warps
     const int t = warp >> 2;                  // Q tile of this warpgroup
     const int quarter = warp & 3;             // TMEM lane quarter of this warp
@@ -307,9 +319,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
 #pragma unroll
         for (int i = 0; i < 128; ++i) s[i] = (i < jhi && i >= jlo) ? s[i] : -INFINITY;
       }
-      float mx = s[0];
+      // row max: 8 chains of 3-input max
+      float m8[8];
 #pragma unroll
-      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+      for (int i = 0; i < 8; ++i) m8[i] = fmaxf(s[i], s[i + 8]);
+#pragma unroll
+      for (int i = 16; i < 128; i += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) m8[k] = max3(m8[k], s[i + k], s[i + 8 + k]);
+      const float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
 
       // Lazy rescale: move the reference max only when it grew by more than 2^8 in exp2 terms.
       const float m_new = fmaxf(m_run, mx);
@@ -323,18 +341,39 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         }
       }
       const float neg_mc = (m_run == -INFINITY) ? 0.f : -m_run * c;
-      float sum = 0.f;
-      uint32_t pk[64];
+
+      // P = exp2(s * c - m * c) on fp32 pairs: one pair in four on the FMA pipe, the rest on
+      // MUFU; P is packed to the input type and stored to TMEM 16 columns at a time.
+      const uint64_t c2 = f2_pack(c, c);
+      const uint64_t nm2 = f2_pack(neg_mc, neg_mc);
+      uint64_t acc[4];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float p0 = fast_exp2(fmaf(s[2 * i], c, neg_mc));
-        const float p1 = fast_exp2(fmaf(s[2 * i + 1], c, neg_mc));
-        sum += p0 + p1;
-        pk[i] = pack2<BF16>(p0, p1);
+      for (int i = 0; i < 4; ++i) acc[i] = f2_pack(0.f, 0.f);
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int ii = ch * 16 + i;
+          const uint64_t x = f2_fma(f2_pack(s[2 * ii], s[2 * ii + 1]), c2, nm2);
+          uint64_t pp;
+          if ((ii & 3) == 3) {
+            pp = exp2_fma2(x);
+          } else {
+            float x0, x1;
+            f2_unpack(x, x0, x1);
+            pp = f2_pack(fast_exp2(x0), fast_exp2(x1));
+          }
+          acc[ii & 3] = f2_add(acc[ii & 3], pp);
+          float p0, p1;
+          f2_unpack(pp, p0, p1);
+          pk[i] = pack2<BF16>(p0, p1);
+        }
+        tmem_st16(t_s + ch * 16, pk);
       }
-      l_run = l_run * alpha + sum;
-      tmem_st32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      float sa, sb;
+      f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), sa, sb);
+      l_run = l_run * alpha + (sa + sb);
       // O rescale (only after the first tile: before it O holds nothing).
       if (warp_rescale && j > 0) {
 #pragma unroll
@@ -342,14 +381,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
           uint32_t o[32];
           tmem_ld32(t_o + cb, o);
           tmem_wait_ld();
+          const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          for (int i = 0; i < 16; ++i) {
+            float lo, hi;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2), lo, hi);
+            o[2 * i] = __float_as_uint(lo);
+            o[2 * i + 1] = __float_as_uint(hi);
+          }
           tmem_st32(t_o + cb, o);
         }
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&sm.bar_p_full[t]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.bar_p_full[t]));
     }
 
     // ---- epilogue: O / l, LSE

@@ -117,9 +117,23 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, float* ls
                int Hkv, int Nq, int Nk, float scale, int causal, int win_l, int win_r,
                float softcap, int dtype, cudaStream_t st) {
   static bool smem_done[kMaxDevices] = {};
+  static bool regs_ok[kMaxDevices] = {};
   constexpr int smem = mfa::fwd_smem_bytes<D>();
   auto kernel = mfa::mfa_fwd_kernel<D, BF16>;
   if (!ensure_smem(kernel, smem, smem_done)) return MFA_ERR_CUDA;
+  {
+    // setmaxnreg redistributes the registers the CTA launched with; refuse to launch if the
+    // split does not fit that pool (the growing warpgroups would wait forever).
+    const int dev = current_device();
+    if (dev < 0) return MFA_ERR_CUDA;
+    if (!regs_ok[dev]) {
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return MFA_ERR_CUDA;
+      if (fa.numRegs * mfa::kFwdThreads < 256 * mfa::kRegsSoftmax + 128 * mfa::kRegsControl)
+        return MFA_ERR_CUDA;
+      regs_ok[dev] = true;
+    }
+  }
   mfa::FwdParams p;
   std::memset(&p, 0, sizeof(p));
   if (!make_map(&p.tm_q, q, dtype, (long long)B * Hq, Nq, D)) return MFA_ERR_CUDA;

@@ -179,6 +179,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -258,13 +267,96 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+__device__ __forceinline__ float fast_rcp(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // tanh from exp: tanh(|y|) = 1 - 2 / (exp(2|y|) + 1), sign restored. Absolute error of a few
-// fp32 ulps of 1 (ex2.approx relative error ~2^-22, correctly rounded division).
+// 1e-7 (ex2.approx and rcp.approx relative errors ~2^-22); exp overflow gives exactly +-1.
 __device__ __forceinline__ float tanh_from_exp(float y) {
-  float ay = fabsf(y);
-  float e = fast_exp2(ay * 2.8853900817779268f);  // 2 * log2(e)
-  float t = 1.0f - __fdiv_rn(2.0f, e + 1.0f);
+  const float e = fast_exp2(fabsf(y) * 2.8853900817779268f);  // 2 * log2(e)
+  const float t = fmaf(-2.0f, fast_rcp(e + 1.0f), 1.0f);
   return copysignf(t, y);
 }
+
+// ---------------------------------------------------------------- packed fp32 pairs
+// sm_100 executes add / sub / mul / fma on fp32 pairs in one instruction (.f32x2).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// exp2 on the FMA/ALU pipes for a pair of values, used for a share of the softmax exponentials
+// so that the MUFU unit is not the only exp2 path. Range reduction x = n + f, n = round(x),
+// f in [-1/2, 1/2]: adding 1.5 * 2^23 leaves round(x) in the low mantissa bits (Cody and Waite
+// style reduction); 2^n is written straight into the exponent field; 2^f is a degree-4
+// polynomial fitted by csrc/fit_exp2_poly.py (near-minimax relative error 2.9e-6 on
+// [-1/2, 1/2], p(0) = 1). Inputs at or below -127 (and -inf) give exactly 0; inputs must be
+// below 128.
+constexpr float kExp2C1 = 6.931242347e-01f;
+constexpr float kExp2C2 = 2.402409911e-01f;
+constexpr float kExp2C3 = 5.590614304e-02f;
+constexpr float kExp2C4 = 9.582744911e-03f;
+
+__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -127.0f), fmaxf(x1, -127.0f));
+  const uint64_t t = f2_add(xc, f2_pack(12582912.0f, 12582912.0f));
+  const uint64_t n = f2_sub(t, f2_pack(12582912.0f, 12582912.0f));
+  const uint64_t f = f2_sub(xc, n);
+  uint64_t p = f2_fma(f2_pack(kExp2C4, kExp2C4), f, f2_pack(kExp2C3, kExp2C3));
+  p = f2_fma(p, f, f2_pack(kExp2C2, kExp2C2));
+  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
+  p = f2_fma(p, f, f2_pack(1.0f, 1.0f));
+  float t0, t1;
+  f2_unpack(t, t0, t1);
+  // (bits(t) - bits(1.5 * 2^23) + 127) << 23, i.e. 2^n as fp32 bits (0 when n = -127)
+  const uint32_t k = (uint32_t)(127 - 0x4B400000) << 23;
+  const uint32_t e0 = ((uint32_t)__float_as_int(t0) << 23) + k;
+  const uint32_t e1 = ((uint32_t)__float_as_int(t1) << 23) + k;
+  return f2_mul(p, f2_pack(__uint_as_float(e0), __uint_as_float(e1)));
+}
+
+// Register split of the forward kernel (setmaxnreg): the two softmax warpgroups grow to 200
+// registers per thread, the producer / MMA warpgroup shrinks to 104. The kernel launches with
+// 384 threads x 168 registers = 64512; 256 x 200 + 128 x 104 = 64512 is exactly that pool (the
+// host checks the launch register count before the first launch, since a split above the pool
+// would wait forever).
+constexpr int kRegsSoftmax = 200;
+constexpr int kRegsControl = 104;
+__device__ __forceinline__ void regs_softmax() { asm volatile("setmaxnreg.inc.sync.aligned.u32 200;"); }
+__device__ __forceinline__ void regs_control() { asm volatile("setmaxnreg.dec.sync.aligned.u32 104;"); }
 
 }  // namespace mfa
