@@ -302,8 +302,30 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
 
       const int k0 = (kt_lo + j) * kFwdBN;
       if (p.softcap > 0.f) {
+        // s <- cap * tanh(s * scale / cap). When every |y| = |s| * scale / cap of this warp's
+        // rows is small, tanh(y) = y * q(y^2) on packed pairs; otherwise the exp form.
+        float am8[8];
 #pragma unroll
-        for (int i = 0; i < 128; ++i) s[i] = p.softcap * tanh_from_exp(s[i] * p.cap_in);
+        for (int i = 0; i < 8; ++i) am8[i] = fmaxf(fabsf(s[i]), fabsf(s[i + 8]));
+#pragma unroll
+        for (int i = 16; i < 128; i += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) am8[k] = max3(am8[k], fabsf(s[i + k]), fabsf(s[i + 8 + k]));
+        const float amax = max3(max3(am8[0], am8[1], am8[2]), max3(am8[3], am8[4], am8[5]),
+                                fmaxf(am8[6], am8[7]));
+        if (__all_sync(0xffffffffu, amax * p.cap_in <= kTanhPolyMax)) {
+          const uint64_t ci = f2_pack(p.cap_in, p.cap_in);
+          const uint64_t cap = f2_pack(p.softcap, p.softcap);
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const uint64_t y = f2_mul(f2_pack(s[2 * i], s[2 * i + 1]), ci);
+            const uint64_t t = f2_mul(f2_mul(y, tanh_q2(f2_mul(y, y))), cap);
+            f2_unpack(t, s[2 * i], s[2 * i + 1]);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 128; ++i) s[i] = p.softcap * tanh_from_exp(s[i] * p.cap_in);
+        }
       }
       // Element masks only where some row of this Q tile may not see some key of the tile.
       bool interior = (k0 + kFwdBN <= p.Nk);

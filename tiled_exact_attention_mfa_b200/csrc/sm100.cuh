@@ -349,6 +349,23 @@ __device__ __forceinline__ uint64_t exp2_fma2(uint64_t x) {
   return f2_mul(p, f2_pack(__uint_as_float(e0), __uint_as_float(e1)));
 }
 
+// tanh(y) ~ y * q(y^2) for |y| <= kTanhPolyMax: q is a degree-4 polynomial in u = y^2 with
+// q(0) = 1, fitted by csrc/fit_tanh_poly.py (near-minimax relative error 2.1e-7, absolute
+// error 1.1e-7 on [0, 0.625]).
+constexpr float kTanhPolyMax = 0.625f;
+constexpr float kTanhQ1 = -3.333234191e-01f;
+constexpr float kTanhQ2 = 1.330818683e-01f;
+constexpr float kTanhQ3 = -5.194849521e-02f;
+constexpr float kTanhQ4 = 1.519625355e-02f;
+
+// q(u) for a pair of u values.
+__device__ __forceinline__ uint64_t tanh_q2(uint64_t u) {
+  uint64_t q = f2_fma(f2_pack(kTanhQ4, kTanhQ4), u, f2_pack(kTanhQ3, kTanhQ3));
+  q = f2_fma(q, u, f2_pack(kTanhQ2, kTanhQ2));
+  q = f2_fma(q, u, f2_pack(kTanhQ1, kTanhQ1));
+  return f2_fma(q, u, f2_pack(1.0f, 1.0f));
+}
+
 // Register split of the forward kernel (setmaxnreg): the two softmax warpgroups grow to 200
 // registers per thread, the producer / MMA warpgroup shrinks to 104. The kernel launches with
 // 384 threads x 168 registers = 64512; 256 x 200 + 128 x 104 = 64512 is exactly that pool (the
