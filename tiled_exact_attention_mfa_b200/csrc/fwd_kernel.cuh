@@ -46,6 +46,11 @@ constexpr int kFwdThreads = 384;  // 8 softmax warps + producer + MMA + 2 idle
 #endif
 constexpr bool kQKBehindPV = MFA_QK_BEHIND_PV != 0;
 constexpr float kRescaleLog2 = 8.0f;
+#ifndef MFA_POLY_MASK
+#define MFA_POLY_MASK 0x0ull
+#endif
+// Pairs of P computed with the FMA-pipe exp2 (bit i of the mask = pair i of the 64 per row).
+__host__ __device__ constexpr bool kPolyPair(int i) { return (MFA_POLY_MASK >> i) & 1ull; }
 
 struct FwdParams {
   CUtensorMap tm_q;  // [B*Hq][Nq][D]
@@ -379,7 +384,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
           const int ii = ch * 16 + i;
           const uint64_t x = f2_fma(f2_pack(s[2 * ii], s[2 * ii + 1]), c2, nm2);
           uint64_t pp;
-          if ((ii & 3) == 3) {
+          if (kPolyPair(ii)) {
             pp = exp2_fma2(x);
           } else {
             float x0, x1;
