@@ -81,11 +81,14 @@ struct DecodePlan {
   int groups;
 };
 
-DecodePlan decode_plan(int B, int Hkv, int max_pages) {
+DecodePlan decode_plan(int B, int Hkv, int D, int max_pages) {
   DecodePlan pl;
+  // kv heads per CTA: the largest divisor of Hkv whose token row (heads x D x 2 bytes) fits in
+  // 1 KB, so that a 3-stage K+V page ring stays near 100 KB and two CTAs share an SM (one
+  // streams pages while the other starts up or drains).
   pl.heads_per_cta = 1;
   for (int h = 8; h >= 1; --h)
-    if (Hkv % h == 0) {
+    if (Hkv % h == 0 && h * D * 2 <= 1024) {
       pl.heads_per_cta = h;
       break;
     }
@@ -274,7 +277,7 @@ static int validate_decode(int B, int Nq, int Hq, int Hkv, int D, int page_size,
 size_t mfa_decode_workspace_size(int B, int Nq, int Hq, int Hkv, int D, int max_pages_per_seq,
                                  int page_size) {
   if (validate_decode(B, Nq, Hq, Hkv, D, page_size, max_pages_per_seq) != MFA_OK) return 0;
-  DecodePlan pl = decode_plan(B, Hkv, max_pages_per_seq);
+  DecodePlan pl = decode_plan(B, Hkv, D, max_pages_per_seq);
   const size_t rows = (size_t)B * pl.max_splits * Hq * Nq;
   return align256(rows * D * sizeof(float)) + align256(rows * 2 * sizeof(float));
 }
@@ -300,7 +303,7 @@ int mfa_decode_splitkv(const void* q, const void* k_pages, const void* v_pages,
   const size_t need = mfa_decode_workspace_size(B, Nq, Hq, Hkv, D, max_pages_per_seq, page_size);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
     return MFA_ERR_WORKSPACE;
-  DecodePlan pl = decode_plan(B, Hkv, max_pages_per_seq);
+  DecodePlan pl = decode_plan(B, Hkv, D, max_pages_per_seq);
   mfa::DecodeParams p;
   std::memset(&p, 0, sizeof(p));
   p.q = static_cast<const uint16_t*>(q);
