@@ -300,8 +300,38 @@ __global__ void __launch_bounds__(9 * 32) mfa_decode_phase1_kernel(const __grid_
   }
 }
 
+// Block-wide reductions over D threads (D / 32 warps).
+template <int D>
+__device__ __forceinline__ float block_max(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = red[0];
+#pragma unroll
+  for (int w = 1; w < D / 32; ++w) r = fmaxf(r, red[w]);
+  __syncthreads();
+  return r;
+}
+template <int D>
+__device__ __forceinline__ float block_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = red[0];
+#pragma unroll
+  for (int w = 1; w < D / 32; ++w) r += red[w];
+  __syncthreads();
+  return r;
+}
+
+// One CTA per (query row, sequence), one thread per output column. The split statistics are
+// read cooperatively (threads stride over the splits) and the weighted sum of partial outputs is
+// unrolled four ways so that the loads of several splits are in flight at once.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(D) mfa_decode_combine_kernel(const __grid_constant__ DecodeParams p) {
+  __shared__ float red[D / 32];
   const int row = blockIdx.x;  // h * Nq + t
   const int b = blockIdx.y;
   const int d = threadIdx.x;
@@ -309,20 +339,41 @@ __global__ void __launch_bounds__(D) mfa_decode_combine_kernel(const __grid_cons
   const int n_pages = (len + kDecPage - 1) / kDecPage;
   const int n_splits = (n_pages + p.pages_per_split - 1) / p.pages_per_split;
   const size_t rows_all = (size_t)p.Hq * p.Nq;
-  float M = -INFINITY;
-  for (int s = 0; s < n_splits; ++s)
-    M = fmaxf(M, p.ws_ml[(((size_t)b * p.max_splits + s) * rows_all + row) * 2]);
-  float L = 0.f, acc = 0.f;
+  const size_t slot0 = (size_t)b * p.max_splits * rows_all + row;  // slot of split s: slot0 + s * rows_all
+  const float2* ml = reinterpret_cast<const float2*>(p.ws_ml);
+
+  float m_loc = -INFINITY;
+  for (int s = d; s < n_splits; s += D) m_loc = fmaxf(m_loc, ml[slot0 + (size_t)s * rows_all].x);
+  const float M = block_max<D>(m_loc, red);
+  float l_loc = 0.f;
+  if (M > -INFINITY)
+    for (int s = d; s < n_splits; s += D) {
+      const float2 v = ml[slot0 + (size_t)s * rows_all];
+      l_loc += (v.x == -INFINITY) ? 0.f : fast_exp2(v.x - M) * v.y;
+    }
+  const float L = block_sum<D>(l_loc, red);
+
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
   if (M > -INFINITY) {
-    for (int s = 0; s < n_splits; ++s) {
-      const size_t slot = ((size_t)b * p.max_splits + s) * rows_all + row;
-      const float2 ml = *reinterpret_cast<const float2*>(p.ws_ml + slot * 2);
-      const float w = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - M);
-      L += w * ml.y;
-      acc += w * p.ws_o[slot * D + d];
+    const float* o = p.ws_o + slot0 * D + d;
+    const size_t stride = rows_all * D;
+    int s = 0;
+    for (; s + 4 <= n_splits; s += 4) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float mu = ml[slot0 + (size_t)(s + u) * rows_all].x;
+        const float w = (mu == -INFINITY) ? 0.f : fast_exp2(mu - M);
+        acc[u] = fmaf(w, o[(size_t)(s + u) * stride], acc[u]);
+      }
+    }
+    for (; s < n_splits; ++s) {
+      const float mu = ml[slot0 + (size_t)s * rows_all].x;
+      const float w = (mu == -INFINITY) ? 0.f : fast_exp2(mu - M);
+      acc[0] = fmaf(w, o[(size_t)s * stride], acc[0]);
     }
   }
-  const float val = (L > 0.f) ? acc / L : 0.f;
+  const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  const float val = (L > 0.f) ? sum / L : 0.f;
   const size_t orow = (size_t)b * rows_all + row;
   uint16_t bits;
   if constexpr (BF16) {
