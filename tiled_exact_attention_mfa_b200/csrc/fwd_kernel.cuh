@@ -79,7 +79,9 @@ struct FwdSmem {
   uint64_t bar_q;
   uint64_t bar_k_full[kFwdStages], bar_k_empty[kFwdStages];
   uint64_t bar_v_full[kFwdStages], bar_v_empty[kFwdStages];
-  uint64_t bar_s_full[kFwdQT], bar_p_full[kFwdQT], bar_o_done[kFwdQT];
+  // P of a Q tile becomes ready in two halves (keys 0-63, 64-127), so the first half of PV can
+  // run while the second half of the exponentials is computed
+  uint64_t bar_s_full[kFwdQT], bar_p_full[kFwdQT][2], bar_o_done[kFwdQT];
   uint64_t bar_final;
   uint32_t tmem_base;
   int abort;
@@ -139,7 +141,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     }
     for (int t = 0; t < kFwdQT; ++t) {
       mbar_init(smem_u32(&sm.bar_s_full[t]), 1);
-      mbar_init(smem_u32(&sm.bar_p_full[t]), kFwdBM / 32);  // one arrival per softmax warp
+      mbar_init(smem_u32(&sm.bar_p_full[t][0]), kFwdBM / 32);  // one arrival per softmax warp
+      mbar_init(smem_u32(&sm.bar_p_full[t][1]), kFwdBM / 32);
       mbar_init(smem_u32(&sm.bar_o_done[t]), 1);
     }
     mbar_init(smem_u32(&sm.bar_final), 1);
@@ -218,10 +221,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
                     smem_desc_sw128(ka + koff, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, int s, bool acc) {
+      // half h covers keys 64h .. 64h + 63 (P columns 32h .. 32h + 31)
+      auto issue_pv = [&](int t, int s, bool acc, int h) {
         const uint32_t va = smem_u32(sm.v[s]);
 #pragma unroll
-        for (int kk = 0; kk < kFwdBN / 16; ++kk) {
+        for (int kk = h * 4; kk < h * 4 + 4; ++kk) {
           tc_mma_ts(tmem + 256 + t * D, tmem + t * kFwdBN + kk * 8,
                     smem_desc_sw128(va + kk * 16 * 128, kSlab, 1024), idesc_pv,
                     (acc || kk > 0) ? 1u : 0u);
@@ -245,9 +249,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         }
         // Q tile 0: PV(j), then QK(j+1) once PV(j) is done (P_0 lives in S_0's columns)
         if (!(ok = mbar_wait(smem_u32(&sm.bar_v_full[s]), ph, abort, 903))) break;
-        if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[0]), j & 1, abort, 904))) break;
+        if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[0][0]), j & 1, abort, 904))) break;
         tc_fence_after();
-        issue_pv(0, s, j > 0);
+        issue_pv(0, s, j > 0, 0);
+        if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[0][1]), j & 1, abort, 914))) break;
+        tc_fence_after();
+        issue_pv(0, s, true, 1);
         tc_commit(smem_u32(&sm.bar_o_done[0]));
         if (more) {
           if (!(ok = mbar_wait(smem_u32(&sm.bar_k_full[s1]), ph1, abort, 905))) break;
@@ -257,9 +264,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
           tc_commit(smem_u32(&sm.bar_s_full[0]));
         }
         // Q tile 1
-        if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[1]), j & 1, abort, 907))) break;
+        if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[1][0]), j & 1, abort, 907))) break;
         tc_fence_after();
-        issue_pv(1, s, j > 0);
+        issue_pv(1, s, j > 0, 0);
+        if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[1][1]), j & 1, abort, 917))) break;
+        tc_fence_after();
+        issue_pv(1, s, true, 1);
         tc_commit(smem_u32(&sm.bar_o_done[1]));
         tc_commit(smem_u32(&sm.bar_v_empty[s]));
         if (more) {
@@ -369,8 +379,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       }
       const float neg_mc = (m_run == -INFINITY) ? 0.f : -m_run * c;
 
-      // P = exp2(s * c - m * c) on fp32 pairs: one pair in four on the FMA pipe, the rest on
-      // MUFU; P is packed to the input type and stored to TMEM 16 columns at a time.
+      // O rescale before any PV of this tile reads P (only after the first tile: before it O
+      // holds nothing). The previous PV of this Q tile has completed: its commit preceded S.
+      if (warp_rescale && j > 0) {
+#pragma unroll
+        for (int cb = 0; cb < D; cb += 32) {
+          uint32_t o[32];
+          tmem_ld32(t_o + cb, o);
+          tmem_wait_ld();
+          const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float lo, hi;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2), lo, hi);
+            o[2 * i] = __float_as_uint(lo);
+            o[2 * i + 1] = __float_as_uint(hi);
+          }
+          tmem_st32(t_o + cb, o);
+        }
+      }
+      // P = exp2(s * c - m * c) on fp32 pairs, packed to the input type and stored to TMEM 16
+      // columns at a time; each half of P is announced as soon as it is stored.
       const uint64_t c2 = f2_pack(c, c);
       const uint64_t nm2 = f2_pack(neg_mc, neg_mc);
       uint64_t acc[4];
@@ -397,32 +426,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
           pk[i] = pack2<BF16>(p0, p1);
         }
         tmem_st16(t_s + ch * 16, pk);
+        if (ch & 1) {
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&sm.bar_p_full[t][ch >> 1]));
+        }
       }
       float sa, sb;
       f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), sa, sb);
       l_run = l_run * alpha + (sa + sb);
-      // O rescale (only after the first tile: before it O holds nothing).
-      if (warp_rescale && j > 0) {
-#pragma unroll
-        for (int cb = 0; cb < D; cb += 32) {
-          uint32_t o[32];
-          tmem_ld32(t_o + cb, o);
-          tmem_wait_ld();
-          const uint64_t a2 = f2_pack(alpha, alpha);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float lo, hi;
-            f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), a2), lo, hi);
-            o[2 * i] = __float_as_uint(lo);
-            o[2 * i + 1] = __float_as_uint(hi);
-          }
-          tmem_st32(t_o + cb, o);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.bar_p_full[t]));
+
     }
 
     // ---- epilogue: O / l, LSE
