@@ -300,8 +300,10 @@ __global__ void __launch_bounds__(9 * 32) mfa_decode_phase1_kernel(const __grid_
   }
 }
 
-// Block-wide reductions over D threads (D / 32 warps).
-template <int D>
+// Threads per combine CTA: kCombineGroups groups of D threads; group q takes splits q, q + G, ...
+constexpr int kCombineThreads = 512;
+
+// Block-wide reductions over kCombineThreads threads.
 __device__ __forceinline__ float block_max(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -309,11 +311,10 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   __syncthreads();
   float r = red[0];
 #pragma unroll
-  for (int w = 1; w < D / 32; ++w) r = fmaxf(r, red[w]);
+  for (int w = 1; w < kCombineThreads / 32; ++w) r = fmaxf(r, red[w]);
   __syncthreads();
   return r;
 }
-template <int D>
 __device__ __forceinline__ float block_sum(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -321,20 +322,24 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   __syncthreads();
   float r = red[0];
 #pragma unroll
-  for (int w = 1; w < D / 32; ++w) r += red[w];
+  for (int w = 1; w < kCombineThreads / 32; ++w) r += red[w];
   __syncthreads();
   return r;
 }
 
-// One CTA per (query row, sequence), one thread per output column. The split statistics are
-// read cooperatively (threads stride over the splits) and the weighted sum of partial outputs is
-// unrolled four ways so that the loads of several splits are in flight at once.
+// One CTA per (query row, sequence). The split statistics are read cooperatively; each of the
+// kCombineThreads / D groups of threads sums the weighted partial outputs of every G-th split
+// (one thread per column, two splits in flight per thread), and the groups are added in shared
+// memory.
 template <int D, bool BF16>
-__global__ void __launch_bounds__(D) mfa_decode_combine_kernel(const __grid_constant__ DecodeParams p) {
-  __shared__ float red[D / 32];
+__global__ void __launch_bounds__(kCombineThreads) mfa_decode_combine_kernel(const __grid_constant__ DecodeParams p) {
+  constexpr int G = kCombineThreads / D;
+  __shared__ float red[kCombineThreads / 32];
+  __shared__ float part[G][D];
   const int row = blockIdx.x;  // h * Nq + t
   const int b = blockIdx.y;
-  const int d = threadIdx.x;
+  const int d = threadIdx.x % D;
+  const int grp = threadIdx.x / D;
   const int len = checked_len(p, b, false);
   const int n_pages = (len + kDecPage - 1) / kDecPage;
   const int n_splits = (n_pages + p.pages_per_split - 1) / p.pages_per_split;
@@ -343,46 +348,51 @@ __global__ void __launch_bounds__(D) mfa_decode_combine_kernel(const __grid_cons
   const float2* ml = reinterpret_cast<const float2*>(p.ws_ml);
 
   float m_loc = -INFINITY;
-  for (int s = d; s < n_splits; s += D) m_loc = fmaxf(m_loc, ml[slot0 + (size_t)s * rows_all].x);
-  const float M = block_max<D>(m_loc, red);
+  for (int s = threadIdx.x; s < n_splits; s += kCombineThreads) m_loc = fmaxf(m_loc, ml[slot0 + (size_t)s * rows_all].x);
+  const float M = block_max(m_loc, red);
   float l_loc = 0.f;
   if (M > -INFINITY)
-    for (int s = d; s < n_splits; s += D) {
+    for (int s = threadIdx.x; s < n_splits; s += kCombineThreads) {
       const float2 v = ml[slot0 + (size_t)s * rows_all];
       l_loc += (v.x == -INFINITY) ? 0.f : fast_exp2(v.x - M) * v.y;
     }
-  const float L = block_sum<D>(l_loc, red);
+  const float L = block_sum(l_loc, red);
 
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float acc0 = 0.f, acc1 = 0.f;
   if (M > -INFINITY) {
     const float* o = p.ws_o + slot0 * D + d;
     const size_t stride = rows_all * D;
-    int s = 0;
-    for (; s + 4 <= n_splits; s += 4) {
+    int s = grp;
+    for (; s + G < n_splits; s += 2 * G) {
+      const float m0 = ml[slot0 + (size_t)s * rows_all].x;
+      const float m1 = ml[slot0 + (size_t)(s + G) * rows_all].x;
+      const float o0 = o[(size_t)s * stride];
+      const float o1 = o[(size_t)(s + G) * stride];
+      acc0 = fmaf((m0 == -INFINITY) ? 0.f : fast_exp2(m0 - M), o0, acc0);
+      acc1 = fmaf((m1 == -INFINITY) ? 0.f : fast_exp2(m1 - M), o1, acc1);
+    }
+    if (s < n_splits) {
+      const float m0 = ml[slot0 + (size_t)s * rows_all].x;
+      acc0 = fmaf((m0 == -INFINITY) ? 0.f : fast_exp2(m0 - M), o[(size_t)s * stride], acc0);
+    }
+  }
+  part[grp][d] = acc0 + acc1;
+  __syncthreads();
+  if (grp == 0) {
+    float sum = part[0][d];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float mu = ml[slot0 + (size_t)(s + u) * rows_all].x;
-        const float w = (mu == -INFINITY) ? 0.f : fast_exp2(mu - M);
-        acc[u] = fmaf(w, o[(size_t)(s + u) * stride], acc[u]);
-      }
+    for (int q = 1; q < G; ++q) sum += part[q][d];
+    const float val = (L > 0.f) ? sum / L : 0.f;
+    const size_t orow = (size_t)b * rows_all + row;
+    uint16_t bits;
+    if constexpr (BF16) {
+      bits = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+    } else {
+      bits = __half_as_ushort(__float2half_rn(val));
     }
-    for (; s < n_splits; ++s) {
-      const float mu = ml[slot0 + (size_t)s * rows_all].x;
-      const float w = (mu == -INFINITY) ? 0.f : fast_exp2(mu - M);
-      acc[0] = fmaf(w, o[(size_t)s * stride], acc[0]);
-    }
+    reinterpret_cast<uint16_t*>(p.out)[orow * D + d] = bits;
+    if (d == 0 && p.lse != nullptr) p.lse[orow] = (L > 0.f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
   }
-  const float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-  const float val = (L > 0.f) ? sum / L : 0.f;
-  const size_t orow = (size_t)b * rows_all + row;
-  uint16_t bits;
-  if constexpr (BF16) {
-    bits = __bfloat16_as_ushort(__float2bfloat16_rn(val));
-  } else {
-    bits = __half_as_ushort(__float2half_rn(val));
-  }
-  reinterpret_cast<uint16_t*>(p.out)[orow * D + d] = bits;
-  if (d == 0 && p.lse != nullptr) p.lse[orow] = (L > 0.f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
 
 }  // namespace mfa

@@ -200,7 +200,7 @@ int launch_decode(const mfa::DecodeParams& p, const DecodePlan& pl, cudaStream_t
   k1<<<g1, (pl.heads_per_cta + 1) * 32, smem, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
   dim3 g2(p.Hq * p.Nq, p.B, 1);
-  mfa::mfa_decode_combine_kernel<D, BF16><<<g2, D, 0, st>>>(p);
+  mfa::mfa_decode_combine_kernel<D, BF16><<<g2, mfa::kCombineThreads, 0, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
   mfa_launch_info li = {};
   li.kernel = 2;
