@@ -78,12 +78,18 @@ def peaks():
     return {"tflops": 1590.0, "tflops_sustained": 1400.0, "gbs": 6650.0, "source": "fallback"}
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCES = {
+    "mfa_fwd_kernel": ("fwd_kernel.cuh", "sm100.cuh"),
+    "mfa_decode_phase1_kernel": ("decode_kernel.cuh", "sm100.cuh"),
+}
+
+
+def kernel_source_hash(kernel: str = "mfa_fwd_kernel") -> str:
+    """Hash of the source files a kernel is built from (a changed kernel invalidates its record)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "tiled_exact_attention_mfa_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in KERNEL_SOURCES[kernel]:
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -93,7 +99,7 @@ def ncu_traffic(workload: str, kernel: str):
     path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(path):
         return None
-    cur = kernel_source_hash()
+    cur = kernel_source_hash(kernel)
     for line in open(path):
         parts = line.split()
         if len(parts) == 4 and not line.startswith("#") and parts[0] == workload and parts[1] == kernel:
@@ -304,6 +310,7 @@ def run_gpu(args):
                                "frac_of_measured_peak": round(tb / pk["gbs"], 4),
                                "frac_of_nominal_peak": round(tb / NOMINAL_GBS, 4),
                                "seq_len_sum": r["seq_len_sum"],
+                               "traffic_phase1": ncu_traffic(name, "mfa_decode_phase1_kernel"),
                                "tflops": round(r["flops"] * world / (r["ms"] * 1e-3) / 1e12, 2)})
             else:
                 r = bench_prefill(case, sk, wu, flush, stream, False, world)
@@ -425,6 +432,21 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_profile(args):
+    """One workload alone (prefill or decode), for profiler captures: no e2e, no CPU baseline,
+    no other workloads. Prints the mean per-step milliseconds."""
+    import torch
+    torch.cuda.set_device(0)
+    stream = torch.cuda.Stream()
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    case = mi.workloads()[args.profile]
+    if isinstance(case, mi.DecodeCase):
+        r = bench_decode(case, args.steps, args.warmup, lambda: flush_buf.fill_(1), stream, 1)
+    else:
+        r = bench_prefill(case, args.steps, args.warmup, lambda: flush_buf.fill_(1), stream, False, 1)
+    print(json.dumps({"profile": args.profile, "ms": round(r["ms"], 5)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -437,10 +459,14 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--profile", default=None, choices=sorted(mi.workloads()),
+                    help="time one workload alone (for profiler captures) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.impl == "reference":
+    if args.profile:
+        run_profile(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)
