@@ -1,6 +1,6 @@
-"""The small-argument softcap polynomial (tanh_q2 in csrc/sm100.cuh) against its error bound:
-coefficients equal to csrc/fit_tanh_poly.py's fit, and an fp32 emulation of y * q(y^2) within
-1.5e-7 absolute (3e-7 relative) of tanh on |y| <= 0.625."""
+"""The small-argument softcap polynomial (kTanhQ*, tanh_q / tanh_q2 in csrc/sm100.cuh) against
+its error bound: coefficients equal to csrc/fit_tanh_poly.py's fit, and an fp32 emulation of
+y * q(y^2) within 1.5e-7 absolute (3e-7 relative) of tanh on |y| <= 0.625."""
 import importlib.util
 import os
 import re
@@ -40,3 +40,4 @@ def test_error_bound():
     assert np.max(np.abs(t - ref)) < 1.5e-7
     nz = ref != 0
     assert np.max(np.abs(t[nz] / ref[nz] - 1)) < 3e-7
+

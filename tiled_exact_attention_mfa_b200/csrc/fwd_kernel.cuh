@@ -66,6 +66,7 @@ struct FwdParams {
   float c_log2;     // factor taking the stored score to the log2 domain
   float softcap;    // 0 = off
   float cap_in;     // scale / softcap
+  float cap_out;    // softcap / scale
   float lse_mul;    // ln 2
 };
 
@@ -316,9 +317,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       float* s = reinterpret_cast<float*>(sraw);
 
       const int k0 = (kt_lo + j) * kFwdBN;
+      // Softcap: the capped score is cap * tanh(s * scale / cap); the value kept per key is that
+      // divided by scale, so the exponent factor c = scale * log2 e is the same as without a cap.
+      // When every |y| = |s| * scale / cap of this warp's rows is small, tanh(y) = y * q(y^2) is
+      // evaluated inside the exponential loop below (FMA work that fills the issue slots left
+      // while MUFU computes exponentials), and the row max is taken on the raw scores: tanh is
+      // increasing, so the kept max is the transform of the raw max. Otherwise every score is
+      // transformed here with tanh from exp2.
+      bool poly = false;
       if (p.softcap > 0.f) {
-        // s <- cap * tanh(s * scale / cap). When every |y| = |s| * scale / cap of this warp's
-        // rows is small, tanh(y) = y * q(y^2) on packed pairs; otherwise the exp form.
         float am8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) am8[i] = fmaxf(fabsf(s[i]), fabsf(s[i + 8]));
@@ -328,18 +335,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
           for (int k = 0; k < 8; ++k) am8[k] = max3(am8[k], fabsf(s[i + k]), fabsf(s[i + 8 + k]));
         const float amax = max3(max3(am8[0], am8[1], am8[2]), max3(am8[3], am8[4], am8[5]),
                                 fmaxf(am8[6], am8[7]));
-        if (__all_sync(0xffffffffu, amax * p.cap_in <= kTanhPolyMax)) {
-          const uint64_t ci = f2_pack(p.cap_in, p.cap_in);
-          const uint64_t cap = f2_pack(p.softcap, p.softcap);
+        poly = __all_sync(0xffffffffu, amax * p.cap_in <= kTanhPolyMax);
+        if (!poly) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const uint64_t y = f2_mul(f2_pack(s[2 * i], s[2 * i + 1]), ci);
-            const uint64_t t = f2_mul(f2_mul(y, tanh_q2(f2_mul(y, y))), cap);
-            f2_unpack(t, s[2 * i], s[2 * i + 1]);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 128; ++i) s[i] = p.softcap * tanh_from_exp(s[i] * p.cap_in);
+          for (int i = 0; i < 128; ++i) s[i] = p.cap_out * tanh_from_exp(s[i] * p.cap_in);
         }
       }
       // Element masks only where some row of this Q tile may not see some key of the tile.
@@ -364,7 +363,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       for (int i = 16; i < 128; i += 16)
 #pragma unroll
         for (int k = 0; k < 8; ++k) m8[k] = max3(m8[k], s[i + k], s[i + 8 + k]);
-      const float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+      float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+      if (poly && mx > -INFINITY) {
+        const float y = mx * p.cap_in;
+        mx = p.cap_out * (y * tanh_q(y * y));
+      }
 
       // Lazy rescale: move the reference max only when it grew by more than 2^8 in exp2 terms.
       const float m_new = fmaxf(m_run, mx);
@@ -405,34 +408,52 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       uint64_t acc[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[i] = f2_pack(0.f, 0.f);
+      // POLY: the kept value of a pair is tanh(y) * cap / scale with y = s * scale / cap, so
+      // x = tanh(y) * (cap log2 e) - m c; a masked score (-inf) gives y = -inf, q = +inf and
+      // x = -inf (the polynomial's leading coefficient is positive).
+      auto exponentials = [&](auto poly_tag) {
+        constexpr bool kPoly = decltype(poly_tag)::value;
+        const uint64_t ci2 = f2_pack(p.cap_in, p.cap_in);
+        const float cc = p.softcap * 1.4426950408889634f;
+        const uint64_t xc2 = kPoly ? f2_pack(cc, cc) : c2;
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t pk[16];
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int ii = ch * 16 + i;
-          const uint64_t x = f2_fma(f2_pack(s[2 * ii], s[2 * ii + 1]), c2, nm2);
-          uint64_t pp;
-          if (kPolyPair(ii)) {
-            pp = exp2_fma2(x);
-          } else {
-            float x0, x1;
-            f2_unpack(x, x0, x1);
-            pp = f2_pack(fast_exp2(x0), fast_exp2(x1));
+          for (int i = 0; i < 16; ++i) {
+            const int ii = ch * 16 + i;
+            uint64_t v = f2_pack(s[2 * ii], s[2 * ii + 1]);
+            if constexpr (kPoly) {
+              const uint64_t y = f2_mul(v, ci2);
+              v = f2_mul(y, tanh_q2(f2_mul(y, y)));
+            }
+            const uint64_t x = f2_fma(v, xc2, nm2);
+            uint64_t pp;
+            if (kPolyPair(ii)) {
+              pp = exp2_fma2(x);
+            } else {
+              float x0, x1;
+              f2_unpack(x, x0, x1);
+              pp = f2_pack(fast_exp2(x0), fast_exp2(x1));
+            }
+            acc[ii & 3] = f2_add(acc[ii & 3], pp);
+            float p0, p1;
+            f2_unpack(pp, p0, p1);
+            pk[i] = pack2<BF16>(p0, p1);
           }
-          acc[ii & 3] = f2_add(acc[ii & 3], pp);
-          float p0, p1;
-          f2_unpack(pp, p0, p1);
-          pk[i] = pack2<BF16>(p0, p1);
+          tmem_st16(t_s + ch * 16, pk);
+          if (ch & 1) {
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.bar_p_full[t][ch >> 1]));
+          }
         }
-        tmem_st16(t_s + ch * 16, pk);
-        if (ch & 1) {
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&sm.bar_p_full[t][ch >> 1]));
-        }
-      }
+      };
+      if (poly)
+        exponentials(std::integral_constant<bool, true>());
+      else
+        exponentials(std::integral_constant<bool, false>());
       float sa, sb;
       f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), sa, sb);
       l_run = l_run * alpha + (sa + sb);

@@ -162,14 +162,17 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, float* ls
     p.tile_counter = static_cast<unsigned long long*>(ctr);
   }
   const float log2e = 1.4426950408889634f;
+  // the kernel keeps (capped score) / scale per key, so the exponent factor is scale * log2 e
+  // with or without a cap
+  p.c_log2 = scale * log2e;
   if (softcap > 0.f) {
     p.softcap = softcap;
     p.cap_in = scale / softcap;
-    p.c_log2 = log2e;
+    p.cap_out = softcap / scale;
   } else {
     p.softcap = 0.f;
     p.cap_in = 0.f;
-    p.c_log2 = scale * log2e;
+    p.cap_out = 0.f;
   }
   p.lse_mul = 0.69314718055994531f;
   const long long grid = (long long)p.n_qblk * B * Hq;

@@ -2,6 +2,7 @@
 // mbarriers, TMA tiled / bulk copies, tcgen05 (TMEM alloc, MMA, commit, ld/st, fences),
 // warp-level mma.sync / ldmatrix for the decode path, and a bounded-wait helper.
 #pragma once
+#include <type_traits>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -358,7 +359,13 @@ constexpr float kTanhQ2 = 1.330818683e-01f;
 constexpr float kTanhQ3 = -5.194849521e-02f;
 constexpr float kTanhQ4 = 1.519625355e-02f;
 
-// q(u) for a pair of u values.
+// q(u) for one u and for a pair of u values.
+__device__ __forceinline__ float tanh_q(float u) {
+  float q = fmaf(kTanhQ4, u, kTanhQ3);
+  q = fmaf(q, u, kTanhQ2);
+  q = fmaf(q, u, kTanhQ1);
+  return fmaf(q, u, 1.0f);
+}
 __device__ __forceinline__ uint64_t tanh_q2(uint64_t u) {
   uint64_t q = f2_fma(f2_pack(kTanhQ4, kTanhQ4), u, f2_pack(kTanhQ3, kTanhQ3));
   q = f2_fma(q, u, f2_pack(kTanhQ2, kTanhQ2));
