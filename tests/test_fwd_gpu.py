@@ -108,8 +108,16 @@ def test_tile_skip_is_bitwise_neutral(cuda_device):
         assert np.array_equal(l1, l2), case.name
 
 
-def tiles_closed_form(case, bm=256, bn=128):
-    """Key tiles intersecting each 256-row block's visible set, counted on the mask itself."""
+def q_rows_per_cta():
+    """Query rows one CTA of the forward kernel covers (128 per Q tile), from its launch record."""
+    import tiled_exact_attention_mfa_b200 as mfa
+    info = mfa.mfa_last_launch_info()
+    assert info["kernel"] == 1
+    return info["tile_m"] * info["q_tiles_per_cta"]
+
+
+def tiles_closed_form(case, bm, bn=128):
+    """Key tiles intersecting each bm-row block's visible set, counted on the mask itself."""
     vis = oracle.visible(case.Nq, case.Nk, case.causal, case.win_l, case.win_r)
     n = 0
     for r0 in range(0, case.Nq, bm):
@@ -132,14 +140,15 @@ def test_visited_tile_count_matches_closed_form(cuda_device):
             got = mfa.mfa_debug_tiles_visited()
         finally:
             mfa.mfa_debug_set_flags(old)
-        assert got == tiles_closed_form(case), case.name
+        bm = q_rows_per_cta()
+        assert got == tiles_closed_form(case, bm), case.name
         old = mfa.mfa_debug_set_flags(mfa.MFA_DEBUG_COUNT_TILES | mfa.MFA_DEBUG_NO_TILE_SKIP)
         try:
             run_gpu(case, q, k, v)
             got = mfa.mfa_debug_tiles_visited()
         finally:
             mfa.mfa_debug_set_flags(old)
-        assert got == -(-case.Nq // 256) * -(-case.Nk // 128) * case.B * case.Hq
+        assert got == -(-case.Nq // bm) * -(-case.Nk // 128) * case.B * case.Hq
     torch.cuda.synchronize()
 
 
@@ -165,4 +174,6 @@ def test_launch_info_reports_the_prefill_kernel(cuda_device):
     run_gpu(case, *case.tensors())
     info = mfa.mfa_last_launch_info()
     assert info["kernel"] == 1 and info["tile_m"] == 128 and info["tile_n"] == 128
-    assert info["grid_x"] == 2 * 2  # ceil(300 / 256) query blocks x 2 heads
+    rows = 128 * info["q_tiles_per_cta"]
+    assert info["q_tiles_per_cta"] in (1, 2)
+    assert info["grid_x"] == -(-300 // rows) * 2  # query blocks x 2 heads
