@@ -23,7 +23,7 @@ _SRC = os.path.join(_HERE, "gen.c")
 
 FP16, BF16 = 0, 1
 DTYPE_NAMES = {FP16: "fp16", BF16: "bf16"}
-STREAM_Q, STREAM_K, STREAM_V, STREAM_LENS, STREAM_PERM = 0, 1, 2, 3, 4
+STREAM_Q, STREAM_K, STREAM_V, STREAM_LENS, STREAM_PERM, STREAM_KEXTRA = 0, 1, 2, 3, 4, 5
 PAGE_SIZE = 16
 
 
@@ -228,6 +228,70 @@ class DecodeCase:
         return q, k, v, table, lens
 
 
+@dataclass
+class VarlenCase:
+    """Packed variable-length prefill: B sequences in one tensor.
+
+    q [total_q, Hq, D], k/v [total_k, Hkv, D]; cu_seqlens_q / cu_seqlens_k int32 [B + 1].
+    Query lengths are uniform integers on [len_lo, len_hi] (stream 3); each key length is its
+    query length plus a uniform integer on [0, k_extra] (stream 5), the shape of a chunked
+    prefill that continues a cached prefix. fixed_q / fixed_k give the lengths explicitly.
+    """
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    D: int
+    dtype: int
+    causal: bool
+    len_lo: int = 1
+    len_hi: int = 1
+    k_extra: int = 0
+    win_l: int = -1
+    win_r: int = -1
+    softcap: float = 0.0
+    mul: float = 1.0
+    seed: int = 1
+    fixed_q: list | None = None
+    fixed_k: list | None = None
+    scale: float | None = None
+
+    def scale_f32(self) -> float:
+        s = self.scale if self.scale is not None else 1.0 / np.sqrt(self.D)
+        return float(np.float32(s))
+
+    def lens(self):
+        """(query lengths, key lengths), int32 [B] each."""
+        if self.fixed_q is not None:
+            nq = np.asarray(self.fixed_q, dtype=np.int32)
+        else:
+            nq = uniform_ints(self.seed, STREAM_LENS, self.B, self.len_lo, self.len_hi).astype(np.int32)
+        if self.fixed_k is not None:
+            nk = np.asarray(self.fixed_k, dtype=np.int32)
+        elif self.k_extra > 0:
+            nk = nq + uniform_ints(self.seed, STREAM_KEXTRA, self.B, 0, self.k_extra).astype(np.int32)
+        else:
+            nk = nq.copy()
+        return nq, nk
+
+    def cu_seqlens(self):
+        """(cu_seqlens_q, cu_seqlens_k), int32 [B + 1] each, starting at 0."""
+        nq, nk = self.lens()
+        cq = np.zeros(self.B + 1, dtype=np.int32)
+        ck = np.zeros(self.B + 1, dtype=np.int32)
+        cq[1:] = np.cumsum(nq)
+        ck[1:] = np.cumsum(nk)
+        return cq, ck
+
+    def tensors(self):
+        """(q, k, v) as uint16 bit patterns in the packed layout."""
+        cq, ck = self.cu_seqlens()
+        q = normal_bits(self.seed, STREAM_Q, (int(cq[-1]), self.Hq, self.D), self.dtype, self.mul)
+        k = normal_bits(self.seed, STREAM_K, (int(ck[-1]), self.Hkv, self.D), self.dtype, self.mul)
+        v = normal_bits(self.seed, STREAM_V, (int(ck[-1]), self.Hkv, self.D), self.dtype, self.mul)
+        return q, k, v
+
+
 def workloads():
     """The named full-size workloads (shapes, flags, seeds and value scales)."""
     return {
@@ -246,6 +310,9 @@ def workloads():
         "gqa_causal_b1_hq32_hkv8_n16384_d128_bf16_cap50": PrefillCase(
             "gqa_causal_b1_hq32_hkv8_n16384_d128_bf16_cap50", 1, 32, 8, 16384, 16384, 128, BF16,
             True, softcap=50.0, mul=0.5, seed=1004),
+        "varlen_causal_b8_h8_d128_fp16_len512_8k": VarlenCase(
+            "varlen_causal_b8_h8_d128_fp16_len512_8k", 8, 8, 8, 128, FP16, True, 512, 8192,
+            seed=1006),
         "decode_b8_hq32_hkv8_d128_bf16_len8k_128k": DecodeCase(
             "decode_b8_hq32_hkv8_d128_bf16_len8k_128k", 8, 1, 32, 8, 128, BF16, 8192, 131072,
             seed=1005),

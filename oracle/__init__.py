@@ -18,7 +18,10 @@ Sources (web pages, cited by title and section):
     with -1 meaning unbounded, native GQA without repeating K/V, tanh softcap (softcap=50.0),
     paged KV with a block_table, two-phase split-KV decode for N_q <= 4.
   * "mxflashattn 1.4.0 -> 1.5.0" (diffend), README: paged decode reads a paged KV cache with
-    page size 16 and GQA 4.
+    page size 16 and GQA 4; public entry points include a varlen forward.
+  * "mlx-mfa 2.5.2" Features: variable-length packed sequences with cu_seqlens; "mlx-mfa
+    2.61.0" (essential correctness update): varlen causal with N_q < N_k changed toward the
+    bottom-right alignment used here per sequence.
 
 Readings where the pages are silent or ambiguous (each restated in the design doc):
   * window: key j is visible from absolute query position a iff a - win_l <= j <= a + win_r
@@ -35,7 +38,8 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["visible", "attention", "attention_rows", "paged_gather", "decode", "decode_rows"]
+__all__ = ["visible", "attention", "attention_rows", "attention_varlen", "attention_varlen_rows",
+           "paged_gather", "decode", "decode_rows"]
 
 
 def visible(Nq: int, Nk: int, causal: bool, win_l: int = -1, win_r: int = -1) -> np.ndarray:
@@ -122,6 +126,53 @@ def attention_rows(q, k, v, rows, scale, causal=False, win_l=-1, win_r=-1, softc
         qi = np.asarray(q[b, h, i:i + 1], dtype=np.float64)
         oi, li = _rows_for_head(qi, np.asarray(k[b, g], dtype=np.float64),
                                 np.asarray(v[b, g], dtype=np.float64), vis[None, :], scale, softcap)
+        o[n], lse[n] = oi[0], li[0]
+    return o, lse
+
+
+def _sequence_views(q, k, v, cu_q, cu_k, b):
+    """Sequence b of a packed batch as [1, H, N, D] arrays (q [total_q, Hq, D] -> [1, Hq, Nq_b, D])."""
+    q0, q1 = int(cu_q[b]), int(cu_q[b + 1])
+    k0, k1 = int(cu_k[b]), int(cu_k[b + 1])
+    qs = np.asarray(q[q0:q1], dtype=np.float64).transpose(1, 0, 2)[None]
+    ks = np.asarray(k[k0:k1], dtype=np.float64).transpose(1, 0, 2)[None]
+    vs = np.asarray(v[k0:k1], dtype=np.float64).transpose(1, 0, 2)[None]
+    return qs, ks, vs
+
+
+def attention_varlen(q, k, v, cu_q, cu_k, scale, causal=False, win_l=-1, win_r=-1, softcap=0.0):
+    """Packed variable-length forward: sequence b (rows cu_q[b]..cu_q[b+1] of q, cu_k[b]..cu_k[b+1]
+    of k / v) is attended on its own with the dense definition, bottom-right aligned per
+    sequence. q [total_q, Hq, D], k/v [total_k, Hkv, D]. Returns (o [total_q, Hq, D],
+    lse [Hq, total_q])."""
+    total_q, Hq, D = np.shape(q)
+    o = np.zeros((total_q, Hq, D))
+    lse = np.full((Hq, total_q), -np.inf)
+    for b in range(len(cu_q) - 1):
+        q0, q1 = int(cu_q[b]), int(cu_q[b + 1])
+        if q1 == q0:
+            continue
+        qs, ks, vs = _sequence_views(q, k, v, cu_q, cu_k, b)
+        ob, lb = attention(qs, ks, vs, scale, causal, win_l, win_r, softcap)
+        o[q0:q1] = ob[0].transpose(1, 0, 2)
+        lse[:, q0:q1] = lb[0]
+    return o, lse
+
+
+def attention_varlen_rows(q, k, v, cu_q, cu_k, rows, scale, causal=False, win_l=-1, win_r=-1,
+                          softcap=0.0):
+    """Selected rows of the packed forward. rows: int array [n, 2] of (h, packed row r).
+    Returns (o [n, D], lse [n])."""
+    rows = np.asarray(rows, dtype=np.int64).reshape(-1, 2)
+    D = np.shape(q)[2]
+    o = np.zeros((len(rows), D))
+    lse = np.full(len(rows), -np.inf)
+    cu_q = np.asarray(cu_q, dtype=np.int64)
+    for n, (h, r) in enumerate(rows):
+        b = int(np.searchsorted(cu_q, r, side="right") - 1)   # sequence holding packed row r
+        qs, ks, vs = _sequence_views(q, k, v, cu_q, cu_k, b)
+        oi, li = attention_rows(qs, ks, vs, [(0, h, r - cu_q[b])], scale, causal, win_l, win_r,
+                                softcap)
         o[n], lse[n] = oi[0], li[0]
     return o, lse
 

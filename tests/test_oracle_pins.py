@@ -309,3 +309,94 @@ def test_decode_rows_helper_matches_pinned_decode():
     for n, (b, h, t) in enumerate(rows):
         np.testing.assert_allclose(o2[n], o[b, h, t], rtol=0, atol=1e-14)
         assert l2[n] == pytest.approx(lse[b, h, t], abs=1e-14)
+
+
+# ---------------------------------------------------------------- packed variable-length batches
+VARLEN = [
+    # Hq, Hkv, D, query lengths, key lengths, causal, win_l, win_r
+    (4, 2, 8, [5, 0, 17, 9], [5, 3, 30, 9], True, -1, -1),
+    (2, 2, 8, [12, 7, 1], [20, 7, 4], False, 3, 2),
+    (6, 3, 4, [8, 8], [2, 0], True, 4, 0),
+]
+
+
+def _packed(lens, H, D):
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    return cu, rng.standard_normal((int(cu[-1]), H, D))
+
+
+@pytest.mark.parametrize("case", VARLEN)
+def test_varlen_matches_torch_sdpa_per_sequence(case):
+    """Each sequence of the packed batch against torch's SDPA on that sequence alone, with the
+    bottom-right band mask built from torch.tril / torch.triu at its own Nq, Nk."""
+    Hq, Hkv, D, nq, nk, causal, wl, wr = case
+    cq, q = _packed(nq, Hq, D)
+    ck, k = _packed(nk, Hkv, D)
+    v = rng.standard_normal(k.shape)
+    o, lse = oracle.attention_varlen(q, k, v, cq, ck, 0.41, causal, wl, wr)
+    assert o.shape == q.shape and lse.shape == (Hq, cq[-1])
+    for b in range(len(nq)):
+        if nq[b] == 0:
+            continue
+        qs = q[cq[b]:cq[b + 1]].transpose(1, 0, 2)[None]
+        ks = k[ck[b]:ck[b + 1]].transpose(1, 0, 2)[None]
+        vs = v[ck[b]:ck[b + 1]].transpose(1, 0, 2)[None]
+        ob = o[cq[b]:cq[b + 1]].transpose(1, 0, 2)[None]
+        lb = lse[:, cq[b]:cq[b + 1]][None]
+        if nk[b] == 0:
+            assert np.all(ob == 0) and np.all(np.isneginf(lb))
+            continue
+        mask = band_mask_torch(nq[b], nk[b], causal, wl, wr)
+        has = mask.any(dim=1).numpy()
+        ref = sdpa_ref(qs, ks, vs, 0.41, mask)
+        np.testing.assert_allclose(ob[:, :, has], ref[:, :, has], rtol=0, atol=1e-12)
+        assert np.all(ob[:, :, ~has] == 0) and np.all(np.isneginf(lb[:, :, ~has]))
+
+
+def test_varlen_zero_query_lse_is_log_count_per_sequence():
+    """Q = 0 in every sequence: LSE of packed row r of sequence b = ln(#keys visible at its own
+    bottom-right offset) — pins the per-sequence offsets and lengths."""
+    nq, nk = [7, 30, 1, 0, 12], [9, 30, 40, 5, 3]
+    cq, _ = _packed(nq, 2, 4)
+    ck, k = _packed(nk, 2, 4)
+    q = np.zeros((int(cq[-1]), 2, 4))
+    v = rng.standard_normal(k.shape)
+    for causal, wl, wr in ((True, -1, -1), (True, 5, 0), (False, 2, 6)):
+        _, lse = oracle.attention_varlen(q, k, v, cq, ck, 0.7, causal, wl, wr)
+        for b in range(len(nq)):
+            cnt = closed_form_count(nq[b], nk[b], causal, wl, wr)
+            for i in range(nq[b]):
+                got = lse[:, cq[b] + i]
+                if cnt[i] == 0:
+                    assert np.all(np.isneginf(got))
+                else:
+                    np.testing.assert_allclose(got, math.log(cnt[i]), rtol=0, atol=1e-13)
+
+
+def test_varlen_sequences_do_not_see_each_other():
+    """Changing one sequence's K / V leaves every other sequence's output bitwise unchanged."""
+    nq, nk = [6, 9, 4], [6, 11, 4]
+    cq, q = _packed(nq, 2, 8)
+    ck, k = _packed(nk, 2, 8)
+    v = rng.standard_normal(k.shape)
+    o1, l1 = oracle.attention_varlen(q, k, v, cq, ck, 0.3, True)
+    k2, v2 = k.copy(), v.copy()
+    k2[ck[1]:ck[2]] += 5.0
+    v2[ck[1]:ck[2]] *= -3.0
+    o2, l2 = oracle.attention_varlen(q, k2, v2, cq, ck, 0.3, True)
+    for b in (0, 2):
+        assert np.array_equal(o1[cq[b]:cq[b + 1]], o2[cq[b]:cq[b + 1]])
+        assert np.array_equal(l1[:, cq[b]:cq[b + 1]], l2[:, cq[b]:cq[b + 1]])
+    assert not np.allclose(o1[cq[1]:cq[2]], o2[cq[1]:cq[2]])
+
+
+def test_varlen_rows_helper_matches_full():
+    nq, nk = [5, 13, 2], [8, 13, 20]
+    cq, q = _packed(nq, 4, 8)
+    ck, k = _packed(nk, 2, 8)
+    v = rng.standard_normal(k.shape)
+    o, lse = oracle.attention_varlen(q, k, v, cq, ck, 0.5, True, 6, -1, softcap=2.0)
+    rows = np.array([(h, r) for h in range(4) for r in range(int(cq[-1]))])
+    orow, lrow = oracle.attention_varlen_rows(q, k, v, cq, ck, rows, 0.5, True, 6, -1, softcap=2.0)
+    np.testing.assert_allclose(orow, o[rows[:, 1], rows[:, 0]], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lrow, lse[rows[:, 0], rows[:, 1]], rtol=0, atol=1e-13)
