@@ -4,8 +4,8 @@ python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mfa|reference] [--wo
 
 One step = one pass of the hot path over one batch: the prefill forward of the named workload
 (default: causal, B=2, H=8, N=4096, D=128, fp16). The same JSON line also carries the other
-workloads (non-causal, sliding window, GQA + softcap prefill, paged split-KV decode), each timed
-the same way. Inputs are seeded synthetic tensors resident in HBM; L2 is flushed (a 256 MiB
+workloads (non-causal, sliding window, GQA + softcap prefill, packed variable-length prefill,
+paged split-KV decode), each timed the same way. Inputs are seeded synthetic tensors resident in HBM; L2 is flushed (a 256 MiB
 write) before every timed step, outside the timed kernel. Times are CUDA events on the launching
 stream; with N > 1 (torchrun) every rank runs its own copy of the workload (weak scaling) and the
 max over ranks is reported.
@@ -37,12 +37,14 @@ L2_FLUSH_BYTES = 256 << 20
 
 
 # --------------------------------------------------------------------------- work accounting
-def visible_pairs(case) -> int:
+def visible_pairs(case, Nq=None, Nk=None) -> int:
     """Visible (query, key) pairs of one head, summed row by row from the interval form."""
-    i = np.arange(case.Nq, dtype=np.int64)
-    a = i + (case.Nk - case.Nq)
+    Nq = case.Nq if Nq is None else int(Nq)
+    Nk = case.Nk if Nk is None else int(Nk)
+    i = np.arange(Nq, dtype=np.int64)
+    a = i + (Nk - Nq)
     lo = np.zeros_like(a) if case.win_l < 0 else np.maximum(0, a - case.win_l)
-    hi = np.full_like(a, case.Nk - 1)
+    hi = np.full_like(a, Nk - 1)
     if case.causal:
         hi = np.minimum(hi, a)
     if case.win_r >= 0:
@@ -58,6 +60,17 @@ def prefill_bytes(case) -> float:
     e = 2
     return (e * case.B * case.Hq * case.Nq * case.D * 2 + e * 2 * case.B * case.Hkv * case.Nk * case.D
             + 4 * case.B * case.Hq * case.Nq)
+
+
+def varlen_flops(case) -> float:
+    nq, nk = case.lens()
+    return 4.0 * case.D * case.Hq * sum(visible_pairs(case, a, b) for a, b in zip(nq, nk))
+
+
+def varlen_bytes(case) -> float:
+    nq, nk = case.lens()
+    tq, tk = int(nq.sum()), int(nk.sum())
+    return 2 * tq * case.Hq * case.D * 2 + 2 * 2 * tk * case.Hkv * case.D + 4 * tq * case.Hq
 
 
 def decode_bytes(case, lens) -> float:
@@ -240,6 +253,30 @@ def bench_prefill(case, steps, warmup, flush, stream, with_e2e, world):
     return res
 
 
+def bench_varlen(case, steps, warmup, flush, stream, world):
+    import torch
+    import tiled_exact_attention_mfa_b200 as mfa
+    dev = torch.device("cuda")
+    q, k, v = case.tensors()
+    cq, ck = case.cu_seqlens()
+    qt, kt, vt = (upload(x, case.dtype, dev) for x in (q, k, v))
+    cqt, ckt = torch.from_numpy(cq).to(dev), torch.from_numpy(ck).to(dev)
+    out = torch.empty_like(qt)
+    lse = torch.empty(case.Hq, qt.shape[0], dtype=torch.float32, device=dev)
+    max_q = int(case.lens()[0].max())
+    scale = case.scale_f32()
+
+    def step():
+        mfa.mfa_fwd_varlen(qt, kt, vt, cqt, ckt, max_q, out, lse, scale=scale, causal=case.causal,
+                           window=(case.win_l, case.win_r), softcap=case.softcap, stream=stream)
+
+    with torch.cuda.stream(stream):
+        ms, bracket = time_steps(step, steps, warmup, flush, stream)
+    return {"ms": max_over_ranks(statistics.mean(ms), world), "ms_min": min(ms),
+            "bracket_ms": bracket, "flops": varlen_flops(case), "bytes": varlen_bytes(case),
+            "total_q": int(cq[-1])}
+
+
 def bench_decode(case, steps, warmup, flush, stream, world):
     import torch
     import tiled_exact_attention_mfa_b200 as mfa
@@ -302,7 +339,18 @@ def run_gpu(args):
             if name == args.workload:
                 continue
             sk, wu = max(3, min(args.steps, 10)), max(3, args.warmup)
-            if isinstance(case, mi.DecodeCase):
+            if isinstance(case, mi.VarlenCase):
+                r = bench_varlen(case, sk, wu, flush, stream, world)
+                tf = r["flops"] * world / (r["ms"] * 1e-3) / 1e12
+                gbs = r["bytes"] * world / (r["ms"] * 1e-3) / 1e9
+                t_floor = max(r["flops"] / (pk["tflops"] * 1e12), r["bytes"] / (pk["gbs"] * 1e9))
+                others.append({"workload": name, "ms": round(r["ms"], 4), "unit": "TFLOP/s",
+                               "value": round(tf, 1), "GB/s": round(gbs, 1),
+                               "total_q": r["total_q"],
+                               "frac_of_measured_tensor_peak": round(tf / pk["tflops"], 4),
+                               "frac_of_nominal_tensor_peak": round(tf / NOMINAL_TFLOPS, 4),
+                               "frac_of_roofline": round(t_floor / (r["ms"] * 1e-3), 4)})
+            elif isinstance(case, mi.DecodeCase):
                 r = bench_decode(case, sk, wu, flush, stream, world)
                 tb = r["bytes"] * world / (r["ms"] * 1e-3) / 1e9
                 others.append({"workload": name, "ms": round(r["ms"], 4), "unit": "GB/s",
@@ -442,6 +490,8 @@ def run_profile(args):
     case = mi.workloads()[args.profile]
     if isinstance(case, mi.DecodeCase):
         r = bench_decode(case, args.steps, args.warmup, lambda: flush_buf.fill_(1), stream, 1)
+    elif isinstance(case, mi.VarlenCase):
+        r = bench_varlen(case, args.steps, args.warmup, lambda: flush_buf.fill_(1), stream, 1)
     else:
         r = bench_prefill(case, args.steps, args.warmup, lambda: flush_buf.fill_(1), stream, False, 1)
     print(json.dumps({"profile": args.profile, "ms": round(r["ms"], 5)}), flush=True)

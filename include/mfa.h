@@ -1,9 +1,10 @@
 /*
  * mfa.h -- C ABI of libmfa.so: exact tiled scaled-dot-product attention on B200 (sm_100a).
  *
- * Two operations:
+ * Operations:
  *   mfa_fwd            dense forward with online softmax: causal and sliding-window tile skip,
  *                      native GQA, optional tanh softcap, optional fp32 log-sum-exp output.
+ *   mfa_fwd_varlen     the same forward over packed variable-length sequences (cu_seqlens).
  *   mfa_decode_splitkv two-phase split-KV decode (N_q <= 4) over a paged KV cache.
  *
  * Sources (web pages, cited by title and section):
@@ -65,6 +66,8 @@ extern "C" {
 #define MFA_ERR_DEVICE_TIMEOUT     -21   /* device status: a bounded wait inside a kernel ran out */
 #define MFA_ERR_DEVICE_BAD_PAGE    -22   /* device status: a block_table entry was outside [0, num_pages) */
 #define MFA_ERR_SCRATCH_TOO_SMALL  -23   /* mfa_decode_splitkv_noalloc: shape needs more than its fixed scratch */
+#define MFA_ERR_DEVICE_BAD_SEQLENS -24   /* device status: a cu_seqlens entry was negative, decreasing or past
+                                            the packed total, or a sequence was longer than max_seqlen_q */
 
 /*
  * mfa_fwd -- exact attention forward (prefill).
@@ -92,6 +95,35 @@ extern "C" {
 int mfa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
             int B, int Hq, int Hkv, int Nq, int Nk, int D, float scale,
             int causal, int win_l, int win_r, float softcap, int dtype, void* stream);
+
+/*
+ * mfa_fwd_varlen -- the same forward over a packed batch of variable-length sequences
+ * ([MFA252] Features "Variable-length -- packed sequences with cu_seqlens"; [MXFA15] README
+ * public entry point flash_attn_varlen_func; [MFA261] 2.61.0 notes that varlen causal with
+ * N_q < N_k was changed toward bottom-right alignment, which this call follows per sequence).
+ *
+ * Sequence b has Nq_b = cu_seqlens_q[b+1] - cu_seqlens_q[b] query rows, stored at rows
+ * cu_seqlens_q[b] ... of q and out, and Nk_b = cu_seqlens_k[b+1] - cu_seqlens_k[b] keys at rows
+ * cu_seqlens_k[b] ... of k and v. Every sequence is attended exactly as mfa_fwd attends one
+ * batch entry with Nq = Nq_b, Nk = Nk_b (a = i + Nk_b - Nq_b; keys of other sequences are never
+ * visible); a sequence with Nk_b = 0 gets out = 0, lse = -inf.
+ *
+ * Arguments
+ *   q    [total_q, Hq, D]  dtype      k, v [total_k, Hkv, D]  dtype          (read only)
+ *   out  [total_q, Hq, D]  dtype      lse  [Hq, total_q] float32, or NULL
+ *   cu_seqlens_q, cu_seqlens_k: int32 [B + 1] device arrays, 4-byte aligned, starting at 0,
+ *   non-decreasing, ending at total_q / total_k;
+ *   max_seqlen_q >= every Nq_b (it sizes the grid); other arguments as mfa_fwd.
+ * The offsets live on the device, so they are checked by the kernel: a malformed entry or a
+ * sequence longer than max_seqlen_q records MFA_ERR_DEVICE_BAD_SEQLENS (mfa_device_status) and
+ * the affected sequence's outputs are not written. Returns MFA_OK after the launch was queued,
+ * or a negative status (nothing launched).
+ */
+int mfa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
+                   const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                   int B, int max_seqlen_q, int total_q, int total_k,
+                   int Hq, int Hkv, int D, float scale,
+                   int causal, int win_l, int win_r, float softcap, int dtype, void* stream);
 
 /*
  * mfa_decode_workspace_size -- bytes of scratch mfa_decode_splitkv needs for this shape.

@@ -79,6 +79,31 @@ def test_fwd_empty_problem_is_noop():
     assert fwd(Nq=0, q=None, k=None, v=None, out=None) == 0
 
 
+def fwd_varlen(**kw):
+    args = dict(q=A, k=A, v=A, out=A, lse=A, cu_q=A, cu_k=A, B=3, max_q=100, total_q=200,
+                total_k=300, Hq=8, Hkv=2, D=128, scale=0.125, causal=1, win_l=-1, win_r=-1,
+                softcap=0.0, dtype=0, stream=None)
+    args.update(kw)
+    return mfa.lib.mfa_fwd_varlen(*args.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=2), -3), (dict(D=32), -4), (dict(B=-1), -5), (dict(total_k=-1), -5),
+    (dict(max_q=-1), -5), (dict(max_q=201), -5), (dict(Hkv=3), -6), (dict(win_l=-3), -7),
+    (dict(softcap=float("nan")), -8), (dict(scale=0.0), -9), (dict(cu_q=None), -1),
+    (dict(cu_k=None), -1), (dict(k=None), -1), (dict(cu_q=A + 2), -2), (dict(out=A + 8), -2),
+])
+@no_device
+def test_fwd_varlen_rejects_malformed(kw, code):
+    assert fwd_varlen(**kw) == code
+
+
+@no_device
+def test_fwd_varlen_empty_problem_is_noop():
+    assert fwd_varlen(B=0, q=None, k=None, v=None, out=None, cu_q=None, cu_k=None) == 0
+    assert fwd_varlen(total_q=0, max_q=0, q=None, out=None) == 0
+
+
 def dec(**kw):
     ws = kw.pop("ws_bytes", 1 << 30)
     args = dict(q=A, k=A, v=A, table=A, lens=A, out=A, lse=A, B=8, Nq=1, Hq=32, Hkv=8, D=128,

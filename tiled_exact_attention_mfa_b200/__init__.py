@@ -32,6 +32,8 @@ _f = ctypes.c_float
 
 lib.mfa_fwd.restype = _i
 lib.mfa_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _i, _f, _i, _vp]
+lib.mfa_fwd_varlen.restype = _i
+lib.mfa_fwd_varlen.argtypes = [_vp] * 7 + [_i] * 7 + [_f, _i, _i, _i, _f, _i, _vp]
 lib.mfa_decode_workspace_size.restype = ctypes.c_size_t
 lib.mfa_decode_workspace_size.argtypes = [_i] * 7
 lib.mfa_decode_splitkv.restype = _i
@@ -65,7 +67,7 @@ lib.mfa_debug_tiles_visited.argtypes = [_vp, ctypes.POINTER(ctypes.c_ulonglong)]
 lib.mfa_debug_set_decode_split_pages.restype = _i
 lib.mfa_debug_set_decode_split_pages.argtypes = [_i]
 
-EXPORTED = ("mfa_fwd", "mfa_decode_workspace_size", "mfa_decode_splitkv", "mfa_status_string",
+EXPORTED = ("mfa_fwd", "mfa_fwd_varlen", "mfa_decode_workspace_size", "mfa_decode_splitkv", "mfa_status_string",
             "mfa_last_launch_info", "mfa_device_status", "mfa_debug_set_flags",
             "mfa_debug_tiles_visited", "mfa_debug_set_decode_split_pages",
             "mfa_decode_splitkv_noalloc")
@@ -225,3 +227,36 @@ def mfa_debug_tiles_visited(stream=None) -> int:
 
 def mfa_debug_set_decode_split_pages(pages: int) -> int:
     return lib.mfa_debug_set_decode_split_pages(pages)
+
+
+def mfa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, out=None, lse=None, *,
+                   scale=None, causal=False, window=(-1, -1), softcap=0.0, return_lse=True,
+                   stream=None):
+    """Packed variable-length forward. q [total_q,Hq,D], k/v [total_k,Hkv,D], cu_seqlens_* int32
+    [B+1] on the device; returns (out [total_q,Hq,D], lse [Hq,total_q] or None)."""
+    torch = _torch()
+    total_q, Hq, D = q.shape
+    total_k, Hkv, _ = k.shape
+    if k.shape != v.shape or k.shape[2] != D:
+        raise ValueError("k and v must be [total_k, Hkv, D] matching q")
+    if q.dtype != k.dtype or q.dtype != v.dtype:
+        raise TypeError("q, k and v must share one dtype")
+    for c in (cu_seqlens_q, cu_seqlens_k):
+        if c.dtype != torch.int32 or c.dim() != 1:
+            raise TypeError("cu_seqlens must be 1-D int32 tensors")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both hold B + 1 offsets")
+    B = cu_seqlens_q.numel() - 1
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    wl, wr = window
+    rc = lib.mfa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q),
+                            _ptr(cu_seqlens_k), B, int(max_seqlen_q), total_q, total_k, Hq, Hkv, D,
+                            float(scale), int(bool(causal)), int(wl), int(wr), float(softcap),
+                            _dtype_code(q), _stream(stream))
+    _check(rc, "mfa_fwd_varlen")
+    return out, lse

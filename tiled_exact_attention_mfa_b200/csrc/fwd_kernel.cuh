@@ -59,6 +59,11 @@ struct FwdParams {
   void* out;
   float* lse;
   unsigned long long* tile_counter;
+  // packed variable-length batches: sequence b holds rows [cu_q[b], cu_q[b+1]) of q / out and
+  // [cu_k[b], cu_k[b+1]) of k / v (device arrays of B + 1 offsets); NULL for the dense layout
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
   int B, Hq, Hkv, Nq, Nk, G;
   int causal, win_l, win_r;
   int n_qblk;       // number of 256-row query blocks per head
@@ -93,16 +98,19 @@ constexpr int fwd_smem_bytes() {
   return (int)sizeof(FwdSmem<D>) + 1024;  // + alignment slack for the 1024-byte swizzle atoms
 }
 
-// Visible key range [lo, hi) of absolute query positions [a0, a1] (inclusive).
-__device__ __forceinline__ void key_range(const FwdParams& p, int a0, int a1, int& lo, int& hi) {
+// Visible key range [lo, hi) of absolute query positions [a0, a1] (inclusive) among Nk keys.
+__device__ __forceinline__ void key_range(const FwdParams& p, int Nk, int a0, int a1, int& lo, int& hi) {
   lo = 0;
-  hi = p.Nk;
+  hi = Nk;
   if (p.causal) hi = min(hi, a1 + 1);
   if (p.win_r >= 0) hi = min(hi, a1 + p.win_r + 1);
   if (p.win_l >= 0) lo = max(lo, a0 - p.win_l);
 }
 
-template <int D, bool BF16>
+// VARLEN: q / out are [total_q, Hq, D] and k / v [total_k, Hkv, D] with per-sequence offsets
+// (cu_q, cu_k), read through tensor maps ordered (D, head, token); lse is [Hq, total_q]. Otherwise q / out are [B, Hq, Nq, D], k / v
+// [B, Hkv, Nk, D] and lse [B, Hq, Nq].
+template <int D, bool BF16, bool VARLEN>
 __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_constant__ FwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   FwdSmem<D>& sm = *reinterpret_cast<FwdSmem<D>*>(
@@ -119,14 +127,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
   const int h = bh % p.Hq;
   const int g = h / p.G;
   const int q0 = qb * (kFwdBM * kFwdQT);
-  const int off = p.Nk - p.Nq;
-  const int q_last = min(q0 + kFwdBM * kFwdQT, p.Nq) - 1;
+  int Nq = p.Nq, Nk = p.Nk;  // this sequence's query and key counts
+  int rq = 0, rk = 0;        // its first row in the packed q / k (VARLEN)
+  if constexpr (VARLEN) {
+    rq = p.cu_q[b];
+    rk = p.cu_k[b];
+    const int eq = p.cu_q[b + 1], ek = p.cu_k[b + 1];
+    if (rq < 0 || eq < rq || eq > p.total_q || rk < 0 || ek < rk || ek > p.total_k) {
+      if (threadIdx.x == 0 && qb == 0 && h == 0) record_status(-24, b);
+      return;  // the whole CTA, before any barrier or TMEM allocation
+    }
+    Nq = eq - rq;
+    Nk = ek - rk;
+    // rows past the grid's query blocks would never be computed: report the short max_seqlen_q
+    if (threadIdx.x == 0 && qb == p.n_qblk - 1 && h == 0 && Nq > p.n_qblk * kFwdBM * kFwdQT)
+      record_status(-24, b);
+    if (q0 >= Nq) return;  // a shorter sequence has fewer query blocks
+  }
+  const int off = Nk - Nq;
+  const int q_last = min(q0 + kFwdBM * kFwdQT, Nq) - 1;
 
   int lo, hi;
-  key_range(p, q0 + off, q_last + off, lo, hi);
+  key_range(p, Nk, q0 + off, q_last + off, lo, hi);
   if (p.flags & 1) {
     lo = 0;
-    hi = p.Nk;
+    hi = Nk;
   }
   const int kt_lo = lo / kFwdBN;
   const int n_tiles = (hi > lo) ? ((hi + kFwdBN - 1) / kFwdBN - kt_lo) : 0;
@@ -179,8 +204,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       mbar_expect_tx(bq, kFwdQT * kTileBytes);
       for (int t = 0; t < kFwdQT; ++t)
         for (int sl = 0; sl < kSlabs; ++sl)
-          tma_load_3d(smem_u32(sm.q[t]) + sl * kSlab, &p.tm_q, bq, sl * 64, q0 + t * kFwdBM,
-                      b * p.Hq + h);
+          if constexpr (VARLEN)
+            tma_load_3d(smem_u32(sm.q[t]) + sl * kSlab, &p.tm_q, bq, sl * 64, h, rq + q0 + t * kFwdBM);
+          else
+            tma_load_3d(smem_u32(sm.q[t]) + sl * kSlab, &p.tm_q, bq, sl * 64, q0 + t * kFwdBM,
+                        b * p.Hq + h);
       int issued_k[kFwdStages] = {0, 0}, issued_v[kFwdStages] = {0, 0};
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j % kFwdStages;
@@ -190,13 +218,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         const uint32_t bk = smem_u32(&sm.bar_k_full[s]);
         mbar_expect_tx(bk, kTileBytes);
         for (int sl = 0; sl < kSlabs; ++sl)
-          tma_load_3d(smem_u32(sm.k[s]) + sl * kSlab, &p.tm_k, bk, sl * 64, row, b * p.Hkv + g);
+          tma_load_3d(smem_u32(sm.k[s]) + sl * kSlab, &p.tm_k, bk, sl * 64, VARLEN ? g : row,
+                      VARLEN ? rk + row : b * p.Hkv + g);
         issued_k[s] = use + 1;
         if (use > 0 && !mbar_wait(smem_u32(&sm.bar_v_empty[s]), (use - 1) & 1, abort, 802)) break;
         const uint32_t bv = smem_u32(&sm.bar_v_full[s]);
         mbar_expect_tx(bv, kTileBytes);
         for (int sl = 0; sl < kSlabs; ++sl)
-          tma_load_3d(smem_u32(sm.v[s]) + sl * kSlab, &p.tm_v, bv, sl * 64, row, b * p.Hkv + g);
+          tma_load_3d(smem_u32(sm.v[s]) + sl * kSlab, &p.tm_v, bv, sl * 64, VARLEN ? g : row,
+                      VARLEN ? rk + row : b * p.Hkv + g);
         issued_v[s] = use + 1;
       }
       // Make sure no copy into this CTA's shared memory is still in flight when it exits.
@@ -342,13 +372,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         }
       }
       // Element masks only where some row of this Q tile may not see some key of the tile.
-      bool interior = (k0 + kFwdBN <= p.Nk);
+      bool interior = (k0 + kFwdBN <= Nk);
       if (p.causal) interior = interior && (k0 + kFwdBN - 1 <= a_lo);
       if (p.win_r >= 0) interior = interior && (k0 + kFwdBN - 1 <= a_lo + p.win_r);
       if (p.win_l >= 0) interior = interior && (k0 >= a_hi - p.win_l);
       if (p.flags & 1) interior = false;
       if (!interior) {
-        int jhi = p.Nk - k0;                                   // keys >= Nk
+        int jhi = Nk - k0;                                     // keys >= Nk
         if (p.causal) jhi = min(jhi, a - k0 + 1);
         if (p.win_r >= 0) jhi = min(jhi, a + p.win_r - k0 + 1);
         const int jlo = (p.win_l >= 0) ? (a - p.win_l - k0) : -1;
@@ -469,8 +499,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     have_o = __all_sync(0xffffffffu, have_o);
     {
     }
-    const bool valid = row < p.Nq;
-    const size_t obase = ((size_t)(b * p.Hq + h) * p.Nq + (size_t)row) * D;
+    const bool valid = row < Nq;
+    const size_t orow = VARLEN ? (size_t)(rq + row) * p.Hq + h : (size_t)(b * p.Hq + h) * Nq + row;
+    const size_t obase = orow * D;
     const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
 #pragma unroll
     for (int cb = 0; cb < D; cb += 32) {
@@ -496,7 +527,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       }
     }
     if (valid && p.lse != nullptr) {
-      p.lse[(size_t)(b * p.Hq + h) * p.Nq + row] =
+      p.lse[VARLEN ? (size_t)h * p.total_q + rq + row : (size_t)(b * p.Hq + h) * Nq + row] =
           (l_run > 0.f) ? (m_run * c + log2f(l_run)) * p.lse_mul : -INFINITY;
     }
   }

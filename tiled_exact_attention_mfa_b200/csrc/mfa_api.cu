@@ -58,6 +58,22 @@ bool make_map(CUtensorMap* m, const void* base, int dtype, long long outer, long
   return r == CUDA_SUCCESS;
 }
 
+// Packed variable-length layout [total, H, D]: a 3-D map ordered (D, head, token) so that one
+// box (64 elements x 1 head x 128 tokens) is the same 128-row x 128-byte slab as in make_map.
+bool make_map_packed(CUtensorMap* m, const void* base, int dtype, long long total, int H, int D) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)total};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dtype == MFA_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Opt a kernel into its dynamic shared memory size once per device.
 template <typename K>
 bool ensure_smem(K kernel, int bytes, bool (&done)[kMaxDevices]) {
@@ -115,14 +131,29 @@ int check_sizes(long long a, long long b, long long c, long long d) {
   return MFA_OK;
 }
 
-template <int D, bool BF16>
-int launch_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
-               int Hkv, int Nq, int Nk, float scale, int causal, int win_l, int win_r,
-               float softcap, int dtype, cudaStream_t st) {
+// Arguments of one forward launch (dense, or packed variable-length when cu_q != NULL; then Nq
+// is the longest sequence's query count, which sizes the grid).
+struct FwdCall {
+  const void *q, *k, *v;
+  void* out;
+  float* lse;
+  int B, Hq, Hkv, Nq, Nk;
+  float scale;
+  int causal, win_l, win_r;
+  float softcap;
+  int dtype;
+  const int32_t *cu_q, *cu_k;
+  int total_q, total_k;
+};
+
+template <int D, bool BF16, bool VARLEN>
+int launch_fwd(const FwdCall& c, cudaStream_t st) {
+  const int B = c.B, Hq = c.Hq, Hkv = c.Hkv, Nq = c.Nq, Nk = c.Nk, dtype = c.dtype;
+  const float scale = c.scale, softcap = c.softcap;
   static bool smem_done[kMaxDevices] = {};
   static bool regs_ok[kMaxDevices] = {};
   constexpr int smem = mfa::fwd_smem_bytes<D>();
-  auto kernel = mfa::mfa_fwd_kernel<D, BF16>;
+  auto kernel = mfa::mfa_fwd_kernel<D, BF16, VARLEN>;
   if (!ensure_smem(kernel, smem, smem_done)) return MFA_ERR_CUDA;
   {
     // setmaxnreg redistributes the registers the CTA launched with; refuse to launch if the
@@ -139,20 +170,30 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, float* ls
   }
   mfa::FwdParams p;
   std::memset(&p, 0, sizeof(p));
-  if (!make_map(&p.tm_q, q, dtype, (long long)B * Hq, Nq, D)) return MFA_ERR_CUDA;
-  if (!make_map(&p.tm_k, k, dtype, (long long)B * Hkv, Nk, D)) return MFA_ERR_CUDA;
-  if (!make_map(&p.tm_v, v, dtype, (long long)B * Hkv, Nk, D)) return MFA_ERR_CUDA;
-  p.out = out;
-  p.lse = lse;
+  if (VARLEN) {
+    if (!make_map_packed(&p.tm_q, c.q, dtype, c.total_q, Hq, D)) return MFA_ERR_CUDA;
+    if (!make_map_packed(&p.tm_k, c.k, dtype, c.total_k, Hkv, D)) return MFA_ERR_CUDA;
+    if (!make_map_packed(&p.tm_v, c.v, dtype, c.total_k, Hkv, D)) return MFA_ERR_CUDA;
+    p.cu_q = c.cu_q;
+    p.cu_k = c.cu_k;
+    p.total_q = c.total_q;
+    p.total_k = c.total_k;
+  } else {
+    if (!make_map(&p.tm_q, c.q, dtype, (long long)B * Hq, Nq, D)) return MFA_ERR_CUDA;
+    if (!make_map(&p.tm_k, c.k, dtype, (long long)B * Hkv, Nk, D)) return MFA_ERR_CUDA;
+    if (!make_map(&p.tm_v, c.v, dtype, (long long)B * Hkv, Nk, D)) return MFA_ERR_CUDA;
+  }
+  p.out = c.out;
+  p.lse = c.lse;
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.Nq = Nq;
   p.Nk = Nk;
   p.G = Hq / Hkv;
-  p.causal = causal ? 1 : 0;
-  p.win_l = win_l;
-  p.win_r = win_r;
+  p.causal = c.causal ? 1 : 0;
+  p.win_l = c.win_l;
+  p.win_r = c.win_r;
   const int rows_per_cta = mfa::kFwdBM * mfa::kFwdQT;
   p.n_qblk = (Nq + rows_per_cta - 1) / rows_per_cta;
   p.flags = g_debug_flags;
@@ -219,6 +260,42 @@ int launch_decode(const mfa::DecodeParams& p, const DecodePlan& pl, cudaStream_t
   return MFA_OK;
 }
 
+// Checks shared by the dense and the packed forward.
+int validate_fwd_common(int Hq, int Hkv, int D, int dtype, int win_l, int win_r,
+                               float softcap, float scale) {
+  if (dtype != MFA_DTYPE_FP16 && dtype != MFA_DTYPE_BF16) return MFA_ERR_BAD_DTYPE;
+  if (D != 64 && D != 128) return MFA_ERR_BAD_HEAD_DIM;
+  if (Hq < 0) return MFA_ERR_BAD_SHAPE;
+  if (Hkv < 1 || Hq % Hkv != 0) return MFA_ERR_GQA_GEOMETRY;
+  if (win_l < -1 || win_r < -1) return MFA_ERR_BAD_WINDOW;
+  if (!std::isfinite(softcap) || softcap < 0.f) return MFA_ERR_BAD_SOFTCAP;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return MFA_ERR_BAD_SCALE;
+  return MFA_OK;
+}
+
+// Every row sees no key: out = 0, lse = -inf (rows = number of (query, head) pairs).
+int launch_fill_empty(void* out, float* lse, size_t rows, int D, int dtype, cudaStream_t st) {
+  if (dtype == MFA_DTYPE_BF16)
+    mfa::mfa_fill_empty_kernel<true><<<148, 256, 0, st>>>(out, lse, rows, D);
+  else
+    mfa::mfa_fill_empty_kernel<false><<<148, 256, 0, st>>>(out, lse, rows, D);
+  if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
+  mfa_launch_info li = {};
+  li.kernel = 3;
+  li.grid_x = 148;
+  li.grid_y = li.grid_z = 1;
+  li.block_threads = 256;
+  g_last = li;
+  return MFA_OK;
+}
+
+template <bool VARLEN>
+int dispatch_fwd(const FwdCall& c, int D, cudaStream_t st) {
+  const bool bf = c.dtype == MFA_DTYPE_BF16;
+  if (D == 128) return bf ? launch_fwd<128, true, VARLEN>(c, st) : launch_fwd<128, false, VARLEN>(c, st);
+  return bf ? launch_fwd<64, true, VARLEN>(c, st) : launch_fwd<64, false, VARLEN>(c, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -226,14 +303,9 @@ extern "C" {
 int mfa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
             int Hkv, int Nq, int Nk, int D, float scale, int causal, int win_l, int win_r,
             float softcap, int dtype, void* stream) {
-  if (dtype != MFA_DTYPE_FP16 && dtype != MFA_DTYPE_BF16) return MFA_ERR_BAD_DTYPE;
-  if (D != 64 && D != 128) return MFA_ERR_BAD_HEAD_DIM;
-  if (B < 0 || Hq < 0 || Nq < 0 || Nk < 0) return MFA_ERR_BAD_SHAPE;
-  if (Hkv < 1 || Hq % Hkv != 0) return MFA_ERR_GQA_GEOMETRY;
-  if (win_l < -1 || win_r < -1) return MFA_ERR_BAD_WINDOW;
-  if (!std::isfinite(softcap) || softcap < 0.f) return MFA_ERR_BAD_SOFTCAP;
-  if (!std::isfinite(scale) || !(scale > 0.f)) return MFA_ERR_BAD_SCALE;
-  int rc;
+  int rc = validate_fwd_common(Hq, Hkv, D, dtype, win_l, win_r, softcap, scale);
+  if (rc != MFA_OK) return rc;
+  if (B < 0 || Nq < 0 || Nk < 0) return MFA_ERR_BAD_SHAPE;
   if ((rc = check_sizes(B, Hq, Nq, D)) != MFA_OK) return rc;
   if ((rc = check_sizes(B, Hkv, Nk, D)) != MFA_OK) return rc;
   if ((long long)B * Hq > 0x7FFFFFFFLL || (long long)B * Hkv > 0x7FFFFFFFLL) return MFA_ERR_BAD_SHAPE;
@@ -242,27 +314,35 @@ int mfa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, 
   if (!aligned16(q) || !aligned16(out) || !aligned16(lse) || (Nk > 0 && (!aligned16(k) || !aligned16(v))))
     return MFA_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (Nk == 0) {
-    const size_t rows = (size_t)B * Hq * Nq;
-    if (dtype == MFA_DTYPE_BF16)
-      mfa::mfa_fill_empty_kernel<true><<<148, 256, 0, st>>>(out, lse, rows, D);
-    else
-      mfa::mfa_fill_empty_kernel<false><<<148, 256, 0, st>>>(out, lse, rows, D);
-    if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
-    mfa_launch_info li = {};
-    li.kernel = 3;
-    li.grid_x = 148;
-    li.grid_y = li.grid_z = 1;
-    li.block_threads = 256;
-    g_last = li;
-    return MFA_OK;
-  }
-  const bool bf = dtype == MFA_DTYPE_BF16;
-  if (D == 128)
-    return bf ? launch_fwd<128, true>(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, scale, causal, win_l, win_r, softcap, dtype, st)
-              : launch_fwd<128, false>(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, scale, causal, win_l, win_r, softcap, dtype, st);
-  return bf ? launch_fwd<64, true>(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, scale, causal, win_l, win_r, softcap, dtype, st)
-            : launch_fwd<64, false>(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, scale, causal, win_l, win_r, softcap, dtype, st);
+  if (Nk == 0) return launch_fill_empty(out, lse, (size_t)B * Hq * Nq, D, dtype, st);
+  FwdCall c = {q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, scale, causal, win_l, win_r, softcap, dtype,
+               nullptr, nullptr, 0, 0};
+  return dispatch_fwd<false>(c, D, st);
+}
+
+int mfa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
+                   const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B, int max_seqlen_q,
+                   int total_q, int total_k, int Hq, int Hkv, int D, float scale, int causal,
+                   int win_l, int win_r, float softcap, int dtype, void* stream) {
+  int rc = validate_fwd_common(Hq, Hkv, D, dtype, win_l, win_r, softcap, scale);
+  if (rc != MFA_OK) return rc;
+  if (B < 0 || max_seqlen_q < 0 || total_q < 0 || total_k < 0) return MFA_ERR_BAD_SHAPE;
+  if (max_seqlen_q > total_q) return MFA_ERR_BAD_SHAPE;
+  if ((rc = check_sizes(total_q, Hq, D, 1)) != MFA_OK) return rc;
+  if ((rc = check_sizes(total_k, Hkv, D, 1)) != MFA_OK) return rc;
+  if ((long long)B * Hq > 0x7FFFFFFFLL) return MFA_ERR_BAD_SHAPE;
+  if (B == 0 || Hq == 0 || total_q == 0 || max_seqlen_q == 0) return MFA_OK;
+  if (!q || !out || !cu_seqlens_q || !cu_seqlens_k || (total_k > 0 && (!k || !v)))
+    return MFA_ERR_NULL_POINTER;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(lse) ||
+      (total_k > 0 && (!aligned16(k) || !aligned16(v))) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+    return MFA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (total_k == 0) return launch_fill_empty(out, lse, (size_t)total_q * Hq, D, dtype, st);
+  FwdCall c = {q, k, v, out, lse, B, Hq, Hkv, max_seqlen_q, 0, scale, causal, win_l, win_r, softcap,
+               dtype, cu_seqlens_q, cu_seqlens_k, total_q, total_k};
+  return dispatch_fwd<true>(c, D, st);
 }
 
 static int validate_decode(int B, int Nq, int Hq, int Hkv, int D, int page_size, int max_pages) {
@@ -364,6 +444,7 @@ const char* mfa_status_string(int code) {
     case MFA_ERR_CUDA: return "a CUDA call or kernel launch failed";
     case MFA_ERR_DEVICE_TIMEOUT: return "device: a bounded wait inside a kernel ran out";
     case MFA_ERR_DEVICE_BAD_PAGE: return "device: block_table or seq_lens entry out of range";
+    case MFA_ERR_DEVICE_BAD_SEQLENS: return "device: cu_seqlens entry negative, decreasing, past the packed total, or a sequence longer than max_seqlen_q";
     case MFA_ERR_SCRATCH_TOO_SMALL: return "decode shape needs more workspace than the fixed 64 MiB scratch of mfa_decode_splitkv_noalloc";
     default: return "unknown status";
   }
