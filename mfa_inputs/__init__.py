@@ -23,7 +23,8 @@ _SRC = os.path.join(_HERE, "gen.c")
 
 FP16, BF16 = 0, 1
 DTYPE_NAMES = {FP16: "fp16", BF16: "bf16"}
-STREAM_Q, STREAM_K, STREAM_V, STREAM_LENS, STREAM_PERM, STREAM_KEXTRA = 0, 1, 2, 3, 4, 5
+STREAM_Q, STREAM_K, STREAM_V, STREAM_LENS, STREAM_PERM, STREAM_KEXTRA, STREAM_MASK = 0, 1, 2, 3, 4, 5, 6
+SPARSE_BLOCK = 128  # query rows x keys per block-mask entry (the forward kernel's tile)
 PAGE_SIZE = 16
 
 
@@ -292,6 +293,71 @@ class VarlenCase:
         return q, k, v
 
 
+@dataclass
+class SparseCase:
+    """Block-sparse prefill: dense q [B,Hq,N,D], k/v [B,Hkv,N,D] and a block mask uint8
+    [B, Hq, nb, nb] (nb = ceil(N / 128)); a zero entry removes a 128 x 128 block of (query rows,
+    keys) from the visible set.
+
+    pattern "spatial2d": the N tokens are grid[0] x grid[1] blocks of 128 on a 2-D grid in
+    row-major order, and block (r1, c1) attends block (r2, c2) iff max(|r1 - r2|, |c1 - c2|) <=
+    radius (a local neighbourhood, as in the pages' spatial 2-D masks); the same for every head.
+    pattern "random": every entry is on with probability density (stream 6, per batch and head),
+    and the diagonal blocks are always on.
+    """
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    N: int
+    D: int
+    dtype: int
+    causal: bool
+    pattern: str = "random"
+    density: float = 0.3
+    grid: tuple = (1, 1)
+    radius: int = 1
+    win_l: int = -1
+    win_r: int = -1
+    softcap: float = 0.0
+    mul: float = 1.0
+    seed: int = 1
+    scale: float | None = None
+
+    @property
+    def Nq(self):
+        return self.N
+
+    @property
+    def Nk(self):
+        return self.N
+
+    def scale_f32(self) -> float:
+        s = self.scale if self.scale is not None else 1.0 / np.sqrt(self.D)
+        return float(np.float32(s))
+
+    def block_mask(self) -> np.ndarray:
+        nb = -(-self.N // SPARSE_BLOCK)
+        if self.pattern == "spatial2d":
+            gh, gw = self.grid
+            assert gh * gw == nb, "grid must tile the sequence in 128-token blocks"
+            r, c = np.divmod(np.arange(nb), gw)
+            m = (np.maximum(np.abs(r[:, None] - r[None, :]), np.abs(c[:, None] - c[None, :]))
+                 <= self.radius).astype(np.uint8)
+            return np.broadcast_to(m, (self.B, self.Hq, nb, nb)).copy()
+        u = uniform_ints(self.seed, STREAM_MASK, self.B * self.Hq * nb * nb, 0, 999)
+        m = (u.reshape(self.B, self.Hq, nb, nb) < int(round(self.density * 1000))).astype(np.uint8)
+        m[:, :, np.arange(nb), np.arange(nb)] = 1
+        return m
+
+    def tensors(self):
+        """(q, k, v) as uint16 bit patterns and the block mask."""
+        q = normal_bits(self.seed, STREAM_Q, (self.B, self.Hq, self.N, self.D), self.dtype, self.mul)
+        k = normal_bits(self.seed, STREAM_K, (self.B, self.Hkv, self.N, self.D), self.dtype, self.mul)
+        v = normal_bits(self.seed, STREAM_V, (self.B, self.Hkv, self.N, self.D), self.dtype, self.mul)
+        return q, k, v, self.block_mask()
+
+
 def workloads():
     """The named full-size workloads (shapes, flags, seeds and value scales)."""
     return {
@@ -313,6 +379,9 @@ def workloads():
         "varlen_causal_b8_h8_d128_fp16_len512_8k": VarlenCase(
             "varlen_causal_b8_h8_d128_fp16_len512_8k", 8, 8, 8, 128, FP16, True, 512, 8192,
             seed=1006),
+        "sparse_spatial2d_b1_h16_n16384_d128_fp16": SparseCase(
+            "sparse_spatial2d_b1_h16_n16384_d128_fp16", 1, 16, 16, 16384, 128, FP16, False,
+            pattern="spatial2d", grid=(16, 8), radius=2, seed=1007),
         "decode_b8_hq32_hkv8_d128_bf16_len8k_128k": DecodeCase(
             "decode_b8_hq32_hkv8_d128_bf16_len8k_128k", 8, 1, 32, 8, 128, BF16, 8192, 131072,
             seed=1005),

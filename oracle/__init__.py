@@ -22,6 +22,9 @@ Sources (web pages, cited by title and section):
   * "mlx-mfa 2.5.2" Features: variable-length packed sequences with cu_seqlens; "mlx-mfa
     2.61.0" (essential correctness update): varlen causal with N_q < N_k changed toward the
     bottom-right alignment used here per sequence.
+  * "mlx-mfa 2.5.2" Features and Usage: block-sparse attention, flash_attention_sparse(q, k, v,
+    block_mask, causal=...), a block mask whose zero blocks are never attended; here a block is
+    `block` query rows x `block` keys and the mask further restricts the causal / window set.
 
 Readings where the pages are silent or ambiguous (each restated in the design doc):
   * window: key j is visible from absolute query position a iff a - win_l <= j <= a + win_r
@@ -39,7 +42,8 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = ["visible", "attention", "attention_rows", "attention_varlen", "attention_varlen_rows",
-           "paged_gather", "decode", "decode_rows"]
+           "attention_blocksparse", "attention_blocksparse_rows", "paged_gather", "decode",
+           "decode_rows"]
 
 
 def visible(Nq: int, Nk: int, causal: bool, win_l: int = -1, win_r: int = -1) -> np.ndarray:
@@ -173,6 +177,62 @@ def attention_varlen_rows(q, k, v, cu_q, cu_k, rows, scale, causal=False, win_l=
         qs, ks, vs = _sequence_views(q, k, v, cu_q, cu_k, b)
         oi, li = attention_rows(qs, ks, vs, [(0, h, r - cu_q[b])], scale, causal, win_l, win_r,
                                 softcap)
+        o[n], lse[n] = oi[0], li[0]
+    return o, lse
+
+
+def _block_visibility(block_mask, b, h, Nq, Nk, block):
+    """[Nq, Nk] boolean: query row i may attend key j as far as the block mask is concerned."""
+    m = np.asarray(block_mask[b, h], dtype=bool)
+    return np.repeat(np.repeat(m, block, axis=0), block, axis=1)[:Nq, :Nk]
+
+
+def attention_blocksparse(q, k, v, block_mask, scale, causal=False, win_l=-1, win_r=-1,
+                          softcap=0.0, block=128):
+    """Block-sparse forward: the dense definition with visibility vis(i, j) AND
+    block_mask[b, h, i // block, j // block] != 0. q [B,Hq,Nq,D], k/v [B,Hkv,Nk,D],
+    block_mask [B, Hq, ceil(Nq/block), ceil(Nk/block)]. Returns (o [B,Hq,Nq,D], lse [B,Hq,Nq])."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, Hq, Nq, D = q.shape
+    _, Hkv, Nk, _ = k.shape
+    G = Hq // Hkv
+    vis = visible(Nq, Nk, causal, win_l, win_r)
+    o = np.zeros((B, Hq, Nq, D))
+    lse = np.full((B, Hq, Nq), -np.inf)
+    for b in range(B):
+        for h in range(Hq):
+            vb = vis & _block_visibility(block_mask, b, h, Nq, Nk, block)
+            o[b, h], lse[b, h] = _rows_for_head(q[b, h], k[b, h // G], v[b, h // G], vb, scale,
+                                                softcap)
+    return o, lse
+
+
+def attention_blocksparse_rows(q, k, v, block_mask, rows, scale, causal=False, win_l=-1,
+                               win_r=-1, softcap=0.0, block=128):
+    """Selected rows (b, h, i) of the block-sparse forward. Returns (o [n, D], lse [n])."""
+    B, Hq, Nq, D = np.shape(q)
+    _, Hkv, Nk, _ = np.shape(k)
+    G = Hq // Hkv
+    rows = np.asarray(rows, dtype=np.int64).reshape(-1, 3)
+    o = np.zeros((len(rows), D))
+    lse = np.full(len(rows), -np.inf)
+    j = np.arange(Nk, dtype=np.int64)
+    for n, (b, h, i) in enumerate(rows):
+        a = i + Nk - Nq
+        vis = np.ones(Nk, dtype=bool)
+        if causal:
+            vis &= j <= a
+        if win_l >= 0:
+            vis &= j >= a - win_l
+        if win_r >= 0:
+            vis &= j <= a + win_r
+        keep = np.repeat(np.asarray(block_mask[b, h, i // block], dtype=bool), block)[:Nk]
+        qi = np.asarray(q[b, h, i:i + 1], dtype=np.float64)
+        oi, li = _rows_for_head(qi, np.asarray(k[b, h // G], dtype=np.float64),
+                                np.asarray(v[b, h // G], dtype=np.float64),
+                                (vis & keep)[None, :], scale, softcap)
         o[n], lse[n] = oi[0], li[0]
     return o, lse
 

@@ -400,3 +400,88 @@ def test_varlen_rows_helper_matches_full():
     orow, lrow = oracle.attention_varlen_rows(q, k, v, cq, ck, rows, 0.5, True, 6, -1, softcap=2.0)
     np.testing.assert_allclose(orow, o[rows[:, 1], rows[:, 0]], rtol=0, atol=1e-13)
     np.testing.assert_allclose(lrow, lse[rows[:, 0], rows[:, 1]], rtol=0, atol=1e-13)
+
+
+# ---------------------------------------------------------------- block-sparse masks
+def _torch_block_mask(bm, Nq, Nk, block):
+    """[Nq, Nk] boolean from a block mask, expanded with torch.repeat_interleave."""
+    t = torch.from_numpy(np.asarray(bm, dtype=bool))
+    return t.repeat_interleave(block, 0).repeat_interleave(block, 1)[:Nq, :Nk]
+
+
+@pytest.mark.parametrize("causal,wl,wr", [(False, -1, -1), (True, -1, -1), (True, 9, 0), (False, 4, 6)])
+def test_blocksparse_matches_torch_sdpa(causal, wl, wr):
+    """Against torch's SDPA with the band mask AND the block mask (expanded by torch)."""
+    B, Hq, Hkv, Nq, Nk, D, blk = 2, 4, 2, 37, 45, 8, 8
+    q = rng.standard_normal((B, Hq, Nq, D))
+    k = rng.standard_normal((B, Hkv, Nk, D))
+    v = rng.standard_normal((B, Hkv, Nk, D))
+    bm = (rng.random((B, Hq, -(-Nq // blk), -(-Nk // blk))) < 0.5).astype(np.uint8)
+    o, lse = oracle.attention_blocksparse(q, k, v, bm, 0.3, causal, wl, wr, block=blk)
+    band = band_mask_torch(Nq, Nk, causal, wl, wr)
+    G = Hq // Hkv
+    for b in range(B):
+        for h in range(Hq):
+            m = band & _torch_block_mask(bm[b, h], Nq, Nk, blk)
+            has = m.any(dim=1).numpy()
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                torch.from_numpy(q[b, h][None, None]), torch.from_numpy(k[b, h // G][None, None]),
+                torch.from_numpy(v[b, h // G][None, None]), attn_mask=m, scale=0.3).numpy()[0, 0]
+            np.testing.assert_allclose(o[b, h, has], ref[has], rtol=0, atol=1e-12)
+            assert np.all(o[b, h, ~has] == 0) and np.all(np.isneginf(lse[b, h, ~has]))
+
+
+def test_blocksparse_all_ones_is_dense_and_all_zeros_is_empty():
+    B, Hq, Hkv, Nq, Nk, D, blk = 1, 2, 1, 40, 40, 8, 16
+    q = rng.standard_normal((B, Hq, Nq, D))
+    k = rng.standard_normal((B, Hkv, Nk, D))
+    v = rng.standard_normal((B, Hkv, Nk, D))
+    ones = np.ones((B, Hq, 3, 3), dtype=np.uint8)
+    o1, l1 = oracle.attention_blocksparse(q, k, v, ones, 0.4, True, block=blk)
+    o2, l2 = oracle.attention(q, k, v, 0.4, True)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+    o3, l3 = oracle.attention_blocksparse(q, k, v, 0 * ones, 0.4, True, block=blk)
+    assert np.all(o3 == 0) and np.all(np.isneginf(l3))
+
+
+def test_blocksparse_zero_query_lse_counts_active_keys():
+    """Q = 0: LSE of row i = ln(#keys that are band-visible AND in an active block), counted by
+    interval arithmetic per active key block."""
+    Nq, Nk, blk = 50, 70, 16
+    bm = (rng.random((1, 1, 4, 5)) < 0.6).astype(np.uint8)
+    bm[0, 0, :, 0] = 1
+    q = np.zeros((1, 1, Nq, 4))
+    k = rng.standard_normal((1, 1, Nk, 4))
+    v = rng.standard_normal((1, 1, Nk, 4))
+    for causal, wl, wr in ((True, -1, -1), (True, 20, 0), (False, 7, 3)):
+        _, lse = oracle.attention_blocksparse(q, k, v, bm, 1.0, causal, wl, wr, block=blk)
+        for i in range(Nq):
+            a = i + Nk - Nq
+            lo = 0 if wl < 0 else max(0, a - wl)
+            hi = Nk - 1
+            if causal:
+                hi = min(hi, a)
+            if wr >= 0:
+                hi = min(hi, a + wr)
+            cnt = 0
+            for jb in range(5):
+                if bm[0, 0, i // blk, jb]:
+                    cnt += max(0, min(hi, jb * blk + blk - 1, Nk - 1) - max(lo, jb * blk) + 1)
+            if cnt == 0:
+                assert np.isneginf(lse[0, 0, i])
+            else:
+                assert abs(lse[0, 0, i] - math.log(cnt)) < 1e-13
+
+
+def test_blocksparse_rows_helper_matches_full():
+    B, Hq, Hkv, Nq, Nk, D, blk = 2, 4, 2, 30, 44, 8, 8
+    q = rng.standard_normal((B, Hq, Nq, D))
+    k = rng.standard_normal((B, Hkv, Nk, D))
+    v = rng.standard_normal((B, Hkv, Nk, D))
+    bm = (rng.random((B, Hq, 4, 6)) < 0.5).astype(np.uint8)
+    o, lse = oracle.attention_blocksparse(q, k, v, bm, 0.5, True, 12, -1, softcap=3.0, block=blk)
+    rows = np.array([(b, h, i) for b in range(B) for h in range(Hq) for i in range(Nq)])
+    orow, lrow = oracle.attention_blocksparse_rows(q, k, v, bm, rows, 0.5, True, 12, -1,
+                                                   softcap=3.0, block=blk)
+    np.testing.assert_allclose(orow, o[rows[:, 0], rows[:, 1], rows[:, 2]], rtol=0, atol=1e-13)
+    np.testing.assert_array_equal(np.isneginf(lrow), np.isneginf(lse[rows[:, 0], rows[:, 1], rows[:, 2]]))
