@@ -5,7 +5,7 @@ python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mfa|reference] [--wo
 One step = one pass of the hot path over one batch: the prefill forward of the named workload
 (default: causal, B=2, H=8, N=4096, D=128, fp16). The same JSON line also carries the other
 workloads (non-causal, sliding window, GQA + softcap prefill, packed variable-length prefill,
-paged split-KV decode), each timed the same way. Inputs are seeded synthetic tensors resident in HBM; L2 is flushed (a 256 MiB
+block-sparse prefill, paged split-KV decode), each timed the same way. Inputs are seeded synthetic tensors resident in HBM; L2 is flushed (a 256 MiB
 write) before every timed step, outside the timed kernel. Times are CUDA events on the launching
 stream; with N > 1 (torchrun) every rank runs its own copy of the workload (weak scaling) and the
 max over ranks is reported.
@@ -60,6 +60,31 @@ def prefill_bytes(case) -> float:
     e = 2
     return (e * case.B * case.Hq * case.Nq * case.D * 2 + e * 2 * case.B * case.Hkv * case.Nk * case.D
             + 4 * case.B * case.Hq * case.Nq)
+
+
+def sparse_pairs(case, mask) -> int:
+    """Visible (query, key) pairs summed over batch and heads: the causal / window interval of
+    each row intersected with the key blocks its 128-row mask row has on."""
+    blk = mi.SPARSE_BLOCK
+    i = np.arange(case.Nq, dtype=np.int64)
+    a = i + (case.Nk - case.Nq)
+    lo = np.zeros_like(a) if case.win_l < 0 else np.maximum(0, a - case.win_l)
+    hi = np.full_like(a, case.Nk - 1)
+    if case.causal:
+        hi = np.minimum(hi, a)
+    if case.win_r >= 0:
+        hi = np.minimum(hi, a + case.win_r)
+    nkb = mask.shape[3]
+    kb_lo = np.arange(nkb, dtype=np.int64) * blk
+    kb_hi = np.minimum(kb_lo + blk - 1, case.Nk - 1)
+    # overlap[i, kb] of row i's interval with key block kb
+    ov = np.maximum(0, np.minimum(hi[:, None], kb_hi[None, :]) - np.maximum(lo[:, None], kb_lo[None, :]) + 1)
+    total = 0
+    for b in range(mask.shape[0]):
+        for h in range(mask.shape[1]):
+            on = mask[b, h][i // blk].astype(bool)          # [Nq, nkb]
+            total += int((ov * on).sum())
+    return total
 
 
 def varlen_flops(case) -> float:
@@ -277,6 +302,31 @@ def bench_varlen(case, steps, warmup, flush, stream, world):
             "total_q": int(cq[-1])}
 
 
+def bench_sparse(case, steps, warmup, flush, stream, world):
+    import torch
+    import tiled_exact_attention_mfa_b200 as mfa
+    dev = torch.device("cuda")
+    q, k, v, m = case.tensors()
+    qt, kt, vt = (upload(x, case.dtype, dev) for x in (q, k, v))
+    mt = torch.from_numpy(m).to(dev)
+    out = torch.empty_like(qt)
+    lse = torch.empty(case.B, case.Hq, case.Nq, dtype=torch.float32, device=dev)
+    scale = case.scale_f32()
+
+    def step():
+        mfa.mfa_fwd_blocksparse(qt, kt, vt, mt, out, lse, scale=scale, causal=case.causal,
+                                window=(case.win_l, case.win_r), softcap=case.softcap, stream=stream)
+
+    with torch.cuda.stream(stream):
+        ms, bracket = time_steps(step, steps, warmup, flush, stream)
+    pairs = sparse_pairs(case, m)
+    byts = 2 * case.B * case.Hq * case.Nq * case.D * 2 + 2 * 2 * case.B * case.Hkv * case.Nk * case.D \
+        + 4 * case.B * case.Hq * case.Nq + m.size
+    return {"ms": max_over_ranks(statistics.mean(ms), world), "ms_min": min(ms),
+            "bracket_ms": bracket, "flops": 4.0 * case.D * pairs, "bytes": float(byts),
+            "density": float(m.mean())}
+
+
 def bench_decode(case, steps, warmup, flush, stream, world):
     import torch
     import tiled_exact_attention_mfa_b200 as mfa
@@ -339,14 +389,18 @@ def run_gpu(args):
             if name == args.workload:
                 continue
             sk, wu = max(3, min(args.steps, 10)), max(3, args.warmup)
-            if isinstance(case, mi.VarlenCase):
-                r = bench_varlen(case, sk, wu, flush, stream, world)
+            if isinstance(case, (mi.VarlenCase, mi.SparseCase)):
+                if isinstance(case, mi.VarlenCase):
+                    r = bench_varlen(case, sk, wu, flush, stream, world)
+                else:
+                    r = bench_sparse(case, sk, wu, flush, stream, world)
                 tf = r["flops"] * world / (r["ms"] * 1e-3) / 1e12
                 gbs = r["bytes"] * world / (r["ms"] * 1e-3) / 1e9
                 t_floor = max(r["flops"] / (pk["tflops"] * 1e12), r["bytes"] / (pk["gbs"] * 1e9))
                 others.append({"workload": name, "ms": round(r["ms"], 4), "unit": "TFLOP/s",
                                "value": round(tf, 1), "GB/s": round(gbs, 1),
-                               "total_q": r["total_q"],
+                               **({"total_q": r["total_q"]} if "total_q" in r else
+                                  {"block_density": round(r["density"], 4)}),
                                "frac_of_measured_tensor_peak": round(tf / pk["tflops"], 4),
                                "frac_of_nominal_tensor_peak": round(tf / NOMINAL_TFLOPS, 4),
                                "frac_of_roofline": round(t_floor / (r["ms"] * 1e-3), 4)})
@@ -492,6 +546,8 @@ def run_profile(args):
         r = bench_decode(case, args.steps, args.warmup, lambda: flush_buf.fill_(1), stream, 1)
     elif isinstance(case, mi.VarlenCase):
         r = bench_varlen(case, args.steps, args.warmup, lambda: flush_buf.fill_(1), stream, 1)
+    elif isinstance(case, mi.SparseCase):
+        r = bench_sparse(case, args.steps, args.warmup, lambda: flush_buf.fill_(1), stream, 1)
     else:
         r = bench_prefill(case, args.steps, args.warmup, lambda: flush_buf.fill_(1), stream, False, 1)
     print(json.dumps({"profile": args.profile, "ms": round(r["ms"], 5)}), flush=True)

@@ -5,6 +5,7 @@
  *   mfa_fwd            dense forward with online softmax: causal and sliding-window tile skip,
  *                      native GQA, optional tanh softcap, optional fp32 log-sum-exp output.
  *   mfa_fwd_varlen     the same forward over packed variable-length sequences (cu_seqlens).
+ *   mfa_fwd_blocksparse the same forward restricted by a 128 x 128 block mask.
  *   mfa_decode_splitkv two-phase split-KV decode (N_q <= 4) over a paged KV cache.
  *
  * Sources (web pages, cited by title and section):
@@ -61,7 +62,8 @@ extern "C" {
 #define MFA_ERR_NQ_TOO_LARGE       -10   /* decode with N_q > 4 */
 #define MFA_ERR_PAGE_SIZE          -11   /* page_size != 16 */
 #define MFA_ERR_WORKSPACE          -12   /* workspace NULL, misaligned or smaller than required */
-#define MFA_ERR_UNSUPPORTED        -13   /* decode with (Hq / Hkv) * N_q > 16 query rows per kv head */
+#define MFA_ERR_UNSUPPORTED        -13   /* decode with (Hq / Hkv) * N_q > 16 query rows per kv head, or a
+                                            block-sparse call with more than 2048 key tiles */
 #define MFA_ERR_CUDA               -20   /* a CUDA runtime/driver call or a launch failed */
 #define MFA_ERR_DEVICE_TIMEOUT     -21   /* device status: a bounded wait inside a kernel ran out */
 #define MFA_ERR_DEVICE_BAD_PAGE    -22   /* device status: a block_table entry was outside [0, num_pages) */
@@ -124,6 +126,26 @@ int mfa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float
                    int B, int max_seqlen_q, int total_q, int total_k,
                    int Hq, int Hkv, int D, float scale,
                    int causal, int win_l, int win_r, float softcap, int dtype, void* stream);
+
+/*
+ * mfa_fwd_blocksparse -- the dense forward restricted by a block mask ([MFA252] Features
+ * "Block-sparse attention -- block_mask tensor skips entire tiles"; Usage
+ * flash_attention_sparse(q, k, v, block_mask, causal=True)).
+ *
+ * Query row i of (b, h) may attend key j only if block_mask[b][h][i / 128][j / 128] != 0, in
+ * addition to the causal / window predicates of mfa_fwd: vis(j) becomes vis(j) && mask bit. A
+ * 128 x 128 block is one tile of the kernel, so a zero entry is never loaded or computed for the
+ * query tile it belongs to (when both 128-row tiles of a 256-row block have it off). Rows left
+ * with no visible key get out = 0, lse = -inf.
+ *
+ * Arguments as mfa_fwd, plus
+ *   block_mask  uint8 [B, Hq, ceil(Nq / 128), ceil(Nk / 128)], row-major   (device)
+ *   ceil(Nk / 128) <= 2048 (Nk <= 262,144), else MFA_ERR_UNSUPPORTED.
+ */
+int mfa_fwd_blocksparse(const void* q, const void* k, const void* v, void* out, float* lse,
+                        const uint8_t* block_mask,
+                        int B, int Hq, int Hkv, int Nq, int Nk, int D, float scale,
+                        int causal, int win_l, int win_r, float softcap, int dtype, void* stream);
 
 /*
  * mfa_decode_workspace_size -- bytes of scratch mfa_decode_splitkv needs for this shape.

@@ -104,6 +104,24 @@ def test_fwd_varlen_empty_problem_is_noop():
     assert fwd_varlen(total_q=0, max_q=0, q=None, out=None) == 0
 
 
+def fwd_sparse(**kw):
+    args = dict(q=A, k=A, v=A, out=A, lse=A, mask=A, B=1, Hq=4, Hkv=2, Nq=512, Nk=512, D=128,
+                scale=0.1, causal=0, win_l=-1, win_r=-1, softcap=0.0, dtype=1, stream=None)
+    args.update(kw)
+    return mfa.lib.mfa_fwd_blocksparse(*args.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=9), -3), (dict(D=100), -4), (dict(Nq=-1), -5), (dict(Hkv=3), -6),
+    (dict(win_r=-2), -7), (dict(softcap=-3.0), -8), (dict(scale=float("inf")), -9),
+    (dict(mask=None), -1), (dict(q=None), -1), (dict(k=A + 4), -2),
+    (dict(Nk=2048 * 128 + 1), -13),
+])
+@no_device
+def test_fwd_blocksparse_rejects_malformed(kw, code):
+    assert fwd_sparse(**kw) == code
+
+
 def dec(**kw):
     ws = kw.pop("ws_bytes", 1 << 30)
     args = dict(q=A, k=A, v=A, table=A, lens=A, out=A, lse=A, B=8, Nq=1, Hq=32, Hkv=8, D=128,

@@ -34,6 +34,8 @@ lib.mfa_fwd.restype = _i
 lib.mfa_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _i, _f, _i, _vp]
 lib.mfa_fwd_varlen.restype = _i
 lib.mfa_fwd_varlen.argtypes = [_vp] * 7 + [_i] * 7 + [_f, _i, _i, _i, _f, _i, _vp]
+lib.mfa_fwd_blocksparse.restype = _i
+lib.mfa_fwd_blocksparse.argtypes = [_vp] * 6 + [_i] * 6 + [_f, _i, _i, _i, _f, _i, _vp]
 lib.mfa_decode_workspace_size.restype = ctypes.c_size_t
 lib.mfa_decode_workspace_size.argtypes = [_i] * 7
 lib.mfa_decode_splitkv.restype = _i
@@ -67,7 +69,7 @@ lib.mfa_debug_tiles_visited.argtypes = [_vp, ctypes.POINTER(ctypes.c_ulonglong)]
 lib.mfa_debug_set_decode_split_pages.restype = _i
 lib.mfa_debug_set_decode_split_pages.argtypes = [_i]
 
-EXPORTED = ("mfa_fwd", "mfa_fwd_varlen", "mfa_decode_workspace_size", "mfa_decode_splitkv", "mfa_status_string",
+EXPORTED = ("mfa_fwd", "mfa_fwd_varlen", "mfa_fwd_blocksparse", "mfa_decode_workspace_size", "mfa_decode_splitkv", "mfa_status_string",
             "mfa_last_launch_info", "mfa_device_status", "mfa_debug_set_flags",
             "mfa_debug_tiles_visited", "mfa_debug_set_decode_split_pages",
             "mfa_decode_splitkv_noalloc")
@@ -259,4 +261,32 @@ def mfa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, out=None, 
                             float(scale), int(bool(causal)), int(wl), int(wr), float(softcap),
                             _dtype_code(q), _stream(stream))
     _check(rc, "mfa_fwd_varlen")
+    return out, lse
+
+
+def mfa_fwd_blocksparse(q, k, v, block_mask, out=None, lse=None, *, scale=None, causal=False,
+                        window=(-1, -1), softcap=0.0, return_lse=True, stream=None):
+    """Block-sparse forward. q [B,Hq,Nq,D], k/v [B,Hkv,Nk,D], block_mask uint8
+    [B,Hq,ceil(Nq/128),ceil(Nk/128)] on the device; returns (out, lse or None)."""
+    torch = _torch()
+    B, Hq, Nq, D = q.shape
+    _, Hkv, Nk, _ = k.shape
+    if k.shape != v.shape or k.shape[0] != B or k.shape[3] != D:
+        raise ValueError("k and v must be [B, Hkv, Nk, D] matching q")
+    if q.dtype != k.dtype or q.dtype != v.dtype:
+        raise TypeError("q, k and v must share one dtype")
+    want = (B, Hq, -(-Nq // 128), -(-Nk // 128))
+    if block_mask.dtype != torch.uint8 or tuple(block_mask.shape) != want:
+        raise ValueError(f"block_mask must be uint8 of shape {want}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    wl, wr = window
+    rc = lib.mfa_fwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(block_mask),
+                                 B, Hq, Hkv, Nq, Nk, D, float(scale), int(bool(causal)), int(wl),
+                                 int(wr), float(softcap), _dtype_code(q), _stream(stream))
+    _check(rc, "mfa_fwd_blocksparse")
     return out, lse

@@ -46,6 +46,7 @@ constexpr int kFwdThreads = 384;  // 8 softmax warps + producer + MMA + 2 idle
 #endif
 constexpr bool kQKBehindPV = MFA_QK_BEHIND_PV != 0;
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kFwdMaxSparseTiles = 2048;  // key tiles a block-sparse row may span (262,144 keys)
 #ifndef MFA_POLY_MASK
 #define MFA_POLY_MASK 0x0ull
 #endif
@@ -64,6 +65,9 @@ struct FwdParams {
   const int* cu_q;
   const int* cu_k;
   int total_q, total_k;
+  // block-sparse: uint8 [B, Hq, nqt, nkt], one entry per 128-row x 128-key block (0 = skip)
+  const uint8_t* block_mask;
+  int nqt, nkt;
   int B, Hq, Hkv, Nq, Nk, G;
   int causal, win_l, win_r;
   int n_qblk;       // number of 256-row query blocks per head
@@ -75,7 +79,7 @@ struct FwdParams {
   float lse_mul;    // ln 2
 };
 
-template <int D>
+template <int D, bool SPARSE>
 struct FwdSmem {
   static constexpr int kTileBytes = kFwdBM * D * 2;  // one 128 x D tile of 16-bit values
   static constexpr int kSlabBytes = 128 * 128;       // 128 rows x 64 columns (128 B) slab
@@ -91,11 +95,14 @@ struct FwdSmem {
   uint64_t bar_final;
   uint32_t tmem_base;
   int abort;
+  int n_act;                                  // block-sparse: key tiles this CTA visits
+  uint16_t act_tile[SPARSE ? kFwdMaxSparseTiles : 1];  // ... their indices (from kt_lo), ascending
+  uint8_t act_bits[SPARSE ? kFwdMaxSparseTiles : 1];   // ... bit t: Q tile t's block is on
 };
 
-template <int D>
+template <int D, bool SPARSE>
 constexpr int fwd_smem_bytes() {
-  return (int)sizeof(FwdSmem<D>) + 1024;  // + alignment slack for the 1024-byte swizzle atoms
+  return (int)sizeof(FwdSmem<D, SPARSE>) + 1024;  // + alignment slack for the 1024-byte swizzle atoms
 }
 
 // Visible key range [lo, hi) of absolute query positions [a0, a1] (inclusive) among Nk keys.
@@ -110,10 +117,13 @@ __device__ __forceinline__ void key_range(const FwdParams& p, int Nk, int a0, in
 // VARLEN: q / out are [total_q, Hq, D] and k / v [total_k, Hkv, D] with per-sequence offsets
 // (cu_q, cu_k), read through tensor maps ordered (D, head, token); lse is [Hq, total_q]. Otherwise q / out are [B, Hq, Nq, D], k / v
 // [B, Hkv, Nk, D] and lse [B, Hq, Nq].
-template <int D, bool BF16, bool VARLEN>
+// SPARSE: dense layout plus a block mask; a CTA visits only key tiles whose block is on for one
+// of its Q tiles, and a Q tile whose block is off on a visited tile masks it entirely.
+template <int D, bool BF16, bool VARLEN, bool SPARSE>
 __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_constant__ FwdParams p) {
+  static_assert(!(VARLEN && SPARSE), "block masks are defined on the dense layout");
   extern __shared__ uint8_t smem_raw[];
-  FwdSmem<D>& sm = *reinterpret_cast<FwdSmem<D>*>(
+  FwdSmem<D, SPARSE>& sm = *reinterpret_cast<FwdSmem<D, SPARSE>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
   const int warp = threadIdx.x >> 5;
@@ -174,7 +184,35 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     mbar_init(smem_u32(&sm.bar_final), 1);
     sm.abort = 0;
     fence_barrier_init();
-    if ((p.flags & 2) && n_tiles > 0) atomicAdd(p.tile_counter, (unsigned long long)n_tiles);
+  }
+  if (SPARSE && warp == 0) {
+    // Active key tiles of the block mask rows of this CTA's two Q tiles, compacted in order:
+    // 32 lanes read 8 tiles each per step (all loads issued before the ballots).
+    const int qt0 = q0 / kFwdBM;
+    const uint8_t* r0 = p.block_mask + ((size_t)(b * p.Hq + h) * p.nqt + qt0) * p.nkt + kt_lo;
+    const uint8_t* r1 = (qt0 + 1 < p.nqt) ? r0 + p.nkt : nullptr;
+    int count = 0;
+    for (int base = 0; base < n_tiles; base += 32 * 8) {
+      uint8_t a0[8], a1[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int jj = base + i * 32 + lane;
+        a0[i] = jj < n_tiles ? r0[jj] : 0;
+        a1[i] = (r1 != nullptr && jj < n_tiles) ? r1[jj] : 0;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const bool act = (a0[i] | a1[i]) != 0;
+        const unsigned bal = __ballot_sync(0xffffffffu, act);
+        if (act) {
+          const int pos = count + __popc(bal & ((1u << lane) - 1u));
+          sm.act_tile[pos] = (uint16_t)(base + i * 32 + lane);
+          sm.act_bits[pos] = (uint8_t)((a0[i] != 0 ? 1 : 0) | (a1[i] != 0 ? 2 : 0));
+        }
+        count += __popc(bal);
+      }
+    }
+    if (lane == 0) sm.n_act = count;
   }
   if (warp == 9) {
     tmem_alloc(smem_u32(&sm.tmem_base), 512);
@@ -189,17 +227,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  // the key tiles every role walks: u-th visited tile = kt_lo + tile_of(u)
+  const int n_act = SPARSE ? sm.n_act : n_tiles;
+  auto tile_of = [&](int u) -> int {
+    if constexpr (SPARSE) return sm.act_tile[u]; else return u;
+  };
+  if (threadIdx.x == 0 && (p.flags & 2) && n_act > 0)
+    atomicAdd(p.tile_counter, (unsigned long long)n_act);
   volatile int* abort = &sm.abort;
 
   constexpr int kSlabs = D / 64;
-  constexpr uint32_t kTileBytes = FwdSmem<D>::kTileBytes;
-  constexpr int kSlab = FwdSmem<D>::kSlabBytes;
+  constexpr uint32_t kTileBytes = FwdSmem<D, SPARSE>::kTileBytes;
+  constexpr int kSlab = FwdSmem<D, SPARSE>::kSlabBytes;
 
   if (warp >= 8) {
    regs_control();
    if (warp == 8) {
     // ================================================================ TMA producer
-    if (lane == 0 && n_tiles > 0) {
+    if (lane == 0 && n_act > 0) {
       const uint32_t bq = smem_u32(&sm.bar_q);
       mbar_expect_tx(bq, kFwdQT * kTileBytes);
       for (int t = 0; t < kFwdQT; ++t)
@@ -210,10 +255,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
             tma_load_3d(smem_u32(sm.q[t]) + sl * kSlab, &p.tm_q, bq, sl * 64, q0 + t * kFwdBM,
                         b * p.Hq + h);
       int issued_k[kFwdStages] = {0, 0}, issued_v[kFwdStages] = {0, 0};
-      for (int j = 0; j < n_tiles; ++j) {
-        const int s = j % kFwdStages;
-        const int use = j / kFwdStages;
-        const int row = (kt_lo + j) * kFwdBN;
+      for (int u = 0; u < n_act; ++u) {
+        const int s = u % kFwdStages;
+        const int use = u / kFwdStages;
+        const int row = (kt_lo + tile_of(u)) * kFwdBN;
         if (use > 0 && !mbar_wait(smem_u32(&sm.bar_k_empty[s]), (use - 1) & 1, abort, 801)) break;
         const uint32_t bk = smem_u32(&sm.bar_k_full[s]);
         mbar_expect_tx(bk, kTileBytes);
@@ -239,7 +284,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     }
   } else if (warp == 9) {
     // ================================================================ MMA issuer
-    if (lane == 0 && n_tiles > 0) {
+    if (lane == 0 && n_act > 0) {
       const uint32_t idesc_qk = idesc_f16(BF16 ? 1 : 0, kFwdBM, kFwdBN, 0);
       const uint32_t idesc_pv = idesc_f16(BF16 ? 1 : 0, kFwdBM, D, 1);
       auto issue_qk = [&](int t, int s) {
@@ -263,12 +308,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         }
       };
       bool ok = mbar_wait(smem_u32(&sm.bar_q), 0, abort, 901);
-      for (int j = 0; ok && j < n_tiles; ++j) {
+      for (int j = 0; ok && j < n_act; ++j) {  // j counts visited tiles
         const int s = j % kFwdStages;
         const uint32_t ph = (j / kFwdStages) & 1;
         const int s1 = (j + 1) % kFwdStages;
         const uint32_t ph1 = ((j + 1) / kFwdStages) & 1;
-        const bool more = j + 1 < n_tiles;
+        const bool more = j + 1 < n_act;
         if (j == 0) {
           if (!(ok = mbar_wait(smem_u32(&sm.bar_k_full[s]), ph, abort, 902))) break;
           tc_fence_after();
@@ -334,7 +379,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     float m_run = -INFINITY;  // running max of the stored (scaled, capped) score
     float l_run = 0.f;
 
-    for (int j = 0; j < n_tiles; ++j) {
+    for (int j = 0; j < n_act; ++j) {  // j counts visited tiles
       const bool got = mbar_wait(smem_u32(&sm.bar_s_full[t]), j & 1, abort, 1001 + t);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
@@ -346,7 +391,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       tmem_wait_ld();
       float* s = reinterpret_cast<float*>(sraw);
 
-      const int k0 = (kt_lo + j) * kFwdBN;
+      const int k0 = (kt_lo + tile_of(j)) * kFwdBN;
+      // block-sparse: this Q tile's block is off on a tile visited for the other Q tile
+      const bool off_block = SPARSE && !((sm.act_bits[SPARSE ? j : 0] >> t) & 1);
       // Softcap: the capped score is cap * tanh(s * scale / cap); the value kept per key is that
       // divided by scale, so the exponent factor c = scale * log2 e is the same as without a cap.
       // When every |y| = |s| * scale / cap of this warp's rows is small, tanh(y) = y * q(y^2) is
@@ -377,10 +424,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       if (p.win_r >= 0) interior = interior && (k0 + kFwdBN - 1 <= a_lo + p.win_r);
       if (p.win_l >= 0) interior = interior && (k0 >= a_hi - p.win_l);
       if (p.flags & 1) interior = false;
+      if (off_block) interior = false;
       if (!interior) {
         int jhi = Nk - k0;                                     // keys >= Nk
         if (p.causal) jhi = min(jhi, a - k0 + 1);
         if (p.win_r >= 0) jhi = min(jhi, a + p.win_r - k0 + 1);
+        if (off_block) jhi = 0;
         const int jlo = (p.win_l >= 0) ? (a - p.win_l - k0) : -1;
 #pragma unroll
         for (int i = 0; i < 128; ++i) s[i] = (i < jhi && i >= jlo) ? s[i] : -INFINITY;
@@ -492,8 +541,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
 
     // ---- epilogue: O / l, LSE
     bool have_o = false;
-    if (n_tiles > 0 && !*abort) {
-      have_o = mbar_wait(smem_u32(&sm.bar_o_done[t]), (n_tiles - 1) & 1, abort, 1003 + t);
+    if (n_act > 0 && !*abort) {
+      have_o = mbar_wait(smem_u32(&sm.bar_o_done[t]), (n_act - 1) & 1, abort, 1003 + t);
       tc_fence_after();
     }
     have_o = __all_sync(0xffffffffu, have_o);

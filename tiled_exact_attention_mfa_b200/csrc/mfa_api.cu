@@ -144,16 +144,17 @@ struct FwdCall {
   int dtype;
   const int32_t *cu_q, *cu_k;
   int total_q, total_k;
+  const uint8_t* block_mask;  // block-sparse: [B, Hq, ceil(Nq/128), ceil(Nk/128)]
 };
 
-template <int D, bool BF16, bool VARLEN>
+template <int D, bool BF16, bool VARLEN, bool SPARSE>
 int launch_fwd(const FwdCall& c, cudaStream_t st) {
   const int B = c.B, Hq = c.Hq, Hkv = c.Hkv, Nq = c.Nq, Nk = c.Nk, dtype = c.dtype;
   const float scale = c.scale, softcap = c.softcap;
   static bool smem_done[kMaxDevices] = {};
   static bool regs_ok[kMaxDevices] = {};
-  constexpr int smem = mfa::fwd_smem_bytes<D>();
-  auto kernel = mfa::mfa_fwd_kernel<D, BF16, VARLEN>;
+  constexpr int smem = mfa::fwd_smem_bytes<D, SPARSE>();
+  auto kernel = mfa::mfa_fwd_kernel<D, BF16, VARLEN, SPARSE>;
   if (!ensure_smem(kernel, smem, smem_done)) return MFA_ERR_CUDA;
   {
     // setmaxnreg redistributes the registers the CTA launched with; refuse to launch if the
@@ -185,6 +186,11 @@ int launch_fwd(const FwdCall& c, cudaStream_t st) {
   }
   p.out = c.out;
   p.lse = c.lse;
+  if (SPARSE) {
+    p.block_mask = c.block_mask;
+    p.nqt = (Nq + mfa::kFwdBM - 1) / mfa::kFwdBM;
+    p.nkt = (Nk + mfa::kFwdBN - 1) / mfa::kFwdBN;
+  }
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -289,11 +295,12 @@ int launch_fill_empty(void* out, float* lse, size_t rows, int D, int dtype, cuda
   return MFA_OK;
 }
 
-template <bool VARLEN>
+template <bool VARLEN, bool SPARSE>
 int dispatch_fwd(const FwdCall& c, int D, cudaStream_t st) {
   const bool bf = c.dtype == MFA_DTYPE_BF16;
-  if (D == 128) return bf ? launch_fwd<128, true, VARLEN>(c, st) : launch_fwd<128, false, VARLEN>(c, st);
-  return bf ? launch_fwd<64, true, VARLEN>(c, st) : launch_fwd<64, false, VARLEN>(c, st);
+  if (D == 128)
+    return bf ? launch_fwd<128, true, VARLEN, SPARSE>(c, st) : launch_fwd<128, false, VARLEN, SPARSE>(c, st);
+  return bf ? launch_fwd<64, true, VARLEN, SPARSE>(c, st) : launch_fwd<64, false, VARLEN, SPARSE>(c, st);
 }
 
 }  // namespace
@@ -316,8 +323,30 @@ int mfa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (Nk == 0) return launch_fill_empty(out, lse, (size_t)B * Hq * Nq, D, dtype, st);
   FwdCall c = {q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, scale, causal, win_l, win_r, softcap, dtype,
-               nullptr, nullptr, 0, 0};
-  return dispatch_fwd<false>(c, D, st);
+               nullptr, nullptr, 0, 0, nullptr};
+  return dispatch_fwd<false, false>(c, D, st);
+}
+
+int mfa_fwd_blocksparse(const void* q, const void* k, const void* v, void* out, float* lse,
+                        const uint8_t* block_mask, int B, int Hq, int Hkv, int Nq, int Nk, int D,
+                        float scale, int causal, int win_l, int win_r, float softcap, int dtype,
+                        void* stream) {
+  int rc = validate_fwd_common(Hq, Hkv, D, dtype, win_l, win_r, softcap, scale);
+  if (rc != MFA_OK) return rc;
+  if (B < 0 || Nq < 0 || Nk < 0) return MFA_ERR_BAD_SHAPE;
+  if ((rc = check_sizes(B, Hq, Nq, D)) != MFA_OK) return rc;
+  if ((rc = check_sizes(B, Hkv, Nk, D)) != MFA_OK) return rc;
+  if ((long long)B * Hq > 0x7FFFFFFFLL || (long long)B * Hkv > 0x7FFFFFFFLL) return MFA_ERR_BAD_SHAPE;
+  if ((long long)(Nk + mfa::kFwdBN - 1) / mfa::kFwdBN > mfa::kFwdMaxSparseTiles) return MFA_ERR_UNSUPPORTED;
+  if (B == 0 || Hq == 0 || Nq == 0) return MFA_OK;
+  if (!q || !out || !block_mask || (Nk > 0 && (!k || !v))) return MFA_ERR_NULL_POINTER;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(lse) || (Nk > 0 && (!aligned16(k) || !aligned16(v))))
+    return MFA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (Nk == 0) return launch_fill_empty(out, lse, (size_t)B * Hq * Nq, D, dtype, st);
+  FwdCall c = {q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, scale, causal, win_l, win_r, softcap, dtype,
+               nullptr, nullptr, 0, 0, block_mask};
+  return dispatch_fwd<false, true>(c, D, st);
 }
 
 int mfa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
@@ -341,8 +370,8 @@ int mfa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (total_k == 0) return launch_fill_empty(out, lse, (size_t)total_q * Hq, D, dtype, st);
   FwdCall c = {q, k, v, out, lse, B, Hq, Hkv, max_seqlen_q, 0, scale, causal, win_l, win_r, softcap,
-               dtype, cu_seqlens_q, cu_seqlens_k, total_q, total_k};
-  return dispatch_fwd<true>(c, D, st);
+               dtype, cu_seqlens_q, cu_seqlens_k, total_q, total_k, nullptr};
+  return dispatch_fwd<true, false>(c, D, st);
 }
 
 static int validate_decode(int B, int Nq, int Hq, int Hkv, int D, int page_size, int max_pages) {
