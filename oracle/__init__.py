@@ -22,6 +22,10 @@ Sources (web pages, cited by title and section):
   * "mlx-mfa 2.5.2" Features: variable-length packed sequences with cu_seqlens; "mlx-mfa
     2.61.0" (essential correctness update): varlen causal with N_q < N_k changed toward the
     bottom-right alignment used here per sequence.
+  * "mlx-bun 0.4.0 -> 1.0.0, src/model/flash-attention.ts", Backward: three passes that
+    recompute the scores — D_i = rowsum(dO_i * O_i); per key row p = exp(s - L_i),
+    dp = dO_i . v_j, ds = p (dp - D_i), dV_j += p dO_i, dK_j += ds q_i scale; per query row
+    dq_i += ds k_j scale.
   * "mlx-mfa 2.5.2" Features and Usage: block-sparse attention, flash_attention_sparse(q, k, v,
     block_mask, causal=...), a block mask whose zero blocks are never attended; here a block is
     `block` query rows x `block` keys and the mask further restricts the causal / window set.
@@ -42,8 +46,8 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = ["visible", "attention", "attention_rows", "attention_varlen", "attention_varlen_rows",
-           "attention_blocksparse", "attention_blocksparse_rows", "paged_gather", "decode",
-           "decode_rows"]
+           "attention_blocksparse", "attention_blocksparse_rows", "attention_backward",
+           "paged_gather", "decode", "decode_rows"]
 
 
 def visible(Nq: int, Nk: int, causal: bool, win_l: int = -1, win_r: int = -1) -> np.ndarray:
@@ -235,6 +239,49 @@ def attention_blocksparse_rows(q, k, v, block_mask, rows, scale, causal=False, w
                                 (vis & keep)[None, :], scale, softcap)
         o[n], lse[n] = oi[0], li[0]
     return o, lse
+
+
+def attention_backward(q, k, v, do, scale, causal=False, win_l=-1, win_r=-1, softcap=0.0):
+    """Gradients of sum(O * dO) with O the forward above: returns (dq, dk, dv) in fp64 with the
+    shapes of q, k, v. Written from the definition: for each (b, h) the probabilities P are
+    materialised, dV = P^T dO, dP = dO V^T, D = rowsum(dO * O), dC = P * (dP - D), and with a cap
+    dS = dC * (1 - tanh^2(s / cap)) (the derivative of cap * tanh(s / cap)), dQ = scale dS K,
+    dK = scale dS^T Q (summed over the query heads of a kv group)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    B, Hq, Nq, D = q.shape
+    _, Hkv, Nk, _ = k.shape
+    G = Hq // Hkv
+    vis = visible(Nq, Nk, causal, win_l, win_r)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            s = scale * (q[b, h] @ k[b, g].T)
+            if softcap > 0:
+                t = np.tanh(s / softcap)
+                c = softcap * t
+            else:
+                c = s
+            c = np.where(vis, c, -np.inf)
+            m = np.max(c, axis=1, keepdims=True)
+            m = np.where(np.isfinite(m), m, 0.0)
+            w = np.where(vis, np.exp(c - m), 0.0)
+            l = w.sum(axis=1, keepdims=True)
+            p = np.divide(w, l, out=np.zeros_like(w), where=l > 0)
+            o = p @ v[b, g]
+            dp = do[b, h] @ v[b, g].T
+            dvec = np.sum(do[b, h] * o, axis=1, keepdims=True)
+            dc = p * (dp - dvec)
+            ds = dc * (1.0 - t * t) if softcap > 0 else dc
+            dq[b, h] = scale * (ds @ k[b, g])
+            dk[b, g] += scale * (ds.T @ q[b, h])
+            dv[b, g] += p.T @ do[b, h]
+    return dq, dk, dv
 
 
 def paged_gather(k_pages, v_pages, block_table, seq_len: int, b: int, page_size: int = 16):

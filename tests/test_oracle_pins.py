@@ -485,3 +485,79 @@ def test_blocksparse_rows_helper_matches_full():
                                                    softcap=3.0, block=blk)
     np.testing.assert_allclose(orow, o[rows[:, 0], rows[:, 1], rows[:, 2]], rtol=0, atol=1e-13)
     np.testing.assert_array_equal(np.isneginf(lrow), np.isneginf(lse[rows[:, 0], rows[:, 1], rows[:, 2]]))
+
+
+# ---------------------------------------------------------------- backward
+def _torch_grads(q, k, v, do, scale, mask):
+    G = q.shape[1] // k.shape[1]
+    qt, kt, vt = (torch.from_numpy(x).requires_grad_(True) for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(
+        qt, kt.repeat_interleave(G, dim=1), vt.repeat_interleave(G, dim=1), attn_mask=mask,
+        scale=scale)
+    (o * torch.from_numpy(do)).sum().backward()
+    return qt.grad.numpy(), kt.grad.numpy(), vt.grad.numpy()
+
+
+@pytest.mark.parametrize("case", [
+    (1, 4, 2, 23, 31, 8, False, -1, -1),
+    (2, 2, 2, 30, 30, 8, True, -1, -1),
+    (1, 6, 3, 25, 40, 4, True, 7, 0),
+    (1, 2, 1, 33, 33, 8, False, 5, 3),
+])
+def test_backward_matches_torch_autograd(case):
+    """Against torch autograd through fp64 SDPA (rows with at least one visible key)."""
+    B, Hq, Hkv, Nq, Nk, D, causal, wl, wr = case
+    q = rng.standard_normal((B, Hq, Nq, D))
+    k = rng.standard_normal((B, Hkv, Nk, D))
+    v = rng.standard_normal((B, Hkv, Nk, D))
+    do = rng.standard_normal((B, Hq, Nq, D))
+    mask = band_mask_torch(Nq, Nk, causal, wl, wr)
+    assert bool(mask.any(dim=1).all()), "every row needs a visible key for the torch reference"
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, 0.35, causal, wl, wr)
+    tq, tk, tv = _torch_grads(q, k, v, do, 0.35, mask)
+    np.testing.assert_allclose(dq, tq, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dk, tk, rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dv, tv, rtol=0, atol=1e-11)
+
+
+def test_backward_softcap_matches_finite_differences():
+    """With a cap (no library reference): central differences of sum(O * dO) through the forward
+    oracle, on every coordinate of a small case."""
+    B, Hq, Hkv, Nq, Nk, D = 1, 2, 1, 5, 7, 3
+    q = rng.standard_normal((B, Hq, Nq, D))
+    k = rng.standard_normal((B, Hkv, Nk, D))
+    v = rng.standard_normal((B, Hkv, Nk, D))
+    do = rng.standard_normal((B, Hq, Nq, D))
+    cap, scale, eps = 1.7, 0.9, 1e-6
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, scale, True, 3, -1, softcap=cap)
+
+    def loss(q_, k_, v_):
+        o, _ = oracle.attention(q_, k_, v_, scale, True, 3, -1, softcap=cap)
+        return float(np.sum(o * do))
+
+    for x, g in ((q, dq), (k, dk), (v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            x[idx] += eps
+            up = loss(q, k, v)
+            x[idx] -= 2 * eps
+            dn = loss(q, k, v)
+            x[idx] += eps
+            num[idx] = (up - dn) / (2 * eps)
+        np.testing.assert_allclose(g, num, rtol=0, atol=2e-8)
+
+
+def test_backward_gqa_is_mha_on_repeated_heads_and_empty_rows_give_zero():
+    B, Hq, Hkv, Nq, Nk, D = 1, 4, 2, 12, 9, 4
+    q = rng.standard_normal((B, Hq, Nq, D))
+    k = rng.standard_normal((B, Hkv, Nk, D))
+    v = rng.standard_normal((B, Hkv, Nk, D))
+    do = rng.standard_normal((B, Hq, Nq, D))
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, 0.5, True)
+    kr, vr = np.repeat(k, 2, axis=1), np.repeat(v, 2, axis=1)
+    dq2, dk2, dv2 = oracle.attention_backward(q, kr, vr, do, 0.5, True)
+    np.testing.assert_allclose(dq, dq2, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dk, dk2.reshape(B, Hkv, 2, Nk, D).sum(axis=2), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dv, dv2.reshape(B, Hkv, 2, Nk, D).sum(axis=2), rtol=0, atol=1e-13)
+    # Nq > Nk causal: the first Nq - Nk rows see no key, so their dq is zero
+    assert np.all(dq[:, :, :Nq - Nk] == 0)
