@@ -6,6 +6,7 @@
  *                      native GQA, optional tanh softcap, optional fp32 log-sum-exp output.
  *   mfa_fwd_varlen     the same forward over packed variable-length sequences (cu_seqlens).
  *   mfa_fwd_blocksparse the same forward restricted by a 128 x 128 block mask.
+ *   mfa_bwd            backward of mfa_fwd (dq, dk, dv from out and lse).
  *   mfa_decode_splitkv two-phase split-KV decode (N_q <= 4) over a paged KV cache.
  *
  * Sources (web pages, cited by title and section):
@@ -146,6 +147,37 @@ int mfa_fwd_blocksparse(const void* q, const void* k, const void* v, void* out, 
                         const uint8_t* block_mask,
                         int B, int Hq, int Hkv, int Nq, int Nk, int D, float scale,
                         int causal, int win_l, int win_r, float softcap, int dtype, void* stream);
+
+/*
+ * mfa_bwd_workspace_size -- bytes of scratch mfa_bwd needs: one fp32 per query row
+ * (rowsum(dO * O)), 256-byte rounded. Returns 0 for invalid arguments.
+ */
+size_t mfa_bwd_workspace_size(int B, int Hq, int Nq);
+
+/*
+ * mfa_bwd -- backward of mfa_fwd: the gradients of sum(out * dout) with respect to q, k, v,
+ * given the forward's out and lse ([MLXBUN] Backward: three passes -- D-vec, dKV, dQ -- that
+ * recompute the scores from the saved log-sum-exp).
+ *
+ * With p_ij = exp(c_ij - lse_i) for visible pairs (c the scaled, optionally capped score),
+ *   D_i  = sum_d dout[i,d] out[i,d],   dp_ij = <dout_i, v_j>,
+ *   ds_ij = p_ij (dp_ij - D_i) (times 1 - tanh^2(s_ij / softcap) when softcap > 0),
+ *   dq_i = scale sum_j ds_ij k_j,  dk_j = scale sum_i ds_ij q_i,  dv_j = sum_i p_ij dout_i,
+ * with dk, dv summed over the query heads of each kv group. Every output element is written
+ * by exactly one thread (no atomics): repeated calls give bitwise the same result.
+ *
+ * Arguments
+ *   q, out, dout, dq  [B, Hq, Nq, D] dtype     k, v, dk, dv [B, Hkv, Nk, D] dtype    (device)
+ *   lse  [B, Hq, Nq] float32 as written by mfa_fwd for the same arguments              (device)
+ *   workspace: device scratch of at least mfa_bwd_workspace_size(B, Hq, Nq) bytes, 256-byte
+ *   aligned, caller-owned; other arguments as mfa_fwd. Nk == 0 gives dq = 0; Nq == 0 gives
+ *   dk = dv = 0. Returns MFA_OK after the launches were queued.
+ */
+int mfa_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
+            const float* lse, void* dq, void* dk, void* dv,
+            int B, int Hq, int Hkv, int Nq, int Nk, int D, float scale,
+            int causal, int win_l, int win_r, float softcap, int dtype,
+            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * mfa_decode_workspace_size -- bytes of scratch mfa_decode_splitkv needs for this shape.

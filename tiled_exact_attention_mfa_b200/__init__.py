@@ -36,6 +36,10 @@ lib.mfa_fwd_varlen.restype = _i
 lib.mfa_fwd_varlen.argtypes = [_vp] * 7 + [_i] * 7 + [_f, _i, _i, _i, _f, _i, _vp]
 lib.mfa_fwd_blocksparse.restype = _i
 lib.mfa_fwd_blocksparse.argtypes = [_vp] * 6 + [_i] * 6 + [_f, _i, _i, _i, _f, _i, _vp]
+lib.mfa_bwd_workspace_size.restype = ctypes.c_size_t
+lib.mfa_bwd_workspace_size.argtypes = [_i, _i, _i]
+lib.mfa_bwd.restype = _i
+lib.mfa_bwd.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _i, _i, _i, _f, _i, _vp, ctypes.c_size_t, _vp]
 lib.mfa_decode_workspace_size.restype = ctypes.c_size_t
 lib.mfa_decode_workspace_size.argtypes = [_i] * 7
 lib.mfa_decode_splitkv.restype = _i
@@ -69,7 +73,8 @@ lib.mfa_debug_tiles_visited.argtypes = [_vp, ctypes.POINTER(ctypes.c_ulonglong)]
 lib.mfa_debug_set_decode_split_pages.restype = _i
 lib.mfa_debug_set_decode_split_pages.argtypes = [_i]
 
-EXPORTED = ("mfa_fwd", "mfa_fwd_varlen", "mfa_fwd_blocksparse", "mfa_decode_workspace_size", "mfa_decode_splitkv", "mfa_status_string",
+EXPORTED = ("mfa_fwd", "mfa_fwd_varlen", "mfa_fwd_blocksparse", "mfa_bwd_workspace_size", "mfa_bwd",
+            "mfa_decode_workspace_size", "mfa_decode_splitkv", "mfa_status_string",
             "mfa_last_launch_info", "mfa_device_status", "mfa_debug_set_flags",
             "mfa_debug_tiles_visited", "mfa_debug_set_decode_split_pages",
             "mfa_decode_splitkv_noalloc")
@@ -290,3 +295,38 @@ def mfa_fwd_blocksparse(q, k, v, block_mask, out=None, lse=None, *, scale=None, 
                                  int(wr), float(softcap), _dtype_code(q), _stream(stream))
     _check(rc, "mfa_fwd_blocksparse")
     return out, lse
+
+
+def mfa_bwd_workspace_size(B: int, Hq: int, Nq: int) -> int:
+    return lib.mfa_bwd_workspace_size(B, Hq, Nq)
+
+
+def mfa_bwd(q, k, v, out, dout, lse, dq=None, dk=None, dv=None, *, scale=None, causal=False,
+            window=(-1, -1), softcap=0.0, workspace=None, stream=None):
+    """Backward of mfa_fwd: gradients of sum(out * dout) given the forward's out and lse.
+    q/dq/out/dout [B,Hq,Nq,D], k/v/dk/dv [B,Hkv,Nk,D], lse [B,Hq,Nq] fp32; returns (dq, dk, dv)."""
+    torch = _torch()
+    B, Hq, Nq, D = q.shape
+    _, Hkv, Nk, _ = k.shape
+    for t in (out, dout):
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("out and dout must match q")
+    if k.shape != v.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("k and v must be [B, Hkv, Nk, D] of q's dtype")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, Hq, Nq):
+        raise ValueError("lse must be float32 [B, Hq, Nq]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = mfa_bwd_workspace_size(B, Hq, Nq)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    wl, wr = window
+    rc = lib.mfa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq),
+                     _ptr(dk), _ptr(dv), B, Hq, Hkv, Nq, Nk, D, float(scale), int(bool(causal)),
+                     int(wl), int(wr), float(softcap), _dtype_code(q), _ptr(workspace),
+                     workspace.numel(), _stream(stream))
+    _check(rc, "mfa_bwd")
+    return dq, dk, dv

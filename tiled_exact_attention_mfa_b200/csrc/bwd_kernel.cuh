@@ -1,0 +1,655 @@
+// bwd_kernel.cuh -- exact attention backward for sm_100a: dQ, dK, dV of sum(O * dO).
+//
+// Algorithm: the three-pass FlashAttention-2 backward of "mlx-bun 0.4.0 -> 1.0.0,
+// src/model/flash-attention.ts" (Backward: D-vec, dKV and dQ dispatches that recompute the scores
+// from the saved log-sum-exp L): D_i = rowsum(dO_i * O_i); for a visible pair (i, j)
+// p = exp(c_ij - L_i) with c the (capped) scaled score, dp = dO_i . v_j, ds = p (dp - D_i)
+// (times 1 - tanh^2(s / cap) with a cap), dV_j += p dO_i, dK_j += scale ds q_i,
+// dQ_i += scale ds k_j. No pass writes another pass's output, so every output is computed by
+// one CTA and the result is deterministic (no atomics).
+//
+// B200 mapping. Both main passes run one CTA of 192 threads per 128-row tile:
+//   warps 0-3  elementwise: one TMEM lane = one row of the CTA's tile (a key row in the dKV
+//              pass, a query row in the dQ pass); the 128 scores and 128 dP values of the row
+//              are processed 32 columns at a time, P and dS packed to the input type and
+//              stored back over the columns they came from.
+//   warp 4     producer: TMA loads of the streamed tiles through a 2-stage ring (plus, in the
+//              dKV pass, the 128 L and D values of each query tile, bounds-checked loads).
+//   warp 5     TMEM owner and single-thread tcgen05.mma issuer.
+// dKV pass (CTA = 128 keys of one kv head; loops over the query heads of its group and the
+//   query tiles that can see the keys): S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = 128
+//   queries, K = D, operands K-major in smem), then dV += P^T dO and dK += dS^T Q (P^T, dS^T
+//   from TMEM; dO, Q read MN-major from the same smem tiles). TMEM: S^T [0,128), dP^T
+//   [128,256), dV [256,256+D), dK [256+D,256+2D).
+// dQ pass (CTA = 128 query rows of one head; loops over the key tiles the rows can see):
+//   S = Q K^T, dP = dO V^T, then dQ += dS K (dS from TMEM, K MN-major). TMEM: S [0,128),
+//   dP [128,256), dQ [256,256+D).
+// The next step's S / dP MMAs overwrite the columns that hold P / dS, so the MMA thread waits
+// for the previous step's consuming MMAs to complete before issuing them (tcgen05 orders only
+// MMAs that share an accumulator).
+#pragma once
+#include "sm100.cuh"
+
+namespace mfa {
+
+constexpr int kBwdBM = 128;          // rows per tile (TMEM lanes), keys or queries
+constexpr int kBwdThreads = 192;     // 4 elementwise warps + producer + MMA
+constexpr int kBwdStages = 2;
+
+struct BwdParams {
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;  // [B*H][N][D] maps, 64 x 128 boxes, 128-byte swizzle
+  const uint16_t* o;                    // [B, Hq, Nq, D] forward output
+  const uint16_t* dout;                 // [B, Hq, Nq, D]
+  const float* lse;                     // [B, Hq, Nq] natural-log LSE from the forward
+  float* dvec;                          // [B, Hq, Nq] workspace: rowsum(dO * O)
+  void* dq;                             // [B, Hq, Nq, D]
+  void* dk;                             // [B, Hkv, Nk, D]
+  void* dv;                             // [B, Hkv, Nk, D]
+  int B, Hq, Hkv, Nq, Nk, G;
+  int causal, win_l, win_r;
+  int n_qt, n_kt;                       // 128-row query / key tiles per head
+  float scale;
+  float c_log2;                         // scale * log2 e
+  float softcap, cap_in;                // cap, scale / cap (softcap = 0: off)
+};
+
+// ---------------------------------------------------------------- D-vec pass
+// D_i = sum_d dO[i, d] * O[i, d] in fp32, one warp per row.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) mfa_bwd_dvec_kernel(const __grid_constant__ BwdParams p) {
+  const size_t rows = (size_t)p.B * p.Hq * p.Nq;
+  const int lane = threadIdx.x & 31;
+  const size_t warps = (size_t)gridDim.x * (blockDim.x >> 5);
+  for (size_t r = (size_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const uint16_t* o = p.o + r * D;
+    const uint16_t* g = p.dout + r * D;
+    float acc = 0.f;
+#pragma unroll
+    for (int d = lane * 2; d < D; d += 64) {
+      const uint32_t ov = *reinterpret_cast<const uint32_t*>(o + d);
+      const uint32_t gv = *reinterpret_cast<const uint32_t*>(g + d);
+      float o0, o1, g0, g1;
+      unpack2<BF16>(ov, o0, o1);
+      unpack2<BF16>(gv, g0, g1);
+      acc = fmaf(o0, g0, fmaf(o1, g1, acc));
+    }
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    if (lane == 0) p.dvec[r] = acc;
+  }
+}
+
+// Visible query rows [i_lo, i_hi] (inclusive, possibly empty) of key j: query i at absolute
+// position a = i + Nk - Nq sees j iff (!causal || j <= a) && (win_l < 0 || j >= a - win_l) &&
+// (win_r < 0 || j <= a + win_r).
+__device__ __forceinline__ void bwd_rows_of_key(const BwdParams& p, int j, int& i_lo, int& i_hi) {
+  const int off = p.Nk - p.Nq;
+  int a_lo = -0x3fffffff, a_hi = 0x3fffffff;
+  if (p.causal) a_lo = max(a_lo, j);
+  if (p.win_r >= 0) a_lo = max(a_lo, j - p.win_r);
+  if (p.win_l >= 0) a_hi = min(a_hi, j + p.win_l);
+  i_lo = max(0, a_lo - off);
+  i_hi = min(p.Nq - 1, a_hi - off);
+}
+
+// Visible keys [j_lo, j_hi] (inclusive, possibly empty) of query row i.
+__device__ __forceinline__ void bwd_keys_of_row(const BwdParams& p, int i, int& j_lo, int& j_hi) {
+  const int a = i + p.Nk - p.Nq;
+  j_lo = 0;
+  j_hi = p.Nk - 1;
+  if (p.causal) j_hi = min(j_hi, a);
+  if (p.win_r >= 0) j_hi = min(j_hi, a + p.win_r);
+  if (p.win_l >= 0) j_lo = max(j_lo, a - p.win_l);
+}
+
+// tanh(y) for the softcap derivative and value: the small-argument polynomial when the whole
+// warp's arguments allow it, else 1 - 2 / (2^(2|y| log2 e) + 1) with the sign restored.
+__device__ __forceinline__ float bwd_tanh(float y, bool poly) {
+  return poly ? y * tanh_q(y * y) : tanh_from_exp(y);
+}
+
+// ---------------------------------------------------------------- dKV pass
+template <int D>
+struct BwdKvSmem {
+  static constexpr int kTile = kBwdBM * D * 2;
+  uint8_t k[kTile];
+  uint8_t v[kTile];
+  uint8_t q[kBwdStages][kTile];
+  uint8_t dout[kBwdStages][kTile];
+  float nl[kBwdStages][kBwdBM];  // L_i log2 e of the stage's query rows (0 past Nq / no key)
+  float dd[kBwdStages][kBwdBM];  // D_i of the stage's query rows
+  uint64_t bar_kv, bar_full[kBwdStages], bar_empty[kBwdStages];
+  uint64_t bar_sp, bar_ds, bar_mm, bar_final;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int D>
+constexpr int bwd_kv_smem_bytes() {
+  return (int)sizeof(BwdKvSmem<D>) + 1024;
+}
+
+// 128 x D tile of 16-bit values at smem address a as a K-major operand, K step kk (16 columns).
+__device__ __forceinline__ uint64_t bwd_desc_k(uint32_t a, int kk) {
+  return smem_desc_sw128(a + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+}
+// The same tile as an MN-major B operand (rows = K dimension), K step kk (16 rows).
+__device__ __forceinline__ uint64_t bwd_desc_mn(uint32_t a, int kk) {
+  return smem_desc_sw128(a + kk * 16 * 128, 128 * 128, 1024);
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dkv_kernel(const __grid_constant__ BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  BwdKvSmem<D>& sm = *reinterpret_cast<BwdKvSmem<D>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: key tile kt of (b, kv head g); early key tiles (seen by the most causal rows) first
+  const int BK = p.B * p.Hkv;
+  const int kt = (int)(blockIdx.x / BK);
+  const int b = (int)(blockIdx.x % BK) / p.Hkv;
+  const int g = (int)(blockIdx.x % BK) % p.Hkv;
+  const int k0 = kt * kBwdBM;
+  const int k_last = min(k0 + kBwdBM, p.Nk) - 1;
+  // Query rows that see some key of the tile: the first key's lowest row to the last key's
+  // highest (both bounds grow with the key index).
+  int r_lo, r_hi, t0, t1;
+  bwd_rows_of_key(p, k0, r_lo, t0);
+  bwd_rows_of_key(p, k_last, t1, r_hi);
+  const int qt_lo = r_lo / kBwdBM;
+  const int n_qt = (r_hi >= r_lo) ? r_hi / kBwdBM - qt_lo + 1 : 0;
+  const int n_steps = n_qt * p.G;  // query heads of the group x query tiles, head-major
+
+  constexpr int kSlabs = D / 64;
+  constexpr uint32_t kTile = BwdKvSmem<D>::kTile;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&sm.bar_kv), 1);
+    for (int st = 0; st < kBwdStages; ++st) {
+      mbar_init(smem_u32(&sm.bar_full[st]), 1);
+      mbar_init(smem_u32(&sm.bar_empty[st]), 1);
+    }
+    mbar_init(smem_u32(&sm.bar_sp), 1);
+    mbar_init(smem_u32(&sm.bar_ds), 4);
+    mbar_init(smem_u32(&sm.bar_mm), 1);
+    mbar_init(smem_u32(&sm.bar_final), 1);
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(&sm.tmem_base), 512);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+    tma_prefetch_desc(&p.tm_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+
+  if (warp == 4) {
+    // ================================================================ producer
+    if (n_steps > 0) {
+      if (lane == 0) {
+        const uint32_t bkv = smem_u32(&sm.bar_kv);
+        mbar_expect_tx(bkv, 2 * kTile);
+        for (int sl = 0; sl < kSlabs; ++sl) {
+          tma_load_3d(smem_u32(sm.k) + sl * 128 * 128, &p.tm_k, bkv, sl * 64, k0, b * p.Hkv + g);
+          tma_load_3d(smem_u32(sm.v) + sl * 128 * 128, &p.tm_v, bkv, sl * 64, k0, b * p.Hkv + g);
+        }
+      }
+      int issued[kBwdStages] = {};
+      for (int u = 0; u < n_steps; ++u) {
+        const int st = u % kBwdStages;
+        const int use = u / kBwdStages;
+        const int h = g * p.G + u / n_qt;
+        const int row0 = (qt_lo + u % n_qt) * kBwdBM;
+        const bool ok = use == 0 || mbar_wait(smem_u32(&sm.bar_empty[st]), (use - 1) & 1, abort, 1101);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        // L (as L log2 e) and D of the tile's rows, 0 past Nq or where L = -inf (no visible key)
+        const size_t base = (size_t)(b * p.Hq + h) * p.Nq;
+#pragma unroll
+        for (int rr = 0; rr < kBwdBM; rr += 32) {
+          const int i = row0 + rr + lane;
+          float l = 0.f, d = 0.f;
+          if (i < p.Nq) {
+            l = p.lse[base + i];
+            d = p.dvec[base + i];
+            if (!(l > -INFINITY)) l = 0.f;
+          }
+          sm.nl[st][rr + lane] = l * 1.4426950408889634f;
+          sm.dd[st][rr + lane] = d;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          const uint32_t bf = smem_u32(&sm.bar_full[st]);
+          mbar_expect_tx(bf, 2 * kTile);
+          for (int sl = 0; sl < kSlabs; ++sl) {
+            tma_load_3d(smem_u32(sm.q[st]) + sl * 128 * 128, &p.tm_q, bf, sl * 64, row0, b * p.Hq + h);
+            tma_load_3d(smem_u32(sm.dout[st]) + sl * 128 * 128, &p.tm_do, bf, sl * 64, row0, b * p.Hq + h);
+          }
+          issued[st] = use + 1;
+        }
+      }
+      if (lane == 0) {  // no copy into this CTA's shared memory may outlive it
+        volatile int no_abort = 0;
+        mbar_wait(smem_u32(&sm.bar_kv), 0, &no_abort, 1102);
+        for (int st = 0; st < kBwdStages; ++st)
+          if (issued[st] > 0) mbar_wait(smem_u32(&sm.bar_full[st]), (issued[st] - 1) & 1, &no_abort, 1103);
+      }
+    }
+  } else if (warp == 5) {
+    // ================================================================ MMA issuer
+    if (lane == 0 && n_steps > 0) {
+      const uint32_t id_s = idesc_f16(BF16 ? 1 : 0, kBwdBM, kBwdBM, 0);  // S^T, dP^T: 128 x 128
+      const uint32_t id_o = idesc_f16(BF16 ? 1 : 0, kBwdBM, D, 1);       // dV, dK: B MN-major
+      const uint32_t ka = smem_u32(sm.k), va = smem_u32(sm.v);
+      bool ok = mbar_wait(smem_u32(&sm.bar_kv), 0, abort, 1201);
+      for (int u = 0; ok && u < n_steps; ++u) {
+        const int st = u % kBwdStages;
+        if (!(ok = mbar_wait(smem_u32(&sm.bar_full[st]), (u / kBwdStages) & 1, abort, 1202))) break;
+        // P^T / dS^T of step u - 1 live in the S^T / dP^T columns until dV / dK have read them
+        if (u > 0 && !(ok = mbar_wait(smem_u32(&sm.bar_mm), (u - 1) & 1, abort, 1203))) break;
+        tc_fence_after();
+        const uint32_t qa = smem_u32(sm.q[st]), oa = smem_u32(sm.dout[st]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          tc_mma_ss(tmem + 0, bwd_desc_k(ka, kk), bwd_desc_k(qa, kk), id_s, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          tc_mma_ss(tmem + 128, bwd_desc_k(va, kk), bwd_desc_k(oa, kk), id_s, kk > 0 ? 1u : 0u);
+        tc_commit(smem_u32(&sm.bar_sp));
+        if (!(ok = mbar_wait(smem_u32(&sm.bar_ds), u & 1, abort, 1204))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBwdBM / 16; ++kk)
+          tc_mma_ts(tmem + 256, tmem + 0 + kk * 8, bwd_desc_mn(oa, kk), id_o, (u > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < kBwdBM / 16; ++kk)
+          tc_mma_ts(tmem + 256 + D, tmem + 128 + kk * 8, bwd_desc_mn(qa, kk), id_o, (u > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(smem_u32(&sm.bar_mm));
+        tc_commit(smem_u32(&sm.bar_empty[st]));
+      }
+      tc_commit(smem_u32(&sm.bar_final));
+      volatile int no_abort = 0;
+      mbar_wait(smem_u32(&sm.bar_final), 0, &no_abort, 1205);
+    }
+  } else {
+    // ================================================================ elementwise (key rows)
+    const int r = warp * 32 + lane;
+    const int j = k0 + r;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t t_s = tmem + lane_base;
+    const uint32_t t_dp = tmem + lane_base + 128;
+    int ilo, ihi;
+    bwd_rows_of_key(p, j, ilo, ihi);
+    if (j >= p.Nk) {
+      ilo = 1;
+      ihi = 0;
+    }
+    const float c = p.c_log2;
+    const float cc = p.softcap * 1.4426950408889634f;
+    int u = 0;
+    for (; u < n_steps; ++u) {
+      const int st = u % kBwdStages;
+      const int row0 = (qt_lo + u % n_qt) * kBwdBM;
+      const bool got = mbar_wait(smem_u32(&sm.bar_sp), u & 1, abort, 1301);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const bool interior = __all_sync(0xffffffffu, ilo <= row0 && row0 + kBwdBM - 1 <= ihi);
+#pragma unroll 1
+      for (int qc = 0; qc < 4; ++qc) {
+        uint32_t sr[32], dr[32];
+        tmem_ld32(t_s + qc * 32, sr);
+        tmem_ld32(t_dp + qc * 32, dr);
+        tmem_wait_ld();
+        float nlv[32], ddv[32];
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 a = *reinterpret_cast<const float4*>(&sm.nl[st][qc * 32 + i4 * 4]);
+          const float4 d4 = *reinterpret_cast<const float4*>(&sm.dd[st][qc * 32 + i4 * 4]);
+          nlv[i4 * 4 + 0] = a.x; nlv[i4 * 4 + 1] = a.y; nlv[i4 * 4 + 2] = a.z; nlv[i4 * 4 + 3] = a.w;
+          ddv[i4 * 4 + 0] = d4.x; ddv[i4 * 4 + 1] = d4.y; ddv[i4 * 4 + 2] = d4.z; ddv[i4 * 4 + 3] = d4.w;
+        }
+        bool poly = false;
+        if (p.softcap > 0.f) {
+          float am = 0.f;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) am = fmaxf(am, fabsf(__uint_as_float(sr[e])));
+          poly = __all_sync(0xffffffffu, am * p.cap_in <= kTanhPolyMax);
+        }
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int e2 = 0; e2 < 16; ++e2) {
+          float pv[2], dsv[2];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int e = 2 * e2 + h2;
+            const float sv = __uint_as_float(sr[e]);
+            float x, fac = 1.f;
+            if (p.softcap > 0.f) {
+              const float tt = bwd_tanh(sv * p.cap_in, poly);
+              x = fmaf(tt, cc, -nlv[e]);
+              fac = fmaf(-tt, tt, 1.f);
+            } else {
+              x = fmaf(sv, c, -nlv[e]);
+            }
+            float pe = fast_exp2(x);
+            const int i = row0 + qc * 32 + e;
+            if (!interior && (i < ilo || i > ihi)) pe = 0.f;
+            pv[h2] = pe;
+            dsv[h2] = pe * (__uint_as_float(dr[e]) - ddv[e]) * fac;
+          }
+          pk[e2] = pack2<BF16>(pv[0], pv[1]);
+          dk[e2] = pack2<BF16>(dsv[0], dsv[1]);
+        }
+        tmem_st16(t_s + qc * 16, pk);
+        tmem_st16(t_dp + qc * 16, dk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.bar_ds));
+    }
+    // ---- epilogue: dV and scale * dK of this key row
+    bool have = false;
+    if (n_steps > 0 && !*abort) {
+      have = mbar_wait(smem_u32(&sm.bar_mm), (n_steps - 1) & 1, abort, 1302);
+      tc_fence_after();
+    }
+    have = __all_sync(0xffffffffu, have);
+    const size_t obase = ((size_t)(b * p.Hkv + g) * p.Nk + (size_t)j) * D;
+#pragma unroll 1
+    for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
+      const float mul = which ? p.scale : 1.f;
+      uint16_t* dst_base = reinterpret_cast<uint16_t*>(which ? p.dk : p.dv);
+#pragma unroll
+      for (int cb = 0; cb < D; cb += 32) {
+        uint32_t o[32];
+        if (have) {
+          tmem_ld32(tmem + lane_base + 256 + which * D + cb, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        if (j < p.Nk) {
+          uint4* dst = reinterpret_cast<uint4*>(dst_base + obase + cb);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 w;
+            w.x = pack2<BF16>(__uint_as_float(o[v4 * 8 + 0]) * mul, __uint_as_float(o[v4 * 8 + 1]) * mul);
+            w.y = pack2<BF16>(__uint_as_float(o[v4 * 8 + 2]) * mul, __uint_as_float(o[v4 * 8 + 3]) * mul);
+            w.z = pack2<BF16>(__uint_as_float(o[v4 * 8 + 4]) * mul, __uint_as_float(o[v4 * 8 + 5]) * mul);
+            w.w = pack2<BF16>(__uint_as_float(o[v4 * 8 + 6]) * mul, __uint_as_float(o[v4 * 8 + 7]) * mul);
+            dst[v4] = w;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- dQ pass
+template <int D>
+struct BwdQSmem {
+  static constexpr int kTile = kBwdBM * D * 2;
+  uint8_t q[kTile];
+  uint8_t dout[kTile];
+  uint8_t k[kBwdStages][kTile];
+  uint8_t v[kBwdStages][kTile];
+  uint64_t bar_qo, bar_full[kBwdStages], bar_empty[kBwdStages];
+  uint64_t bar_sp, bar_ds, bar_mm, bar_final;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int D>
+constexpr int bwd_q_smem_bytes() {
+  return (int)sizeof(BwdQSmem<D>) + 1024;
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  BwdQSmem<D>& sm = *reinterpret_cast<BwdQSmem<D>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: query tile qt of (b, h); late query tiles (most keys under causal) first
+  const int BH = p.B * p.Hq;
+  const int qt = p.n_qt - 1 - (int)(blockIdx.x / BH);
+  const int b = (int)(blockIdx.x % BH) / p.Hq;
+  const int h = (int)(blockIdx.x % BH) % p.Hq;
+  const int g = h / p.G;
+  const int q0 = qt * kBwdBM;
+  const int q_last = min(q0 + kBwdBM, p.Nq) - 1;
+  // keys seen by some row of the tile: the first row's lowest key to the last row's highest
+  int j_lo, j_hi, t0, t1;
+  bwd_keys_of_row(p, q0, j_lo, t0);
+  bwd_keys_of_row(p, q_last, t1, j_hi);
+  const int kt_lo = max(j_lo, 0) / kBwdBM;
+  const int n_kt = (j_hi >= j_lo && j_hi >= 0) ? j_hi / kBwdBM - kt_lo + 1 : 0;
+
+  constexpr int kSlabs = D / 64;
+  constexpr uint32_t kTile = BwdQSmem<D>::kTile;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&sm.bar_qo), 1);
+    for (int st = 0; st < kBwdStages; ++st) {
+      mbar_init(smem_u32(&sm.bar_full[st]), 1);
+      mbar_init(smem_u32(&sm.bar_empty[st]), 1);
+    }
+    mbar_init(smem_u32(&sm.bar_sp), 1);
+    mbar_init(smem_u32(&sm.bar_ds), 4);
+    mbar_init(smem_u32(&sm.bar_mm), 1);
+    mbar_init(smem_u32(&sm.bar_final), 1);
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(&sm.tmem_base), 512);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+    tma_prefetch_desc(&p.tm_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+
+  if (warp == 4) {
+    // ================================================================ producer
+    if (lane == 0 && n_kt > 0) {
+      const uint32_t bqo = smem_u32(&sm.bar_qo);
+      mbar_expect_tx(bqo, 2 * kTile);
+      for (int sl = 0; sl < kSlabs; ++sl) {
+        tma_load_3d(smem_u32(sm.q) + sl * 128 * 128, &p.tm_q, bqo, sl * 64, q0, b * p.Hq + h);
+        tma_load_3d(smem_u32(sm.dout) + sl * 128 * 128, &p.tm_do, bqo, sl * 64, q0, b * p.Hq + h);
+      }
+      int issued[kBwdStages] = {};
+      for (int u = 0; u < n_kt; ++u) {
+        const int st = u % kBwdStages;
+        const int use = u / kBwdStages;
+        const int row = (kt_lo + u) * kBwdBM;
+        if (use > 0 && !mbar_wait(smem_u32(&sm.bar_empty[st]), (use - 1) & 1, abort, 1401)) break;
+        const uint32_t bf = smem_u32(&sm.bar_full[st]);
+        mbar_expect_tx(bf, 2 * kTile);
+        for (int sl = 0; sl < kSlabs; ++sl) {
+          tma_load_3d(smem_u32(sm.k[st]) + sl * 128 * 128, &p.tm_k, bf, sl * 64, row, b * p.Hkv + g);
+          tma_load_3d(smem_u32(sm.v[st]) + sl * 128 * 128, &p.tm_v, bf, sl * 64, row, b * p.Hkv + g);
+        }
+        issued[st] = use + 1;
+      }
+      volatile int no_abort = 0;
+      mbar_wait(bqo, 0, &no_abort, 1402);
+      for (int st = 0; st < kBwdStages; ++st)
+        if (issued[st] > 0) mbar_wait(smem_u32(&sm.bar_full[st]), (issued[st] - 1) & 1, &no_abort, 1403);
+    }
+  } else if (warp == 5) {
+    // ================================================================ MMA issuer
+    if (lane == 0 && n_kt > 0) {
+      const uint32_t id_s = idesc_f16(BF16 ? 1 : 0, kBwdBM, kBwdBM, 0);  // S, dP: 128 x 128
+      const uint32_t id_o = idesc_f16(BF16 ? 1 : 0, kBwdBM, D, 1);       // dQ: B MN-major
+      const uint32_t qa = smem_u32(sm.q), oa = smem_u32(sm.dout);
+      bool ok = mbar_wait(smem_u32(&sm.bar_qo), 0, abort, 1501);
+      for (int u = 0; ok && u < n_kt; ++u) {
+        const int st = u % kBwdStages;
+        if (!(ok = mbar_wait(smem_u32(&sm.bar_full[st]), (u / kBwdStages) & 1, abort, 1502))) break;
+        // dS of step u - 1 lives in the S columns until the dQ MMA has read it
+        if (u > 0 && !(ok = mbar_wait(smem_u32(&sm.bar_mm), (u - 1) & 1, abort, 1503))) break;
+        tc_fence_after();
+        const uint32_t ka = smem_u32(sm.k[st]), va = smem_u32(sm.v[st]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          tc_mma_ss(tmem + 0, bwd_desc_k(qa, kk), bwd_desc_k(ka, kk), id_s, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          tc_mma_ss(tmem + 128, bwd_desc_k(oa, kk), bwd_desc_k(va, kk), id_s, kk > 0 ? 1u : 0u);
+        tc_commit(smem_u32(&sm.bar_sp));
+        if (!(ok = mbar_wait(smem_u32(&sm.bar_ds), u & 1, abort, 1504))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBwdBM / 16; ++kk)
+          tc_mma_ts(tmem + 256, tmem + 0 + kk * 8, bwd_desc_mn(ka, kk), id_o, (u > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(smem_u32(&sm.bar_mm));
+        tc_commit(smem_u32(&sm.bar_empty[st]));
+      }
+      tc_commit(smem_u32(&sm.bar_final));
+      volatile int no_abort = 0;
+      mbar_wait(smem_u32(&sm.bar_final), 0, &no_abort, 1505);
+    }
+  } else {
+    // ================================================================ elementwise (query rows)
+    const int r = warp * 32 + lane;
+    const int i = q0 + r;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t t_s = tmem + lane_base;
+    const uint32_t t_dp = tmem + lane_base + 128;
+    int klo, khi;
+    bwd_keys_of_row(p, i, klo, khi);
+    float nl = 0.f, dd = 0.f;
+    if (i < p.Nq) {
+      const size_t idx = (size_t)(b * p.Hq + h) * p.Nq + i;
+      nl = p.lse[idx];
+      dd = p.dvec[idx];
+      if (!(nl > -INFINITY)) nl = 0.f;
+      nl *= 1.4426950408889634f;
+    } else {
+      klo = 1;
+      khi = 0;
+    }
+    const float c = p.c_log2;
+    const float cc = p.softcap * 1.4426950408889634f;
+    for (int u = 0; u < n_kt; ++u) {
+      const int k0 = (kt_lo + u) * kBwdBM;
+      const bool got = mbar_wait(smem_u32(&sm.bar_sp), u & 1, abort, 1601);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const bool interior = __all_sync(0xffffffffu, klo <= k0 && k0 + kBwdBM - 1 <= khi);
+#pragma unroll 1
+      for (int qc = 0; qc < 4; ++qc) {
+        uint32_t sr[32], dr[32];
+        tmem_ld32(t_s + qc * 32, sr);
+        tmem_ld32(t_dp + qc * 32, dr);
+        tmem_wait_ld();
+        bool poly = false;
+        if (p.softcap > 0.f) {
+          float am = 0.f;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) am = fmaxf(am, fabsf(__uint_as_float(sr[e])));
+          poly = __all_sync(0xffffffffu, am * p.cap_in <= kTanhPolyMax);
+        }
+        uint32_t dk[16];
+#pragma unroll
+        for (int e2 = 0; e2 < 16; ++e2) {
+          float dsv[2];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int e = 2 * e2 + h2;
+            const float sv = __uint_as_float(sr[e]);
+            float x, fac = 1.f;
+            if (p.softcap > 0.f) {
+              const float tt = bwd_tanh(sv * p.cap_in, poly);
+              x = fmaf(tt, cc, -nl);
+              fac = fmaf(-tt, tt, 1.f);
+            } else {
+              x = fmaf(sv, c, -nl);
+            }
+            float pe = fast_exp2(x);
+            const int j = k0 + qc * 32 + e;
+            if (!interior && (j < klo || j > khi)) pe = 0.f;
+            dsv[h2] = pe * (__uint_as_float(dr[e]) - dd) * fac;
+          }
+          dk[e2] = pack2<BF16>(dsv[0], dsv[1]);
+        }
+        tmem_st16(t_s + qc * 16, dk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.bar_ds));
+    }
+    // ---- epilogue: scale * dQ of this query row
+    bool have = false;
+    if (n_kt > 0 && !*abort) {
+      have = mbar_wait(smem_u32(&sm.bar_mm), (n_kt - 1) & 1, abort, 1602);
+      tc_fence_after();
+    }
+    have = __all_sync(0xffffffffu, have);
+    const size_t obase = ((size_t)(b * p.Hq + h) * p.Nq + (size_t)i) * D;
+#pragma unroll
+    for (int cb = 0; cb < D; cb += 32) {
+      uint32_t o[32];
+      if (have) {
+        tmem_ld32(tmem + lane_base + 256 + cb, o);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = 0u;
+      }
+      if (i < p.Nq) {
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.dq) + obase + cb);
+        const float m = p.scale;
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) {
+          uint4 w;
+          w.x = pack2<BF16>(__uint_as_float(o[v4 * 8 + 0]) * m, __uint_as_float(o[v4 * 8 + 1]) * m);
+          w.y = pack2<BF16>(__uint_as_float(o[v4 * 8 + 2]) * m, __uint_as_float(o[v4 * 8 + 3]) * m);
+          w.z = pack2<BF16>(__uint_as_float(o[v4 * 8 + 4]) * m, __uint_as_float(o[v4 * 8 + 5]) * m);
+          w.w = pack2<BF16>(__uint_as_float(o[v4 * 8 + 6]) * m, __uint_as_float(o[v4 * 8 + 7]) * m);
+          dst[v4] = w;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace mfa

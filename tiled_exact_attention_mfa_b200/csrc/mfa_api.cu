@@ -7,6 +7,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "bwd_kernel.cuh"
 #include "decode_kernel.cuh"
 #include "fwd_kernel.cuh"
 #include "mfa.h"
@@ -303,6 +304,43 @@ int dispatch_fwd(const FwdCall& c, int D, cudaStream_t st) {
   return bf ? launch_fwd<64, true, VARLEN, SPARSE>(c, st) : launch_fwd<64, false, VARLEN, SPARSE>(c, st);
 }
 
+template <int D, bool BF16>
+int launch_bwd(mfa::BwdParams& p, const void* q, const void* k, const void* v, const void* dout,
+               int dtype, cudaStream_t st) {
+  static bool smem_kv[kMaxDevices] = {}, smem_q[kMaxDevices] = {};
+  auto kdkv = mfa::mfa_bwd_dkv_kernel<D, BF16>;
+  auto kdq = mfa::mfa_bwd_dq_kernel<D, BF16>;
+  if (!ensure_smem(kdkv, mfa::bwd_kv_smem_bytes<D>(), smem_kv)) return MFA_ERR_CUDA;
+  if (!ensure_smem(kdq, mfa::bwd_q_smem_bytes<D>(), smem_q)) return MFA_ERR_CUDA;
+  if (!make_map(&p.tm_q, q, dtype, (long long)p.B * p.Hq, p.Nq, D)) return MFA_ERR_CUDA;
+  if (!make_map(&p.tm_do, dout, dtype, (long long)p.B * p.Hq, p.Nq, D)) return MFA_ERR_CUDA;
+  if (!make_map(&p.tm_k, k, dtype, (long long)p.B * p.Hkv, p.Nk, D)) return MFA_ERR_CUDA;
+  if (!make_map(&p.tm_v, v, dtype, (long long)p.B * p.Hkv, p.Nk, D)) return MFA_ERR_CUDA;
+  const long long rows = (long long)p.B * p.Hq * p.Nq;
+  long long g0 = (rows + 7) / 8;
+  if (g0 > 148 * 16) g0 = 148 * 16;
+  mfa::mfa_bwd_dvec_kernel<D, BF16><<<(unsigned)g0, 256, 0, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
+  const long long g1 = (long long)p.n_kt * p.B * p.Hkv;
+  const long long g2 = (long long)p.n_qt * p.B * p.Hq;
+  if (g1 > 0x7FFFFFFFLL || g2 > 0x7FFFFFFFLL) return MFA_ERR_BAD_SHAPE;
+  kdkv<<<(unsigned)g1, mfa::kBwdThreads, mfa::bwd_kv_smem_bytes<D>(), st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
+  kdq<<<(unsigned)g2, mfa::kBwdThreads, mfa::bwd_q_smem_bytes<D>(), st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
+  mfa_launch_info li = {};
+  li.kernel = 4;
+  li.grid_x = (int)g1;
+  li.grid_y = (int)g2;
+  li.grid_z = 1;
+  li.block_threads = mfa::kBwdThreads;
+  li.smem_bytes = mfa::bwd_kv_smem_bytes<D>();
+  li.tile_m = mfa::kBwdBM;
+  li.tile_n = mfa::kBwdBM;
+  g_last = li;
+  return MFA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -384,6 +422,71 @@ static int validate_decode(int B, int Nq, int Hq, int Hkv, int D, int page_size,
   if ((Hq / Hkv) * Nq > 16) return MFA_ERR_UNSUPPORTED;
   if ((long long)max_pages * mfa::kDecPage > 0x7FFFFFFFLL) return MFA_ERR_BAD_SHAPE;
   return MFA_OK;
+}
+
+size_t mfa_bwd_workspace_size(int B, int Hq, int Nq) {
+  if (B < 0 || Hq < 0 || Nq < 0) return 0;
+  if (check_sizes(B, Hq, Nq, 1) != MFA_OK) return 0;
+  return align256((size_t)B * Hq * Nq * sizeof(float));
+}
+
+int mfa_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
+            const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk,
+            int D, float scale, int causal, int win_l, int win_r, float softcap, int dtype,
+            void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = validate_fwd_common(Hq, Hkv, D, dtype, win_l, win_r, softcap, scale);
+  if (rc != MFA_OK) return rc;
+  if (B < 0 || Nq < 0 || Nk < 0) return MFA_ERR_BAD_SHAPE;
+  if ((rc = check_sizes(B, Hq, Nq, D)) != MFA_OK) return rc;
+  if ((rc = check_sizes(B, Hkv, Nk, D)) != MFA_OK) return rc;
+  if ((long long)B * Hq > 0x7FFFFFFFLL || (long long)B * Hkv > 0x7FFFFFFFLL) return MFA_ERR_BAD_SHAPE;
+  if (B == 0 || Hq == 0 || (Nq == 0 && Nk == 0)) return MFA_OK;
+  const bool need_q = Nq > 0, need_k = Nk > 0;
+  if ((need_q && (!q || !out || !dout || !lse || !dq)) || (need_k && (!k || !v || !dk || !dv)))
+    return MFA_ERR_NULL_POINTER;
+  if ((need_q && (!aligned16(q) || !aligned16(out) || !aligned16(dout) || !aligned16(lse) || !aligned16(dq))) ||
+      (need_k && (!aligned16(k) || !aligned16(v) || !aligned16(dk) || !aligned16(dv))))
+    return MFA_ERR_MISALIGNED;
+  const size_t need = mfa_bwd_workspace_size(B, Hq, Nq);
+  if (need_q && need_k &&
+      (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need))
+    return MFA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!need_k) {  // no keys: every query row sees nothing, so dQ = 0
+    return cudaMemsetAsync(dq, 0, (size_t)B * Hq * Nq * D * 2, st) == cudaSuccess ? MFA_OK : MFA_ERR_CUDA;
+  }
+  if (!need_q) {  // no queries: no key receives a gradient
+    if (cudaMemsetAsync(dk, 0, (size_t)B * Hkv * Nk * D * 2, st) != cudaSuccess) return MFA_ERR_CUDA;
+    return cudaMemsetAsync(dv, 0, (size_t)B * Hkv * Nk * D * 2, st) == cudaSuccess ? MFA_OK : MFA_ERR_CUDA;
+  }
+  mfa::BwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.o = static_cast<const uint16_t*>(out);
+  p.dout = static_cast<const uint16_t*>(dout);
+  p.lse = lse;
+  p.dvec = static_cast<float*>(workspace);
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.G = Hq / Hkv;
+  p.causal = causal ? 1 : 0;
+  p.win_l = win_l;
+  p.win_r = win_r;
+  p.n_qt = (Nq + mfa::kBwdBM - 1) / mfa::kBwdBM;
+  p.n_kt = (Nk + mfa::kBwdBM - 1) / mfa::kBwdBM;
+  p.scale = scale;
+  p.c_log2 = scale * 1.4426950408889634f;
+  p.softcap = softcap > 0.f ? softcap : 0.f;
+  p.cap_in = softcap > 0.f ? scale / softcap : 0.f;
+  const bool bf = dtype == MFA_DTYPE_BF16;
+  if (D == 128)
+    return bf ? launch_bwd<128, true>(p, q, k, v, dout, dtype, st) : launch_bwd<128, false>(p, q, k, v, dout, dtype, st);
+  return bf ? launch_bwd<64, true>(p, q, k, v, dout, dtype, st) : launch_bwd<64, false>(p, q, k, v, dout, dtype, st);
 }
 
 size_t mfa_decode_workspace_size(int B, int Nq, int Hq, int Hkv, int D, int max_pages_per_seq,

@@ -262,6 +262,20 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   return r;
 }
 
+// The two 16-bit values of a packed pair (low half first) widened exactly to fp32.
+template <bool BF16>
+__device__ __forceinline__ void unpack2(uint32_t v, float& lo, float& hi) {
+  if constexpr (BF16) {
+    lo = __uint_as_float(v << 16);
+    hi = __uint_as_float(v & 0xffff0000u);
+  } else {
+    const __half2 h = *reinterpret_cast<const __half2*>(&v);
+    const float2 f = __half22float2(h);
+    lo = f.x;
+    hi = f.y;
+  }
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
