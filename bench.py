@@ -327,6 +327,38 @@ def bench_sparse(case, steps, warmup, flush, stream, world):
             "density": float(m.mean())}
 
 
+def bench_backward(case, steps, warmup, flush, stream, world):
+    """mfa_bwd alone on the forward's outputs (computed once, outside the timed region).
+    Algorithmic work: 5 matmuls over the visible pairs (S recomputed, dP, dV, dK, dQ)."""
+    import torch
+    import tiled_exact_attention_mfa_b200 as mfa
+    dev = torch.device("cuda")
+    q, k, v = case.tensors()
+    qt, kt, vt = (upload(x, case.dtype, dev) for x in (q, k, v))
+    win = (case.win_l, case.win_r)
+    out, lse = mfa.mfa_fwd(qt, kt, vt, scale=case.scale_f32(), causal=case.causal, window=win,
+                           softcap=case.softcap, stream=stream)
+    dout = upload(mi.normal_bits(case.seed + 500, mi.STREAM_Q, tuple(qt.shape), case.dtype),
+                  case.dtype, dev)
+    dq, dk, dv = torch.empty_like(qt), torch.empty_like(kt), torch.empty_like(vt)
+    ws = torch.empty(max(mfa.mfa_bwd_workspace_size(case.B, case.Hq, case.Nq), 256),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        mfa.mfa_bwd(qt, kt, vt, out, dout, lse, dq, dk, dv, scale=case.scale_f32(),
+                    causal=case.causal, window=win, softcap=case.softcap, workspace=ws,
+                    stream=stream)
+
+    with torch.cuda.stream(stream):
+        ms, bracket = time_steps(step, steps, warmup, flush, stream)
+    return {"ms": max_over_ranks(statistics.mean(ms), world), "ms_min": min(ms),
+            "bracket_ms": bracket, "flops": 2.5 * prefill_flops(case),
+            "bytes": 2.0 * prefill_bytes(case)}
+
+
+BACKWARD_WORKLOADS = ("causal_b2_h8_n4096_d128_fp16", "noncausal_b2_h8_n4096_d128_fp16")
+
+
 def bench_decode(case, steps, warmup, flush, stream, world):
     import torch
     import tiled_exact_attention_mfa_b200 as mfa
@@ -424,6 +456,15 @@ def run_gpu(args):
                                "frac_of_measured_tensor_peak": round(tf / pk["tflops"], 4),
                                "frac_of_nominal_tensor_peak": round(tf / NOMINAL_TFLOPS, 4),
                                "frac_of_roofline": round(t_floor / (r["ms"] * 1e-3), 4)})
+        for name in BACKWARD_WORKLOADS:
+            sk, wu = max(3, min(args.steps, 10)), max(3, args.warmup)
+            r = bench_backward(W[name], sk, wu, flush, stream, world)
+            tf = r["flops"] * world / (r["ms"] * 1e-3) / 1e12
+            others.append({"workload": name + ":backward", "ms": round(r["ms"], 4),
+                           "unit": "TFLOP/s", "value": round(tf, 1),
+                           "frac_of_measured_tensor_peak": round(tf / pk["tflops"], 4),
+                           "frac_of_nominal_tensor_peak": round(tf / NOMINAL_TFLOPS, 4),
+                           "flops_convention": "2.5 x forward (S, dP, dV, dK, dQ over visible pairs)"})
     clk = clocks.stop()
     tflops = job_throughput(main["flops"], world, main["ms"]) / 1e12
     per_gpu_tflops = main["flops"] / (main["ms"] * 1e-3) / 1e12
@@ -541,8 +582,11 @@ def run_profile(args):
     torch.cuda.set_device(0)
     stream = torch.cuda.Stream()
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    case = mi.workloads()[args.profile]
-    if isinstance(case, mi.DecodeCase):
+    name, _, part = args.profile.partition(":")
+    case = mi.workloads()[name]
+    if part == "backward":
+        r = bench_backward(case, args.steps, args.warmup, lambda: flush_buf.fill_(1), stream, 1)
+    elif isinstance(case, mi.DecodeCase):
         r = bench_decode(case, args.steps, args.warmup, lambda: flush_buf.fill_(1), stream, 1)
     elif isinstance(case, mi.VarlenCase):
         r = bench_varlen(case, args.steps, args.warmup, lambda: flush_buf.fill_(1), stream, 1)
@@ -565,7 +609,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--profile", default=None, choices=sorted(mi.workloads()),
+    ap.add_argument("--profile", default=None,
+                    choices=sorted(mi.workloads()) + [n + ":backward" for n in BACKWARD_WORKLOADS],
                     help="time one workload alone (for profiler captures) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
