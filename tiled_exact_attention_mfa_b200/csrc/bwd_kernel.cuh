@@ -8,14 +8,13 @@
 // dQ_i += scale ds k_j. No pass writes another pass's output, so every output is computed by
 // one CTA and the result is deterministic (no atomics).
 //
-// B200 mapping. Both main passes run one CTA of 192 threads per 128-row tile:
-//   warps 0-3  elementwise: one TMEM lane = one row of the CTA's tile (a key row in the dKV
-//              pass, a query row in the dQ pass); the 128 scores and 128 dP values of the row
-//              are processed 32 columns at a time, P and dS packed to the input type and
-//              stored back over the columns they came from.
-//   warp 4     producer: TMA loads of the streamed tiles through a 2-stage ring (plus, in the
+// B200 mapping. Both main passes run one CTA of 384 threads per 128-row tile:
+//   warps 0-7  elementwise: a TMEM lane is a row of the CTA's tile (a key row in the dKV pass,
+//              a query row in the dQ pass) and two warps share each row, one per 64-column half
+//              of the 128 scores and 128 dP values; P and dS are packed to the input type.
+//   warp 8     producer: TMA loads of the streamed tiles through a 2-stage ring (plus, in the
 //              dKV pass, the 128 L and D values of each query tile, bounds-checked loads).
-//   warp 5     TMEM owner and single-thread tcgen05.mma issuer.
+//   warp 9     TMEM owner and single-thread tcgen05.mma issuer.
 // dKV pass (CTA = 128 keys of one kv head; loops over the query heads of its group and the
 //   query tiles that can see the keys): S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = 128
 //   queries, K = D, operands K-major in smem), then dV += P^T dO and dK += dS^T Q (P^T, dS^T
@@ -33,8 +32,11 @@
 namespace mfa {
 
 constexpr int kBwdBM = 128;          // rows per tile (TMEM lanes), keys or queries
-constexpr int kBwdThreads = 192;     // 4 elementwise warps + producer + MMA
 constexpr int kBwdStages = 2;
+// setmaxnreg split of both main passes (384 threads): two elementwise warpgroups grow to 216
+// registers, the producer / MMA warpgroup shrinks to 72; 256 x 216 + 128 x 72 = 384 x 168.
+constexpr int kBwdQRegsElem = 216;
+constexpr int kBwdQRegsCtl = 72;
 
 struct BwdParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_do;  // [B*H][N][D] maps, 64 x 128 boxes, 128-byte swizzle
@@ -109,6 +111,14 @@ __device__ __forceinline__ float bwd_tanh(float y, bool poly) {
 }
 
 // ---------------------------------------------------------------- dKV pass
+// 384 threads: warps 0-7 elementwise (warp w: key rows on TMEM lanes 32 (w % 4) .., query
+// columns 64 (w / 4) .. of each query tile), warp 8 producer, warp 9 MMA issuer, warps 10-11
+// idle; setmaxnreg as in the dQ pass. Each warp writes its 64 packed P^T (dS^T) values over
+// the first 32 of its own 64 S^T (dP^T) columns, so the two halves of a row never touch each
+// other's columns; the dV / dK MMAs take query steps 0-3 from columns 0-31 and steps 4-7 from
+// columns 64-95 of each region.
+constexpr int kBwdKvThreads = 384;
+
 template <int D>
 struct BwdKvSmem {
   static constexpr int kTile = kBwdBM * D * 2;
@@ -138,8 +148,8 @@ __device__ __forceinline__ uint64_t bwd_desc_mn(uint32_t a, int kk) {
   return smem_desc_sw128(a + kk * 16 * 128, 128 * 128, 1024);
 }
 
-template <int D, bool BF16>
-__global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dkv_kernel(const __grid_constant__ BwdParams p) {
+template <int D, bool BF16, bool SOFTCAP>
+__global__ void __launch_bounds__(kBwdKvThreads, 1) mfa_bwd_dkv_kernel(const __grid_constant__ BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   BwdKvSmem<D>& sm = *reinterpret_cast<BwdKvSmem<D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -171,17 +181,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dkv_kernel(const __gri
       mbar_init(smem_u32(&sm.bar_empty[st]), 1);
     }
     mbar_init(smem_u32(&sm.bar_sp), 1);
-    mbar_init(smem_u32(&sm.bar_ds), 4);
+    mbar_init(smem_u32(&sm.bar_ds), 8);
     mbar_init(smem_u32(&sm.bar_mm), 1);
     mbar_init(smem_u32(&sm.bar_final), 1);
     sm.abort = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(&sm.tmem_base), 512);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     tma_prefetch_desc(&p.tm_q);
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_v);
@@ -193,7 +203,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dkv_kernel(const __gri
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
 
-  if (warp == 4) {
+  if (warp >= 8) {
+   regs_dec<kBwdQRegsCtl>();
+   if (warp == 8) {
     // ================================================================ producer
     if (n_steps > 0) {
       if (lane == 0) {
@@ -244,7 +256,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dkv_kernel(const __gri
           if (issued[st] > 0) mbar_wait(smem_u32(&sm.bar_full[st]), (issued[st] - 1) & 1, &no_abort, 1103);
       }
     }
-  } else if (warp == 5) {
+   } else if (warp == 9) {
     // ================================================================ MMA issuer
     if (lane == 0 && n_steps > 0) {
       const uint32_t id_s = idesc_f16(BF16 ? 1 : 0, kBwdBM, kBwdBM, 0);  // S^T, dP^T: 128 x 128
@@ -267,12 +279,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dkv_kernel(const __gri
         tc_commit(smem_u32(&sm.bar_sp));
         if (!(ok = mbar_wait(smem_u32(&sm.bar_ds), u & 1, abort, 1204))) break;
         tc_fence_after();
+        // packed P^T / dS^T of query step kk (16 queries): half kk / 4 at column 64 (kk / 4)
 #pragma unroll
         for (int kk = 0; kk < kBwdBM / 16; ++kk)
-          tc_mma_ts(tmem + 256, tmem + 0 + kk * 8, bwd_desc_mn(oa, kk), id_o, (u > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + 256, tmem + (kk >> 2) * 64 + (kk & 3) * 8, bwd_desc_mn(oa, kk), id_o,
+                    (u > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < kBwdBM / 16; ++kk)
-          tc_mma_ts(tmem + 256 + D, tmem + 128 + kk * 8, bwd_desc_mn(qa, kk), id_o, (u > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + 256 + D, tmem + 128 + (kk >> 2) * 64 + (kk & 3) * 8, bwd_desc_mn(qa, kk),
+                    id_o, (u > 0 || kk > 0) ? 1u : 0u);
         tc_commit(smem_u32(&sm.bar_mm));
         tc_commit(smem_u32(&sm.bar_empty[st]));
       }
@@ -280,13 +295,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dkv_kernel(const __gri
       volatile int no_abort = 0;
       mbar_wait(smem_u32(&sm.bar_final), 0, &no_abort, 1205);
     }
+   }
   } else {
+    regs_inc<kBwdQRegsElem>();
     // ================================================================ elementwise (key rows)
-    const int r = warp * 32 + lane;
-    const int j = k0 + r;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t t_s = tmem + lane_base;
-    const uint32_t t_dp = tmem + lane_base + 128;
+    const int quarter = warp & 3;
+    const int half = warp >> 2;  // query columns 64 half .. 64 half + 63 of each query tile
+    const int j = k0 + quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     int ilo, ihi;
     bwd_rows_of_key(p, j, ilo, ihi);
     if (j >= p.Nk) {
@@ -295,30 +311,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dkv_kernel(const __gri
     }
     const float c = p.c_log2;
     const float cc = p.softcap * 1.4426950408889634f;
-    int u = 0;
-    for (; u < n_steps; ++u) {
+    for (int u = 0; u < n_steps; ++u) {
       const int st = u % kBwdStages;
-      const int row0 = (qt_lo + u % n_qt) * kBwdBM;
+      const int col0 = (qt_lo + u % n_qt) * kBwdBM + half * 64;  // query row of this warp's column 0
       const bool got = mbar_wait(smem_u32(&sm.bar_sp), u & 1, abort, 1301);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
-      const bool interior = __all_sync(0xffffffffu, ilo <= row0 && row0 + kBwdBM - 1 <= ihi);
+      const bool interior = __all_sync(0xffffffffu, ilo <= col0 && col0 + 63 <= ihi);
+      const float* nlp = &sm.nl[st][half * 64];
+      const float* ddp = &sm.dd[st][half * 64];
 #pragma unroll 1
-      for (int qc = 0; qc < 4; ++qc) {
+      for (int ch = 0; ch < 2; ++ch) {  // 32 query columns at a time, read then written in place
         uint32_t sr[32], dr[32];
-        tmem_ld32(t_s + qc * 32, sr);
-        tmem_ld32(t_dp + qc * 32, dr);
+        tmem_ld32(tmem + lane_base + half * 64 + ch * 32, sr);
+        tmem_ld32(tmem + lane_base + 128 + half * 64 + ch * 32, dr);
         tmem_wait_ld();
-        float nlv[32], ddv[32];
-#pragma unroll
-        for (int i4 = 0; i4 < 8; ++i4) {
-          const float4 a = *reinterpret_cast<const float4*>(&sm.nl[st][qc * 32 + i4 * 4]);
-          const float4 d4 = *reinterpret_cast<const float4*>(&sm.dd[st][qc * 32 + i4 * 4]);
-          nlv[i4 * 4 + 0] = a.x; nlv[i4 * 4 + 1] = a.y; nlv[i4 * 4 + 2] = a.z; nlv[i4 * 4 + 3] = a.w;
-          ddv[i4 * 4 + 0] = d4.x; ddv[i4 * 4 + 1] = d4.y; ddv[i4 * 4 + 2] = d4.z; ddv[i4 * 4 + 3] = d4.w;
-        }
         bool poly = false;
-        if (p.softcap > 0.f) {
+        if (SOFTCAP) {
           float am = 0.f;
 #pragma unroll
           for (int e = 0; e < 32; ++e) am = fmaxf(am, fabsf(__uint_as_float(sr[e])));
@@ -326,38 +335,46 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dkv_kernel(const __gri
         }
         uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int e2 = 0; e2 < 16; ++e2) {
-          float pv[2], dsv[2];
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 n4 = *reinterpret_cast<const float4*>(nlp + ch * 32 + e4 * 4);
+          const float4 d4 = *reinterpret_cast<const float4*>(ddp + ch * 32 + e4 * 4);
+          const float nv[4] = {n4.x, n4.y, n4.z, n4.w};
+          const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pv[4], dsv[4];
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int e = 2 * e2 + h2;
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int e = e4 * 4 + q4;
             const float sv = __uint_as_float(sr[e]);
             float x, fac = 1.f;
-            if (p.softcap > 0.f) {
+            if (SOFTCAP) {
               const float tt = bwd_tanh(sv * p.cap_in, poly);
-              x = fmaf(tt, cc, -nlv[e]);
+              x = fmaf(tt, cc, -nv[q4]);
               fac = fmaf(-tt, tt, 1.f);
             } else {
-              x = fmaf(sv, c, -nlv[e]);
+              x = fmaf(sv, c, -nv[q4]);
             }
             float pe = fast_exp2(x);
-            const int i = row0 + qc * 32 + e;
+            const int i = col0 + ch * 32 + e;
             if (!interior && (i < ilo || i > ihi)) pe = 0.f;
-            pv[h2] = pe;
-            dsv[h2] = pe * (__uint_as_float(dr[e]) - ddv[e]) * fac;
+            pv[q4] = pe;
+            dsv[q4] = pe * (__uint_as_float(dr[e]) - dv4[q4]) * fac;
           }
-          pk[e2] = pack2<BF16>(pv[0], pv[1]);
-          dk[e2] = pack2<BF16>(dsv[0], dsv[1]);
+          pk[2 * e4] = pack2<BF16>(pv[0], pv[1]);
+          pk[2 * e4 + 1] = pack2<BF16>(pv[2], pv[3]);
+          dk[2 * e4] = pack2<BF16>(dsv[0], dsv[1]);
+          dk[2 * e4 + 1] = pack2<BF16>(dsv[2], dsv[3]);
         }
-        tmem_st16(t_s + qc * 16, pk);
-        tmem_st16(t_dp + qc * 16, dk);
+        // packed values of columns 64 half + 32 ch .. land on columns 64 half + 16 ch .., which
+        // this warp has already read
+        tmem_st16(tmem + lane_base + half * 64 + ch * 16, pk);
+        tmem_st16(tmem + lane_base + 128 + half * 64 + ch * 16, dk);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.bar_ds));
     }
-    // ---- epilogue: dV and scale * dK of this key row
+    // ---- epilogue: lower-column warps write dV, upper-column warps scale * dK, of their key rows
     bool have = false;
     if (n_steps > 0 && !*abort) {
       have = mbar_wait(smem_u32(&sm.bar_mm), (n_steps - 1) & 1, abort, 1302);
@@ -365,31 +382,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dkv_kernel(const __gri
     }
     have = __all_sync(0xffffffffu, have);
     const size_t obase = ((size_t)(b * p.Hkv + g) * p.Nk + (size_t)j) * D;
-#pragma unroll 1
-    for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
-      const float mul = which ? p.scale : 1.f;
-      uint16_t* dst_base = reinterpret_cast<uint16_t*>(which ? p.dk : p.dv);
+    const float mul = half ? p.scale : 1.f;
+    uint16_t* dst_base = reinterpret_cast<uint16_t*>(half ? p.dk : p.dv);
 #pragma unroll
-      for (int cb = 0; cb < D; cb += 32) {
-        uint32_t o[32];
-        if (have) {
-          tmem_ld32(tmem + lane_base + 256 + which * D + cb, o);
-          tmem_wait_ld();
-        } else {
+    for (int cb = 0; cb < D; cb += 32) {
+      uint32_t o[32];
+      if (have) {
+        tmem_ld32(tmem + lane_base + 256 + half * D + cb, o);
+        tmem_wait_ld();
+      } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0u;
-        }
-        if (j < p.Nk) {
-          uint4* dst = reinterpret_cast<uint4*>(dst_base + obase + cb);
+        for (int e = 0; e < 32; ++e) o[e] = 0u;
+      }
+      if (j < p.Nk) {
+        uint4* dst = reinterpret_cast<uint4*>(dst_base + obase + cb);
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) {
-            uint4 w;
-            w.x = pack2<BF16>(__uint_as_float(o[v4 * 8 + 0]) * mul, __uint_as_float(o[v4 * 8 + 1]) * mul);
-            w.y = pack2<BF16>(__uint_as_float(o[v4 * 8 + 2]) * mul, __uint_as_float(o[v4 * 8 + 3]) * mul);
-            w.z = pack2<BF16>(__uint_as_float(o[v4 * 8 + 4]) * mul, __uint_as_float(o[v4 * 8 + 5]) * mul);
-            w.w = pack2<BF16>(__uint_as_float(o[v4 * 8 + 6]) * mul, __uint_as_float(o[v4 * 8 + 7]) * mul);
-            dst[v4] = w;
-          }
+        for (int v4 = 0; v4 < 4; ++v4) {
+          uint4 w;
+          w.x = pack2<BF16>(__uint_as_float(o[v4 * 8 + 0]) * mul, __uint_as_float(o[v4 * 8 + 1]) * mul);
+          w.y = pack2<BF16>(__uint_as_float(o[v4 * 8 + 2]) * mul, __uint_as_float(o[v4 * 8 + 3]) * mul);
+          w.z = pack2<BF16>(__uint_as_float(o[v4 * 8 + 4]) * mul, __uint_as_float(o[v4 * 8 + 5]) * mul);
+          w.w = pack2<BF16>(__uint_as_float(o[v4 * 8 + 6]) * mul, __uint_as_float(o[v4 * 8 + 7]) * mul);
+          dst[v4] = w;
         }
       }
     }
@@ -397,7 +411,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dkv_kernel(const __gri
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -405,6 +419,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dkv_kernel(const __gri
 }
 
 // ---------------------------------------------------------------- dQ pass
+// 384 threads: warps 0-7 elementwise (warp w: TMEM lanes 32 (w % 4) .., key columns
+// 64 (w / 4) ..), warp 8 producer, warp 9 MMA issuer, warps 10-11 idle (setmaxnreg works on
+// whole warpgroups: the elementwise warpgroups grow to 216 registers, the rest shrink to 72;
+// 256 x 216 + 128 x 72 = 384 x 168 is the pool the CTA launches with).
+// dS goes to two spare TMEM buffers [384, 448) and [448, 512), so S / dP of key tile u + 1 are
+// computed while the elementwise warps work on tile u: the MMA thread issues them as soon as
+// every elementwise warp has read S / dP of tile u (bar_ld), then dQ += dS K for tile u.
+constexpr int kBwdQThreads = 384;
+
 template <int D>
 struct BwdQSmem {
   static constexpr int kTile = kBwdBM * D * 2;
@@ -413,7 +436,7 @@ struct BwdQSmem {
   uint8_t k[kBwdStages][kTile];
   uint8_t v[kBwdStages][kTile];
   uint64_t bar_qo, bar_full[kBwdStages], bar_empty[kBwdStages];
-  uint64_t bar_sp, bar_ds, bar_mm, bar_final;
+  uint64_t bar_sp, bar_ld, bar_ds, bar_mm, bar_final;
   uint32_t tmem_base;
   int abort;
 };
@@ -423,8 +446,8 @@ constexpr int bwd_q_smem_bytes() {
   return (int)sizeof(BwdQSmem<D>) + 1024;
 }
 
-template <int D, bool BF16>
-__global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
+template <int D, bool BF16, bool SOFTCAP>
+__global__ void __launch_bounds__(kBwdQThreads, 1) mfa_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   BwdQSmem<D>& sm = *reinterpret_cast<BwdQSmem<D>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -455,17 +478,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dq_kernel(const __grid
       mbar_init(smem_u32(&sm.bar_empty[st]), 1);
     }
     mbar_init(smem_u32(&sm.bar_sp), 1);
-    mbar_init(smem_u32(&sm.bar_ds), 4);
+    mbar_init(smem_u32(&sm.bar_ld), 8);
+    mbar_init(smem_u32(&sm.bar_ds), 8);
     mbar_init(smem_u32(&sm.bar_mm), 1);
     mbar_init(smem_u32(&sm.bar_final), 1);
     sm.abort = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(&sm.tmem_base), 512);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     tma_prefetch_desc(&p.tm_q);
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_v);
@@ -477,7 +501,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dq_kernel(const __grid
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
 
-  if (warp == 4) {
+  if (warp >= 8) {
+   regs_dec<kBwdQRegsCtl>();
+   if (warp == 8) {
     // ================================================================ producer
     if (lane == 0 && n_kt > 0) {
       const uint32_t bqo = smem_u32(&sm.bar_qo);
@@ -505,18 +531,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dq_kernel(const __grid
       for (int st = 0; st < kBwdStages; ++st)
         if (issued[st] > 0) mbar_wait(smem_u32(&sm.bar_full[st]), (issued[st] - 1) & 1, &no_abort, 1403);
     }
-  } else if (warp == 5) {
+   } else if (warp == 9) {
     // ================================================================ MMA issuer
     if (lane == 0 && n_kt > 0) {
       const uint32_t id_s = idesc_f16(BF16 ? 1 : 0, kBwdBM, kBwdBM, 0);  // S, dP: 128 x 128
       const uint32_t id_o = idesc_f16(BF16 ? 1 : 0, kBwdBM, D, 1);       // dQ: B MN-major
       const uint32_t qa = smem_u32(sm.q), oa = smem_u32(sm.dout);
-      bool ok = mbar_wait(smem_u32(&sm.bar_qo), 0, abort, 1501);
-      for (int u = 0; ok && u < n_kt; ++u) {
+      auto issue_sdp = [&](int u) -> bool {
         const int st = u % kBwdStages;
-        if (!(ok = mbar_wait(smem_u32(&sm.bar_full[st]), (u / kBwdStages) & 1, abort, 1502))) break;
-        // dS of step u - 1 lives in the S columns until the dQ MMA has read it
-        if (u > 0 && !(ok = mbar_wait(smem_u32(&sm.bar_mm), (u - 1) & 1, abort, 1503))) break;
+        if (!mbar_wait(smem_u32(&sm.bar_full[st]), (u / kBwdStages) & 1, abort, 1502)) return false;
         tc_fence_after();
         const uint32_t ka = smem_u32(sm.k[st]), va = smem_u32(sm.v[st]);
 #pragma unroll
@@ -525,26 +548,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dq_kernel(const __grid
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           tc_mma_ss(tmem + 128, bwd_desc_k(oa, kk), bwd_desc_k(va, kk), id_s, kk > 0 ? 1u : 0u);
-        tc_commit(smem_u32(&sm.bar_sp));
+        tc_commit(smem_u32(&sm.bar_sp));  // also covers every earlier dQ MMA
+        return true;
+      };
+      bool ok = mbar_wait(smem_u32(&sm.bar_qo), 0, abort, 1501) && issue_sdp(0);
+      for (int u = 0; ok && u < n_kt; ++u) {
+        if (u + 1 < n_kt) {
+          // S / dP of tile u + 1 overwrite S / dP of tile u once every elementwise warp has read them
+          if (!(ok = mbar_wait(smem_u32(&sm.bar_ld), u & 1, abort, 1503))) break;
+          if (!(ok = issue_sdp(u + 1))) break;
+        }
         if (!(ok = mbar_wait(smem_u32(&sm.bar_ds), u & 1, abort, 1504))) break;
         tc_fence_after();
+        const uint32_t ka = smem_u32(sm.k[u % kBwdStages]);
+        const uint32_t ds_col = 384 + (u & 1) * 64;
 #pragma unroll
         for (int kk = 0; kk < kBwdBM / 16; ++kk)
-          tc_mma_ts(tmem + 256, tmem + 0 + kk * 8, bwd_desc_mn(ka, kk), id_o, (u > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + 256, tmem + ds_col + kk * 8, bwd_desc_mn(ka, kk), id_o, (u > 0 || kk > 0) ? 1u : 0u);
         tc_commit(smem_u32(&sm.bar_mm));
-        tc_commit(smem_u32(&sm.bar_empty[st]));
+        tc_commit(smem_u32(&sm.bar_empty[u % kBwdStages]));
       }
       tc_commit(smem_u32(&sm.bar_final));
       volatile int no_abort = 0;
       mbar_wait(smem_u32(&sm.bar_final), 0, &no_abort, 1505);
     }
+   }
   } else {
+    regs_inc<kBwdQRegsElem>();
     // ================================================================ elementwise (query rows)
-    const int r = warp * 32 + lane;
-    const int i = q0 + r;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t t_s = tmem + lane_base;
-    const uint32_t t_dp = tmem + lane_base + 128;
+    const int quarter = warp & 3;
+    const int half = warp >> 2;                 // key columns 64 half .. 64 half + 63 of each tile
+    const int i = q0 + quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     int klo, khi;
     bwd_keys_of_row(p, i, klo, khi);
     float nl = 0.f, dd = 0.f;
@@ -561,67 +596,73 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dq_kernel(const __grid
     const float c = p.c_log2;
     const float cc = p.softcap * 1.4426950408889634f;
     for (int u = 0; u < n_kt; ++u) {
-      const int k0 = (kt_lo + u) * kBwdBM;
+      const int kc0 = (kt_lo + u) * kBwdBM + half * 64;  // first key of this warp's columns
       const bool got = mbar_wait(smem_u32(&sm.bar_sp), u & 1, abort, 1601);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
-      const bool interior = __all_sync(0xffffffffu, klo <= k0 && k0 + kBwdBM - 1 <= khi);
-#pragma unroll 1
-      for (int qc = 0; qc < 4; ++qc) {
-        uint32_t sr[32], dr[32];
-        tmem_ld32(t_s + qc * 32, sr);
-        tmem_ld32(t_dp + qc * 32, dr);
-        tmem_wait_ld();
-        bool poly = false;
-        if (p.softcap > 0.f) {
-          float am = 0.f;
+      uint32_t sr[64], dr[64];
+      tmem_ld32(tmem + lane_base + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tmem + lane_base + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tmem + lane_base + 128 + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+      tmem_ld32(tmem + lane_base + 128 + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.bar_ld));  // S / dP columns may be overwritten now
+      const bool interior = __all_sync(0xffffffffu, klo <= kc0 && kc0 + 63 <= khi);
+      bool poly = false;
+      if (SOFTCAP) {
+        float am = 0.f;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) am = fmaxf(am, fabsf(__uint_as_float(sr[e])));
-          poly = __all_sync(0xffffffffu, am * p.cap_in <= kTanhPolyMax);
-        }
-        uint32_t dk[16];
-#pragma unroll
-        for (int e2 = 0; e2 < 16; ++e2) {
-          float dsv[2];
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int e = 2 * e2 + h2;
-            const float sv = __uint_as_float(sr[e]);
-            float x, fac = 1.f;
-            if (p.softcap > 0.f) {
-              const float tt = bwd_tanh(sv * p.cap_in, poly);
-              x = fmaf(tt, cc, -nl);
-              fac = fmaf(-tt, tt, 1.f);
-            } else {
-              x = fmaf(sv, c, -nl);
-            }
-            float pe = fast_exp2(x);
-            const int j = k0 + qc * 32 + e;
-            if (!interior && (j < klo || j > khi)) pe = 0.f;
-            dsv[h2] = pe * (__uint_as_float(dr[e]) - dd) * fac;
-          }
-          dk[e2] = pack2<BF16>(dsv[0], dsv[1]);
-        }
-        tmem_st16(t_s + qc * 16, dk);
+        for (int e = 0; e < 64; ++e) am = fmaxf(am, fabsf(__uint_as_float(sr[e])));
+        poly = __all_sync(0xffffffffu, am * p.cap_in <= kTanhPolyMax);
       }
+      uint32_t dk[32];
+#pragma unroll
+      for (int e2 = 0; e2 < 32; ++e2) {
+        float dsv[2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int e = 2 * e2 + h2;
+          const float sv = __uint_as_float(sr[e]);
+          float x, fac = 1.f;
+          if (SOFTCAP) {
+            const float tt = bwd_tanh(sv * p.cap_in, poly);
+            x = fmaf(tt, cc, -nl);
+            fac = fmaf(-tt, tt, 1.f);
+          } else {
+            x = fmaf(sv, c, -nl);
+          }
+          float pe = fast_exp2(x);
+          const int j = kc0 + e;
+          if (!interior && (j < klo || j > khi)) pe = 0.f;
+          dsv[h2] = pe * (__uint_as_float(dr[e]) - dd) * fac;
+        }
+        dk[e2] = pack2<BF16>(dsv[0], dsv[1]);
+      }
+      // dS of tile u into buffer u % 2; the dQ MMA of tile u - 2 that read it is complete (the
+      // commit that signalled S of tile u came after it)
+      const uint32_t ds_col = 384 + (u & 1) * 64 + half * 32;
+      tmem_st16(tmem + lane_base + ds_col, *reinterpret_cast<uint32_t(*)[16]>(&dk[0]));
+      tmem_st16(tmem + lane_base + ds_col + 16, *reinterpret_cast<uint32_t(*)[16]>(&dk[16]));
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.bar_ds));
     }
-    // ---- epilogue: scale * dQ of this query row
+    // ---- epilogue: scale * dQ of this query row, this warp's half of the columns
     bool have = false;
     if (n_kt > 0 && !*abort) {
       have = mbar_wait(smem_u32(&sm.bar_mm), (n_kt - 1) & 1, abort, 1602);
       tc_fence_after();
     }
     have = __all_sync(0xffffffffu, have);
-    const size_t obase = ((size_t)(b * p.Hq + h) * p.Nq + (size_t)i) * D;
+    const size_t obase = ((size_t)(b * p.Hq + h) * p.Nq + (size_t)i) * D + half * (D / 2);
 #pragma unroll
-    for (int cb = 0; cb < D; cb += 32) {
+    for (int cb = 0; cb < D / 2; cb += 32) {
       uint32_t o[32];
       if (have) {
-        tmem_ld32(tmem + lane_base + 256 + cb, o);
+        tmem_ld32(tmem + lane_base + 256 + half * (D / 2) + cb, o);
         tmem_wait_ld();
       } else {
 #pragma unroll
@@ -645,7 +686,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mfa_bwd_dq_kernel(const __grid
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);

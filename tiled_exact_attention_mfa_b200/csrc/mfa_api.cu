@@ -304,14 +304,31 @@ int dispatch_fwd(const FwdCall& c, int D, cudaStream_t st) {
   return bf ? launch_fwd<64, true, VARLEN, SPARSE>(c, st) : launch_fwd<64, false, VARLEN, SPARSE>(c, st);
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool SOFTCAP>
 int launch_bwd(mfa::BwdParams& p, const void* q, const void* k, const void* v, const void* dout,
                int dtype, cudaStream_t st) {
   static bool smem_kv[kMaxDevices] = {}, smem_q[kMaxDevices] = {};
-  auto kdkv = mfa::mfa_bwd_dkv_kernel<D, BF16>;
-  auto kdq = mfa::mfa_bwd_dq_kernel<D, BF16>;
+  auto kdkv = mfa::mfa_bwd_dkv_kernel<D, BF16, SOFTCAP>;
+  auto kdq = mfa::mfa_bwd_dq_kernel<D, BF16, SOFTCAP>;
   if (!ensure_smem(kdkv, mfa::bwd_kv_smem_bytes<D>(), smem_kv)) return MFA_ERR_CUDA;
   if (!ensure_smem(kdq, mfa::bwd_q_smem_bytes<D>(), smem_q)) return MFA_ERR_CUDA;
+  {
+    // the dQ pass redistributes its launch registers with setmaxnreg: refuse a launch whose
+    // register count would not cover the split (the growing warpgroups would wait forever)
+    static bool regs_ok[kMaxDevices] = {};
+    const int dev = current_device();
+    if (dev < 0) return MFA_ERR_CUDA;
+    if (!regs_ok[dev]) {
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, kdq) != cudaSuccess) return MFA_ERR_CUDA;
+      if (fa.numRegs * mfa::kBwdQThreads < 256 * mfa::kBwdQRegsElem + 128 * mfa::kBwdQRegsCtl)
+        return MFA_ERR_CUDA;
+      if (cudaFuncGetAttributes(&fa, kdkv) != cudaSuccess) return MFA_ERR_CUDA;
+      if (fa.numRegs * mfa::kBwdKvThreads < 256 * mfa::kBwdQRegsElem + 128 * mfa::kBwdQRegsCtl)
+        return MFA_ERR_CUDA;
+      regs_ok[dev] = true;
+    }
+  }
   if (!make_map(&p.tm_q, q, dtype, (long long)p.B * p.Hq, p.Nq, D)) return MFA_ERR_CUDA;
   if (!make_map(&p.tm_do, dout, dtype, (long long)p.B * p.Hq, p.Nq, D)) return MFA_ERR_CUDA;
   if (!make_map(&p.tm_k, k, dtype, (long long)p.B * p.Hkv, p.Nk, D)) return MFA_ERR_CUDA;
@@ -324,16 +341,16 @@ int launch_bwd(mfa::BwdParams& p, const void* q, const void* k, const void* v, c
   const long long g1 = (long long)p.n_kt * p.B * p.Hkv;
   const long long g2 = (long long)p.n_qt * p.B * p.Hq;
   if (g1 > 0x7FFFFFFFLL || g2 > 0x7FFFFFFFLL) return MFA_ERR_BAD_SHAPE;
-  kdkv<<<(unsigned)g1, mfa::kBwdThreads, mfa::bwd_kv_smem_bytes<D>(), st>>>(p);
+  kdkv<<<(unsigned)g1, mfa::kBwdKvThreads, mfa::bwd_kv_smem_bytes<D>(), st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
-  kdq<<<(unsigned)g2, mfa::kBwdThreads, mfa::bwd_q_smem_bytes<D>(), st>>>(p);
+  kdq<<<(unsigned)g2, mfa::kBwdQThreads, mfa::bwd_q_smem_bytes<D>(), st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
   mfa_launch_info li = {};
   li.kernel = 4;
   li.grid_x = (int)g1;
   li.grid_y = (int)g2;
   li.grid_z = 1;
-  li.block_threads = mfa::kBwdThreads;
+  li.block_threads = mfa::kBwdKvThreads;
   li.smem_bytes = mfa::bwd_kv_smem_bytes<D>();
   li.tile_m = mfa::kBwdBM;
   li.tile_n = mfa::kBwdBM;
@@ -484,9 +501,12 @@ int mfa_bwd(const void* q, const void* k, const void* v, const void* out, const 
   p.softcap = softcap > 0.f ? softcap : 0.f;
   p.cap_in = softcap > 0.f ? scale / softcap : 0.f;
   const bool bf = dtype == MFA_DTYPE_BF16;
-  if (D == 128)
-    return bf ? launch_bwd<128, true>(p, q, k, v, dout, dtype, st) : launch_bwd<128, false>(p, q, k, v, dout, dtype, st);
-  return bf ? launch_bwd<64, true>(p, q, k, v, dout, dtype, st) : launch_bwd<64, false>(p, q, k, v, dout, dtype, st);
+  const bool cap = p.softcap > 0.f;
+#define MFA_BWD_CAP(DD, BB) \
+  (cap ? launch_bwd<DD, BB, true>(p, q, k, v, dout, dtype, st) : launch_bwd<DD, BB, false>(p, q, k, v, dout, dtype, st))
+  if (D == 128) return bf ? MFA_BWD_CAP(128, true) : MFA_BWD_CAP(128, false);
+  return bf ? MFA_BWD_CAP(64, true) : MFA_BWD_CAP(64, false);
+#undef MFA_BWD_CAP
 }
 
 size_t mfa_decode_workspace_size(int B, int Nq, int Hq, int Hkv, int D, int max_pages_per_seq,

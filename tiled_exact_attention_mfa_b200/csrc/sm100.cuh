@@ -396,5 +396,10 @@ constexpr int kRegsSoftmax = 200;
 constexpr int kRegsControl = 104;
 __device__ __forceinline__ void regs_softmax() { asm volatile("setmaxnreg.inc.sync.aligned.u32 200;"); }
 __device__ __forceinline__ void regs_control() { asm volatile("setmaxnreg.dec.sync.aligned.u32 104;"); }
+// The same for any split: grow / shrink the executing warpgroup to N registers per thread.
+template <int N>
+__device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N>
+__device__ __forceinline__ void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
 
 }  // namespace mfa
