@@ -148,14 +148,14 @@ struct FwdCall {
   const uint8_t* block_mask;  // block-sparse: [B, Hq, ceil(Nq/128), ceil(Nk/128)]
 };
 
-template <int D, bool BF16, bool VARLEN, bool SPARSE>
+template <int D, bool BF16, bool VARLEN, bool SPARSE, bool SOFTCAP>
 int launch_fwd(const FwdCall& c, cudaStream_t st) {
   const int B = c.B, Hq = c.Hq, Hkv = c.Hkv, Nq = c.Nq, Nk = c.Nk, dtype = c.dtype;
   const float scale = c.scale, softcap = c.softcap;
   static bool smem_done[kMaxDevices] = {};
   static bool regs_ok[kMaxDevices] = {};
   constexpr int smem = mfa::fwd_smem_bytes<D, SPARSE>();
-  auto kernel = mfa::mfa_fwd_kernel<D, BF16, VARLEN, SPARSE>;
+  auto kernel = mfa::mfa_fwd_kernel<D, BF16, VARLEN, SPARSE, SOFTCAP>;
   if (!ensure_smem(kernel, smem, smem_done)) return MFA_ERR_CUDA;
   {
     // setmaxnreg redistributes the registers the CTA launched with; refuse to launch if the
@@ -296,12 +296,20 @@ int launch_fill_empty(void* out, float* lse, size_t rows, int D, int dtype, cuda
   return MFA_OK;
 }
 
-template <bool VARLEN, bool SPARSE>
-int dispatch_fwd(const FwdCall& c, int D, cudaStream_t st) {
+template <bool VARLEN, bool SPARSE, bool SOFTCAP>
+int dispatch_fwd_d(const FwdCall& c, int D, cudaStream_t st) {
   const bool bf = c.dtype == MFA_DTYPE_BF16;
   if (D == 128)
-    return bf ? launch_fwd<128, true, VARLEN, SPARSE>(c, st) : launch_fwd<128, false, VARLEN, SPARSE>(c, st);
-  return bf ? launch_fwd<64, true, VARLEN, SPARSE>(c, st) : launch_fwd<64, false, VARLEN, SPARSE>(c, st);
+    return bf ? launch_fwd<128, true, VARLEN, SPARSE, SOFTCAP>(c, st)
+              : launch_fwd<128, false, VARLEN, SPARSE, SOFTCAP>(c, st);
+  return bf ? launch_fwd<64, true, VARLEN, SPARSE, SOFTCAP>(c, st)
+            : launch_fwd<64, false, VARLEN, SPARSE, SOFTCAP>(c, st);
+}
+
+template <bool VARLEN, bool SPARSE>
+int dispatch_fwd(const FwdCall& c, int D, cudaStream_t st) {
+  return c.softcap > 0.f ? dispatch_fwd_d<VARLEN, SPARSE, true>(c, D, st)
+                         : dispatch_fwd_d<VARLEN, SPARSE, false>(c, D, st);
 }
 
 template <int D, bool BF16, bool SOFTCAP>
