@@ -47,7 +47,7 @@ import numpy as np
 
 __all__ = ["visible", "attention", "attention_rows", "attention_varlen", "attention_varlen_rows",
            "attention_blocksparse", "attention_blocksparse_rows", "attention_backward",
-           "paged_gather", "decode", "decode_rows"]
+           "paged_gather", "attention_paged_prefill", "decode", "decode_rows"]
 
 
 def visible(Nq: int, Nk: int, causal: bool, win_l: int = -1, win_r: int = -1) -> np.ndarray:
@@ -313,6 +313,28 @@ def decode(q, k_pages, v_pages, block_table, seq_lens, scale, causal=True, softc
         kb, vb = paged_gather(k_pages, v_pages, block_table, L, b, page_size)
         ob, lb = attention(q[b:b + 1], kb[None], vb[None], scale, causal=causal, softcap=softcap)
         o[b], lse[b] = ob[0], lb[0]
+    return o, lse
+
+
+def attention_paged_prefill(q, k_pages, v_pages, block_table, seq_lens, cu_q, scale, causal=True,
+                            win_l=-1, win_r=-1, softcap=0.0, page_size: int = 16):
+    """Chunked prefill over a paged cache: sequence b has cu_q[b+1] - cu_q[b] packed query rows
+    (rows of q [total_q, Hq, D]) and seq_lens[b] keys gathered through its block_table row; the
+    dense definition applies per sequence, the queries being the last Nq_b positions
+    (bottom-right). Returns (o [total_q, Hq, D], lse [Hq, total_q])."""
+    total_q, Hq, D = np.shape(q)
+    o = np.zeros((total_q, Hq, D))
+    lse = np.full((Hq, total_q), -np.inf)
+    for b in range(len(cu_q) - 1):
+        q0, q1 = int(cu_q[b]), int(cu_q[b + 1])
+        L = int(seq_lens[b])
+        if q1 == q0 or L == 0:
+            continue
+        kb, vb = paged_gather(k_pages, v_pages, block_table, L, b, page_size)
+        qs = np.asarray(q[q0:q1], dtype=np.float64).transpose(1, 0, 2)[None]
+        ob, lb = attention(qs, kb[None], vb[None], scale, causal, win_l, win_r, softcap)
+        o[q0:q1] = ob[0].transpose(1, 0, 2)
+        lse[:, q0:q1] = lb[0]
     return o, lse
 
 

@@ -561,3 +561,43 @@ def test_backward_gqa_is_mha_on_repeated_heads_and_empty_rows_give_zero():
     np.testing.assert_allclose(dv, dv2.reshape(B, Hkv, 2, Nk, D).sum(axis=2), rtol=0, atol=1e-13)
     # Nq > Nk causal: the first Nq - Nk rows see no key, so their dq is zero
     assert np.all(dq[:, :, :Nq - Nk] == 0)
+
+
+# ---------------------------------------------------------------- paged (chunked) prefill
+def test_paged_prefill_equals_varlen_on_contiguous_and_decode_for_short_chunks():
+    """Pages in identity order hold exactly the contiguous K / V, so the paged prefill equals
+    the packed varlen forward; with 1-4 queries per sequence it equals the decode oracle."""
+    Hq, Hkv, D, page = 4, 2, 8, 16
+    lens = np.array([37, 16, 70], dtype=np.int64)
+    nq = np.array([5, 16, 3], dtype=np.int64)
+    npg = -(-lens // page)
+    kc = [rng.standard_normal((int(L), Hkv, D)) for L in lens]
+    vc = [rng.standard_normal((int(L), Hkv, D)) for L in lens]
+    num = int(npg.sum())
+    kp = np.full((num, page, Hkv, D), np.nan)
+    vp = np.full((num, page, Hkv, D), np.nan)
+    table = np.full((3, int(npg.max())), -1, dtype=np.int64)
+    perm = rng.permutation(num)
+    off = 0
+    for b in range(3):
+        for t in range(int(lens[b])):
+            pg = perm[off + t // page]
+            kp[pg, t % page] = kc[b][t]
+            vp[pg, t % page] = vc[b][t]
+        table[b, :npg[b]] = perm[off:off + npg[b]]
+        off += npg[b]
+    cu_q = np.concatenate([[0], np.cumsum(nq)])
+    cu_k = np.concatenate([[0], np.cumsum(lens)])
+    q = rng.standard_normal((int(cu_q[-1]), Hq, D))
+    for causal, wl, wr in ((True, -1, -1), (True, 9, 0), (False, 4, 2)):
+        o, lse = oracle.attention_paged_prefill(q, kp, vp, table, lens, cu_q, 0.3, causal, wl, wr)
+        ov, lv = oracle.attention_varlen(q, np.concatenate(kc), np.concatenate(vc), cu_q, cu_k,
+                                         0.3, causal, wl, wr)
+        np.testing.assert_allclose(o, ov, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse, lv, rtol=0, atol=1e-13)
+    # short chunks: 3 queries of sequence 2 through the decode oracle
+    qd = q[cu_q[2]:cu_q[3]].transpose(1, 0, 2)[None]
+    od, ld = oracle.decode(qd, kp, vp, table[2:3], lens[2:3], 0.3, causal=True)
+    o, lse = oracle.attention_paged_prefill(q, kp, vp, table, lens, cu_q, 0.3, True)
+    np.testing.assert_allclose(o[cu_q[2]:cu_q[3]], od[0].transpose(1, 0, 2), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse[:, cu_q[2]:cu_q[3]], ld[0], rtol=0, atol=1e-13)
