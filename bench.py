@@ -5,7 +5,8 @@ python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mfa|reference] [--wo
 One step = one pass of the hot path over one batch: the prefill forward of the named workload
 (default: causal, B=2, H=8, N=4096, D=128, fp16). The same JSON line also carries the other
 workloads (non-causal, sliding window, GQA + softcap prefill, packed variable-length prefill,
-block-sparse prefill, paged split-KV decode), each timed the same way. Inputs are seeded synthetic tensors resident in HBM; L2 is flushed (a 256 MiB
+block-sparse prefill, chunked prefill over a paged cache, paged split-KV decode, and the backward
+of the two B=2 H=8 N=4096 workloads), each timed the same way. Inputs are seeded synthetic tensors resident in HBM; L2 is flushed (a 256 MiB
 write) before every timed step, outside the timed kernel. Times are CUDA events on the launching
 stream; with N > 1 (torchrun) every rank runs its own copy of the workload (weak scaling) and the
 max over ranks is reported.
@@ -359,6 +360,37 @@ def bench_backward(case, steps, warmup, flush, stream, world):
 BACKWARD_WORKLOADS = ("causal_b2_h8_n4096_d128_fp16", "noncausal_b2_h8_n4096_d128_fp16")
 
 
+def bench_paged(case, steps, warmup, flush, stream, world):
+    import torch
+    import tiled_exact_attention_mfa_b200 as mfa
+    dev = torch.device("cuda")
+    q, kp, vp, table, lens, cq = case.tensors()
+    qt, kt, vt = (upload(x, case.dtype, dev) for x in (q, kp, vp))
+    tt, lt, ct = (torch.from_numpy(x).to(dev) for x in (table, lens, cq))
+    out = torch.empty_like(qt)
+    lse = torch.empty(case.Hq, qt.shape[0], dtype=torch.float32, device=dev)
+    nq = np.diff(cq)
+    max_q = int(nq.max())
+    scale = case.scale_f32()
+
+    def step():
+        mfa.mfa_fwd_paged(qt, kt, vt, tt, lt, ct, max_q, out, lse, scale=scale, causal=case.causal,
+                          window=(case.win_l, case.win_r), softcap=case.softcap, stream=stream)
+
+    with torch.cuda.stream(stream):
+        ms, bracket = time_steps(step, steps, warmup, flush, stream)
+    pairs = sum(visible_pairs(case_like(case), a, b) for a, b in zip(nq, lens))
+    kv_bytes = float(np.sum(lens)) * case.Hkv * case.D * 2 * 2
+    return {"ms": max_over_ranks(statistics.mean(ms), world), "ms_min": min(ms),
+            "bracket_ms": bracket, "flops": 4.0 * case.D * case.Hq * pairs,
+            "bytes": kv_bytes + 2 * 2 * float(cq[-1]) * case.Hq * case.D, "total_q": int(cq[-1])}
+
+
+def case_like(case):
+    """The masking fields of a workload (for visible_pairs with explicit lengths)."""
+    return mi.PrefillCase("x", 1, 1, 1, 0, 0, case.D, case.dtype, case.causal, case.win_l, case.win_r)
+
+
 def bench_decode(case, steps, warmup, flush, stream, world):
     import torch
     import tiled_exact_attention_mfa_b200 as mfa
@@ -421,9 +453,11 @@ def run_gpu(args):
             if name == args.workload:
                 continue
             sk, wu = max(3, min(args.steps, 10)), max(3, args.warmup)
-            if isinstance(case, (mi.VarlenCase, mi.SparseCase)):
+            if isinstance(case, (mi.VarlenCase, mi.SparseCase, mi.PagedPrefillCase)):
                 if isinstance(case, mi.VarlenCase):
                     r = bench_varlen(case, sk, wu, flush, stream, world)
+                elif isinstance(case, mi.PagedPrefillCase):
+                    r = bench_paged(case, sk, wu, flush, stream, world)
                 else:
                     r = bench_sparse(case, sk, wu, flush, stream, world)
                 tf = r["flops"] * world / (r["ms"] * 1e-3) / 1e12
@@ -592,6 +626,8 @@ def run_profile(args):
         r = bench_varlen(case, args.steps, args.warmup, lambda: flush_buf.fill_(1), stream, 1)
     elif isinstance(case, mi.SparseCase):
         r = bench_sparse(case, args.steps, args.warmup, lambda: flush_buf.fill_(1), stream, 1)
+    elif isinstance(case, mi.PagedPrefillCase):
+        r = bench_paged(case, args.steps, args.warmup, lambda: flush_buf.fill_(1), stream, 1)
     else:
         r = bench_prefill(case, args.steps, args.warmup, lambda: flush_buf.fill_(1), stream, False, 1)
     print(json.dumps({"profile": args.profile, "ms": round(r["ms"], 5)}), flush=True)

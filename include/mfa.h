@@ -6,6 +6,7 @@
  *                      native GQA, optional tanh softcap, optional fp32 log-sum-exp output.
  *   mfa_fwd_varlen     the same forward over packed variable-length sequences (cu_seqlens).
  *   mfa_fwd_blocksparse the same forward restricted by a 128 x 128 block mask.
+ *   mfa_fwd_paged      chunked prefill: packed query chunks over a paged KV cache.
  *   mfa_bwd            backward of mfa_fwd (dq, dk, dv from out and lse).
  *   mfa_decode_splitkv two-phase split-KV decode (N_q <= 4) over a paged KV cache.
  *
@@ -147,6 +148,36 @@ int mfa_fwd_blocksparse(const void* q, const void* k, const void* v, void* out, 
                         const uint8_t* block_mask,
                         int B, int Hq, int Hkv, int Nq, int Nk, int D, float scale,
                         int causal, int win_l, int win_r, float softcap, int dtype, void* stream);
+
+/*
+ * mfa_fwd_paged -- chunked prefill over a paged KV cache: packed variable-length query chunks
+ * attend the keys their sequences hold in the page pool ([MFA252] Features "Paged KV" and
+ * "Variable-length"; [MFA261] notes paged causal with heterogeneous seq_lens corrected toward
+ * the per-sequence bottom-right alignment used here).
+ *
+ * Sequence b has Nq_b = cu_seqlens_q[b+1] - cu_seqlens_q[b] query rows (rows of q / out) and
+ * seq_lens[b] keys; key t is slot t % 16 of page block_table[b][t / 16]. The queries are the
+ * last Nq_b positions (a = i + seq_lens[b] - Nq_b), and each sequence is attended exactly as
+ * mfa_fwd attends one batch entry with Nq = Nq_b, Nk = seq_lens[b]. With Nq_b <= 4 this is
+ * mfa_decode_splitkv's definition.
+ *
+ * Arguments
+ *   q, out       [total_q, Hq, D] dtype; lse [Hq, total_q] float32 or NULL       (device)
+ *   k_pages, v_pages [num_pages, 16, Hkv, D] dtype                                (device)
+ *   block_table  int32 [B, max_pages_per_seq]: entries for t < ceil(seq_lens[b] / 16) must lie
+ *                in [0, num_pages); later entries are never read                    (device)
+ *   seq_lens     int32 [B], each in [0, max_pages_per_seq * 16]                   (device)
+ *   cu_seqlens_q int32 [B + 1] as mfa_fwd_varlen; max_seqlen_q >= every Nq_b; page_size 16.
+ * Page slots at or past a sequence's length may hold any bit pattern (NaN included). Entries
+ * that break these rules are reported through mfa_device_status (MFA_ERR_DEVICE_BAD_PAGE or
+ * MFA_ERR_DEVICE_BAD_SEQLENS); the affected pages read as zeros.
+ */
+int mfa_fwd_paged(const void* q, const void* k_pages, const void* v_pages,
+                  const int32_t* block_table, const int32_t* seq_lens, const int32_t* cu_seqlens_q,
+                  void* out, float* lse, int B, int max_seqlen_q, int total_q,
+                  int Hq, int Hkv, int D, int page_size, int max_pages_per_seq, int num_pages,
+                  float scale, int causal, int win_l, int win_r, float softcap, int dtype,
+                  void* stream);
 
 /*
  * mfa_bwd_workspace_size -- bytes of scratch mfa_bwd needs: one fp32 per query row

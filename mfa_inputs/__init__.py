@@ -358,6 +358,56 @@ class SparseCase:
         return q, k, v, self.block_mask()
 
 
+@dataclass
+class PagedPrefillCase:
+    """Chunked prefill over a paged cache: B sequences with seq_lens uniform on [len_lo, len_hi]
+    (or fixed_lens) keys in a page pool laid out, permuted and NaN-poisoned exactly as a
+    DecodeCase with the same seed; each sequence contributes its last Nq_b positions as packed
+    query rows, Nq_b uniform on [1, min(len_b, q_hi)] (stream 5) or fixed_q."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    D: int
+    dtype: int
+    len_lo: int
+    len_hi: int
+    q_hi: int = 256
+    causal: bool = True
+    win_l: int = -1
+    win_r: int = -1
+    softcap: float = 0.0
+    seed: int = 1
+    fixed_lens: list | None = None
+    fixed_q: list | None = None
+    scale: float | None = None
+
+    def scale_f32(self) -> float:
+        s = self.scale if self.scale is not None else 1.0 / np.sqrt(self.D)
+        return float(np.float32(s))
+
+    def _pool(self) -> "DecodeCase":
+        hi = max(self.fixed_lens) if self.fixed_lens is not None else self.len_hi
+        return DecodeCase(self.name, self.B, 1, self.Hq, self.Hkv, self.D, self.dtype, self.len_lo,
+                          max(int(hi), 1), seed=self.seed, fixed_lens=self.fixed_lens)
+
+    def chunk_lens(self, lens) -> np.ndarray:
+        if self.fixed_q is not None:
+            return np.asarray(self.fixed_q, dtype=np.int32)
+        u = uniform_ints(self.seed, STREAM_KEXTRA, self.B, 0, 1 << 20)
+        cap = np.maximum(1, np.minimum(lens.astype(np.int64), self.q_hi))
+        return (1 + u % cap).astype(np.int32)
+
+    def tensors(self):
+        """(q packed bits, k_pages, v_pages, block_table, seq_lens, cu_seqlens_q)."""
+        _, kp, vp, table, lens = self._pool().tensors()
+        nq = self.chunk_lens(lens)
+        cq = np.zeros(self.B + 1, dtype=np.int32)
+        cq[1:] = np.cumsum(nq)
+        q = normal_bits(self.seed, STREAM_Q, (int(cq[-1]), self.Hq, self.D), self.dtype)
+        return q, kp, vp, table, lens, cq
+
+
 def workloads():
     """The named full-size workloads (shapes, flags, seeds and value scales)."""
     return {
@@ -382,6 +432,9 @@ def workloads():
         "sparse_spatial2d_b1_h16_n16384_d128_fp16": SparseCase(
             "sparse_spatial2d_b1_h16_n16384_d128_fp16", 1, 16, 16, 16384, 128, FP16, False,
             pattern="spatial2d", grid=(16, 8), radius=2, seed=1007),
+        "paged_prefill_b8_hq32_hkv8_d128_bf16_ctx4k_32k": PagedPrefillCase(
+            "paged_prefill_b8_hq32_hkv8_d128_bf16_ctx4k_32k", 8, 32, 8, 128, BF16, 4096, 32768,
+            q_hi=2048, seed=1008),
         "decode_b8_hq32_hkv8_d128_bf16_len8k_128k": DecodeCase(
             "decode_b8_hq32_hkv8_d128_bf16_len8k_128k", 8, 1, 32, 8, 128, BF16, 8192, 131072,
             seed=1005),

@@ -40,6 +40,8 @@ lib.mfa_bwd_workspace_size.restype = ctypes.c_size_t
 lib.mfa_bwd_workspace_size.argtypes = [_i, _i, _i]
 lib.mfa_bwd.restype = _i
 lib.mfa_bwd.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _i, _i, _i, _f, _i, _vp, ctypes.c_size_t, _vp]
+lib.mfa_fwd_paged.restype = _i
+lib.mfa_fwd_paged.argtypes = [_vp] * 8 + [_i] * 9 + [_f, _i, _i, _i, _f, _i, _vp]
 lib.mfa_decode_workspace_size.restype = ctypes.c_size_t
 lib.mfa_decode_workspace_size.argtypes = [_i] * 7
 lib.mfa_decode_splitkv.restype = _i
@@ -73,7 +75,7 @@ lib.mfa_debug_tiles_visited.argtypes = [_vp, ctypes.POINTER(ctypes.c_ulonglong)]
 lib.mfa_debug_set_decode_split_pages.restype = _i
 lib.mfa_debug_set_decode_split_pages.argtypes = [_i]
 
-EXPORTED = ("mfa_fwd", "mfa_fwd_varlen", "mfa_fwd_blocksparse", "mfa_bwd_workspace_size", "mfa_bwd",
+EXPORTED = ("mfa_fwd", "mfa_fwd_varlen", "mfa_fwd_blocksparse", "mfa_fwd_paged", "mfa_bwd_workspace_size", "mfa_bwd",
             "mfa_decode_workspace_size", "mfa_decode_splitkv", "mfa_status_string",
             "mfa_last_launch_info", "mfa_device_status", "mfa_debug_set_flags",
             "mfa_debug_tiles_visited", "mfa_debug_set_decode_split_pages",
@@ -330,3 +332,36 @@ def mfa_bwd(q, k, v, out, dout, lse, dq=None, dk=None, dv=None, *, scale=None, c
                      workspace.numel(), _stream(stream))
     _check(rc, "mfa_bwd")
     return dq, dk, dv
+
+
+def mfa_fwd_paged(q, k_pages, v_pages, block_table, seq_lens, cu_seqlens_q, max_seqlen_q,
+                  out=None, lse=None, *, scale=None, causal=True, window=(-1, -1), softcap=0.0,
+                  return_lse=True, stream=None):
+    """Chunked prefill over a paged cache. q [total_q,Hq,D]; pages [num_pages,16,Hkv,D];
+    block_table int32 [B,max_pages]; seq_lens int32 [B]; cu_seqlens_q int32 [B+1] (device).
+    Returns (out [total_q,Hq,D], lse [Hq,total_q] or None)."""
+    torch = _torch()
+    total_q, Hq, D = q.shape
+    num_pages, page, Hkv, _ = k_pages.shape
+    if k_pages.shape != v_pages.shape or k_pages.shape[3] != D:
+        raise ValueError("k_pages and v_pages must be [num_pages, 16, Hkv, D] matching q")
+    for t in (block_table, seq_lens, cu_seqlens_q):
+        if t.dtype != torch.int32:
+            raise TypeError("block_table, seq_lens and cu_seqlens_q must be int32")
+    B = seq_lens.numel()
+    if cu_seqlens_q.numel() != B + 1 or block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("cu_seqlens_q must hold B + 1 offsets and block_table B rows")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    wl, wr = window
+    rc = lib.mfa_fwd_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seq_lens),
+                           _ptr(cu_seqlens_q), _ptr(out), _ptr(lse), B, int(max_seqlen_q), total_q,
+                           Hq, Hkv, D, page, block_table.shape[1], num_pages, float(scale),
+                           int(bool(causal)), int(wl), int(wr), float(softcap), _dtype_code(q),
+                           _stream(stream))
+    _check(rc, "mfa_fwd_paged")
+    return out, lse

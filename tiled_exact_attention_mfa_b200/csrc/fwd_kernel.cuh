@@ -68,6 +68,11 @@ struct FwdParams {
   // block-sparse: uint8 [B, Hq, nqt, nkt], one entry per 128-row x 128-key block (0 = skip)
   const uint8_t* block_mask;
   int nqt, nkt;
+  // paged keys (with packed queries): sequence b's key t is slot t % 16 of page
+  // block_table[b * max_pages + t / 16] of the pools [num_pages, 16, Hkv, D]; seq_lens[b] keys
+  const int* block_table;
+  const int* seq_lens;
+  int max_pages, num_pages;
   int B, Hq, Hkv, Nq, Nk, G;
   int causal, win_l, win_r;
   int n_qblk;       // number of 256-row query blocks per head
@@ -121,9 +126,15 @@ __device__ __forceinline__ void key_range(const FwdParams& p, int Nk, int a0, in
 // of its Q tiles, and a Q tile whose block is off on a visited tile masks it entirely.
 // SOFTCAP: compiled with the softcap transform (p.softcap > 0); without it the softmax carries
 // no softcap code at all.
-template <int D, bool BF16, bool VARLEN, bool SPARSE, bool SOFTCAP>
+// PAGED (with VARLEN queries): K / V tiles are assembled from 16-token pages through the block
+// table (8 TMA boxes per 128-key tile, maps ordered (D, head, pool token)); pages past the
+// sequence are loaded from past the pool's end, which TMA fills with zeros. Value rows at or past
+// the length inside the last page may hold anything, so before P of that tile is released the
+// first softmax warpgroup zeroes them in shared memory (P is 0 there, but 0 x NaN is NaN).
+template <int D, bool BF16, bool VARLEN, bool SPARSE, bool SOFTCAP, bool PAGED>
 __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_constant__ FwdParams p) {
   static_assert(!(VARLEN && SPARSE), "block masks are defined on the dense layout");
+  static_assert(!PAGED || VARLEN, "paged keys come with packed queries");
   extern __shared__ uint8_t smem_raw[];
   FwdSmem<D, SPARSE>& sm = *reinterpret_cast<FwdSmem<D, SPARSE>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -143,9 +154,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
   int rq = 0, rk = 0;        // its first row in the packed q / k (VARLEN)
   if constexpr (VARLEN) {
     rq = p.cu_q[b];
-    rk = p.cu_k[b];
-    const int eq = p.cu_q[b + 1], ek = p.cu_k[b + 1];
-    if (rq < 0 || eq < rq || eq > p.total_q || rk < 0 || ek < rk || ek > p.total_k) {
+    const int eq = p.cu_q[b + 1];
+    int ek;
+    if constexpr (PAGED) {
+      rk = 0;
+      ek = p.seq_lens[b];
+      if (ek < 0 || ek > p.max_pages * 16) {
+        if (threadIdx.x == 0 && qb == 0 && h == 0) record_status(-22, 0x40000000 + b);
+        return;
+      }
+    } else {
+      rk = p.cu_k[b];
+      ek = p.cu_k[b + 1];
+    }
+    if (rq < 0 || eq < rq || eq > p.total_q || rk < 0 || ek < rk || (!PAGED && ek > p.total_k)) {
       if (threadIdx.x == 0 && qb == 0 && h == 0) record_status(-24, b);
       return;  // the whole CTA, before any barrier or TMEM allocation
     }
@@ -262,18 +284,47 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         const int use = u / kFwdStages;
         const int row = (kt_lo + tile_of(u)) * kFwdBN;
         if (use > 0 && !mbar_wait(smem_u32(&sm.bar_k_empty[s]), (use - 1) & 1, abort, 801)) break;
+        // pool token of each of the tile's 8 pages (past the sequence: past the pool, zero-filled)
+        int ptok[PAGED ? 8 : 1];
+        if constexpr (PAGED) {
+#pragma unroll
+          for (int pi = 0; pi < 8; ++pi) {
+            const int lp = row / 16 + pi;
+            int tok = p.num_pages * 16;
+            if (lp * 16 < Nk) {
+              const int pg = p.block_table[(size_t)b * p.max_pages + lp];
+              if (pg >= 0 && pg < p.num_pages) tok = pg * 16;
+              else record_status(-22, b);
+            }
+            ptok[pi] = tok;
+          }
+        }
         const uint32_t bk = smem_u32(&sm.bar_k_full[s]);
         mbar_expect_tx(bk, kTileBytes);
-        for (int sl = 0; sl < kSlabs; ++sl)
-          tma_load_3d(smem_u32(sm.k[s]) + sl * kSlab, &p.tm_k, bk, sl * 64, VARLEN ? g : row,
-                      VARLEN ? rk + row : b * p.Hkv + g);
+        for (int sl = 0; sl < kSlabs; ++sl) {
+          if constexpr (PAGED) {
+#pragma unroll
+            for (int pi = 0; pi < 8; ++pi)
+              tma_load_3d(smem_u32(sm.k[s]) + sl * kSlab + pi * 16 * 128, &p.tm_k, bk, sl * 64, g, ptok[pi]);
+          } else {
+            tma_load_3d(smem_u32(sm.k[s]) + sl * kSlab, &p.tm_k, bk, sl * 64, VARLEN ? g : row,
+                        VARLEN ? rk + row : b * p.Hkv + g);
+          }
+        }
         issued_k[s] = use + 1;
         if (use > 0 && !mbar_wait(smem_u32(&sm.bar_v_empty[s]), (use - 1) & 1, abort, 802)) break;
         const uint32_t bv = smem_u32(&sm.bar_v_full[s]);
         mbar_expect_tx(bv, kTileBytes);
-        for (int sl = 0; sl < kSlabs; ++sl)
-          tma_load_3d(smem_u32(sm.v[s]) + sl * kSlab, &p.tm_v, bv, sl * 64, VARLEN ? g : row,
-                      VARLEN ? rk + row : b * p.Hkv + g);
+        for (int sl = 0; sl < kSlabs; ++sl) {
+          if constexpr (PAGED) {
+#pragma unroll
+            for (int pi = 0; pi < 8; ++pi)
+              tma_load_3d(smem_u32(sm.v[s]) + sl * kSlab + pi * 16 * 128, &p.tm_v, bv, sl * 64, g, ptok[pi]);
+          } else {
+            tma_load_3d(smem_u32(sm.v[s]) + sl * kSlab, &p.tm_v, bv, sl * 64, VARLEN ? g : row,
+                        VARLEN ? rk + row : b * p.Hkv + g);
+          }
+        }
         issued_v[s] = use + 1;
       }
       // Make sure no copy into this CTA's shared memory is still in flight when it exits.
@@ -484,6 +535,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       }
       // P = exp2(s * c - m * c) on fp32 pairs, packed to the input type and stored to TMEM 16
       // columns at a time; each half of P is announced as soon as it is stored.
+      if constexpr (PAGED) {
+        // the final tile: value rows at or past the length (inside the last page) become 0
+        if (t == 0 && k0 + kFwdBN > Nk) {
+          const int vs = j % kFwdStages;
+          const bool vok = mbar_wait(smem_u32(&sm.bar_v_full[vs]), (j / kFwdStages) & 1, abort, 1009);
+          if (!__all_sync(0xffffffffu, vok)) break;
+          if (r >= Nk - k0) {
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int sl = 0; sl < kSlabs; ++sl) {
+              uint4* rowp = reinterpret_cast<uint4*>(sm.v[vs] + sl * kSlab + r * 128);
+#pragma unroll
+              for (int c16 = 0; c16 < 8; ++c16) rowp[c16] = z;
+            }
+          }
+          fence_proxy_async_smem();  // generic stores, then the tensor core reads them after P
+        }
+      }
       const uint64_t c2 = f2_pack(c, c);
       const uint64_t nm2 = f2_pack(neg_mc, neg_mc);
       uint64_t acc[4];

@@ -75,6 +75,22 @@ bool make_map_packed(CUtensorMap* m, const void* base, int dtype, long long tota
   return r == CUDA_SUCCESS;
 }
 
+// Page pools [num_pages, 16, H, D] seen as [num_pages * 16 tokens, H, D], ordered (D, head,
+// token) with a 64 x 1 x 16 box: one box is one page of one head, 16 rows of a 128-byte slab.
+bool make_map_pages(CUtensorMap* m, const void* base, int dtype, long long tokens, int H, int D) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)tokens};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  cuuint32_t box[3] = {64, 1, 16};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dtype == MFA_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Opt a kernel into its dynamic shared memory size once per device.
 template <typename K>
 bool ensure_smem(K kernel, int bytes, bool (&done)[kMaxDevices]) {
@@ -146,16 +162,18 @@ struct FwdCall {
   const int32_t *cu_q, *cu_k;
   int total_q, total_k;
   const uint8_t* block_mask;  // block-sparse: [B, Hq, ceil(Nq/128), ceil(Nk/128)]
+  const int32_t *block_table, *seq_lens;  // paged keys
+  int max_pages, num_pages;
 };
 
-template <int D, bool BF16, bool VARLEN, bool SPARSE, bool SOFTCAP>
+template <int D, bool BF16, bool VARLEN, bool SPARSE, bool SOFTCAP, bool PAGED>
 int launch_fwd(const FwdCall& c, cudaStream_t st) {
   const int B = c.B, Hq = c.Hq, Hkv = c.Hkv, Nq = c.Nq, Nk = c.Nk, dtype = c.dtype;
   const float scale = c.scale, softcap = c.softcap;
   static bool smem_done[kMaxDevices] = {};
   static bool regs_ok[kMaxDevices] = {};
   constexpr int smem = mfa::fwd_smem_bytes<D, SPARSE>();
-  auto kernel = mfa::mfa_fwd_kernel<D, BF16, VARLEN, SPARSE, SOFTCAP>;
+  auto kernel = mfa::mfa_fwd_kernel<D, BF16, VARLEN, SPARSE, SOFTCAP, PAGED>;
   if (!ensure_smem(kernel, smem, smem_done)) return MFA_ERR_CUDA;
   {
     // setmaxnreg redistributes the registers the CTA launched with; refuse to launch if the
@@ -172,7 +190,17 @@ int launch_fwd(const FwdCall& c, cudaStream_t st) {
   }
   mfa::FwdParams p;
   std::memset(&p, 0, sizeof(p));
-  if (VARLEN) {
+  if (PAGED) {
+    if (!make_map_packed(&p.tm_q, c.q, dtype, c.total_q, Hq, D)) return MFA_ERR_CUDA;
+    if (!make_map_pages(&p.tm_k, c.k, dtype, (long long)c.num_pages * 16, Hkv, D)) return MFA_ERR_CUDA;
+    if (!make_map_pages(&p.tm_v, c.v, dtype, (long long)c.num_pages * 16, Hkv, D)) return MFA_ERR_CUDA;
+    p.cu_q = c.cu_q;
+    p.total_q = c.total_q;
+    p.block_table = c.block_table;
+    p.seq_lens = c.seq_lens;
+    p.max_pages = c.max_pages;
+    p.num_pages = c.num_pages;
+  } else if (VARLEN) {
     if (!make_map_packed(&p.tm_q, c.q, dtype, c.total_q, Hq, D)) return MFA_ERR_CUDA;
     if (!make_map_packed(&p.tm_k, c.k, dtype, c.total_k, Hkv, D)) return MFA_ERR_CUDA;
     if (!make_map_packed(&p.tm_v, c.v, dtype, c.total_k, Hkv, D)) return MFA_ERR_CUDA;
@@ -296,20 +324,20 @@ int launch_fill_empty(void* out, float* lse, size_t rows, int D, int dtype, cuda
   return MFA_OK;
 }
 
-template <bool VARLEN, bool SPARSE, bool SOFTCAP>
+template <bool VARLEN, bool SPARSE, bool SOFTCAP, bool PAGED>
 int dispatch_fwd_d(const FwdCall& c, int D, cudaStream_t st) {
   const bool bf = c.dtype == MFA_DTYPE_BF16;
   if (D == 128)
-    return bf ? launch_fwd<128, true, VARLEN, SPARSE, SOFTCAP>(c, st)
-              : launch_fwd<128, false, VARLEN, SPARSE, SOFTCAP>(c, st);
-  return bf ? launch_fwd<64, true, VARLEN, SPARSE, SOFTCAP>(c, st)
-            : launch_fwd<64, false, VARLEN, SPARSE, SOFTCAP>(c, st);
+    return bf ? launch_fwd<128, true, VARLEN, SPARSE, SOFTCAP, PAGED>(c, st)
+              : launch_fwd<128, false, VARLEN, SPARSE, SOFTCAP, PAGED>(c, st);
+  return bf ? launch_fwd<64, true, VARLEN, SPARSE, SOFTCAP, PAGED>(c, st)
+            : launch_fwd<64, false, VARLEN, SPARSE, SOFTCAP, PAGED>(c, st);
 }
 
-template <bool VARLEN, bool SPARSE>
+template <bool VARLEN, bool SPARSE, bool PAGED = false>
 int dispatch_fwd(const FwdCall& c, int D, cudaStream_t st) {
-  return c.softcap > 0.f ? dispatch_fwd_d<VARLEN, SPARSE, true>(c, D, st)
-                         : dispatch_fwd_d<VARLEN, SPARSE, false>(c, D, st);
+  return c.softcap > 0.f ? dispatch_fwd_d<VARLEN, SPARSE, true, PAGED>(c, D, st)
+                         : dispatch_fwd_d<VARLEN, SPARSE, false, PAGED>(c, D, st);
 }
 
 template <int D, bool BF16, bool SOFTCAP>
@@ -386,7 +414,7 @@ int mfa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (Nk == 0) return launch_fill_empty(out, lse, (size_t)B * Hq * Nq, D, dtype, st);
   FwdCall c = {q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, scale, causal, win_l, win_r, softcap, dtype,
-               nullptr, nullptr, 0, 0, nullptr};
+               nullptr, nullptr, 0, 0, nullptr, nullptr, nullptr, 0, 0};
   return dispatch_fwd<false, false>(c, D, st);
 }
 
@@ -408,7 +436,7 @@ int mfa_fwd_blocksparse(const void* q, const void* k, const void* v, void* out, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (Nk == 0) return launch_fill_empty(out, lse, (size_t)B * Hq * Nq, D, dtype, st);
   FwdCall c = {q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, scale, causal, win_l, win_r, softcap, dtype,
-               nullptr, nullptr, 0, 0, block_mask};
+               nullptr, nullptr, 0, 0, block_mask, nullptr, nullptr, 0, 0};
   return dispatch_fwd<false, true>(c, D, st);
 }
 
@@ -433,8 +461,38 @@ int mfa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (total_k == 0) return launch_fill_empty(out, lse, (size_t)total_q * Hq, D, dtype, st);
   FwdCall c = {q, k, v, out, lse, B, Hq, Hkv, max_seqlen_q, 0, scale, causal, win_l, win_r, softcap,
-               dtype, cu_seqlens_q, cu_seqlens_k, total_q, total_k, nullptr};
+               dtype, cu_seqlens_q, cu_seqlens_k, total_q, total_k, nullptr, nullptr, nullptr, 0, 0};
   return dispatch_fwd<true, false>(c, D, st);
+}
+
+int mfa_fwd_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                  const int32_t* seq_lens, const int32_t* cu_seqlens_q, void* out, float* lse, int B,
+                  int max_seqlen_q, int total_q, int Hq, int Hkv, int D, int page_size,
+                  int max_pages_per_seq, int num_pages, float scale, int causal, int win_l, int win_r,
+                  float softcap, int dtype, void* stream) {
+  int rc = validate_fwd_common(Hq, Hkv, D, dtype, win_l, win_r, softcap, scale);
+  if (rc != MFA_OK) return rc;
+  if (page_size != mfa::kDecPage) return MFA_ERR_PAGE_SIZE;
+  if (B < 0 || max_seqlen_q < 0 || total_q < 0 || max_pages_per_seq < 1 || num_pages < 1)
+    return MFA_ERR_BAD_SHAPE;
+  if (max_seqlen_q > total_q) return MFA_ERR_BAD_SHAPE;
+  if ((rc = check_sizes(total_q, Hq, D, 1)) != MFA_OK) return rc;
+  if ((rc = check_sizes(num_pages, page_size, Hkv, D)) != MFA_OK) return rc;
+  if ((long long)max_pages_per_seq * 16 > 0x3fffffffLL || (long long)num_pages * 16 > 0x3fffffffLL)
+    return MFA_ERR_BAD_SHAPE;
+  if ((long long)B * Hq > 0x7FFFFFFFLL) return MFA_ERR_BAD_SHAPE;
+  if (B == 0 || Hq == 0 || total_q == 0 || max_seqlen_q == 0) return MFA_OK;
+  if (!q || !out || !k_pages || !v_pages || !block_table || !seq_lens || !cu_seqlens_q)
+    return MFA_ERR_NULL_POINTER;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(lse) || !aligned16(k_pages) || !aligned16(v_pages) ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u))
+    return MFA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  FwdCall c = {q, k_pages, v_pages, out, lse, B, Hq, Hkv, max_seqlen_q, 0, scale, causal, win_l, win_r,
+               softcap, dtype, cu_seqlens_q, nullptr, total_q, 0, nullptr, block_table, seq_lens,
+               max_pages_per_seq, num_pages};
+  return dispatch_fwd<true, false, true>(c, D, st);
 }
 
 static int validate_decode(int B, int Nq, int Hq, int Hkv, int D, int page_size, int max_pages) {
