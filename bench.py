@@ -99,13 +99,29 @@ def varlen_bytes(case) -> float:
     return 2 * tq * case.Hq * case.D * 2 + 2 * 2 * tk * case.Hkv * case.D + 4 * tq * case.Hq
 
 
+def decode_tokens(case, lens):
+    """(cached tokens some query row sees, visible (row, token) pairs) summed over sequences:
+    row t of a sequence of length L sees tokens [L - Nq + t - win_l, L - Nq + t] (causal) or
+    [L - Nq + t - win_l, L - 1], clipped to [0, L)."""
+    toks = pairs = 0
+    for L in (int(x) for x in lens):
+        lo_all = L
+        for t in range(case.Nq):
+            hi = min(L - case.Nq + t, L - 1) if case.causal else L - 1
+            lo = max(0, L - case.Nq + t - case.win_l) if case.win_l >= 0 else 0
+            pairs += max(0, hi - lo + 1)
+            lo_all = min(lo_all, lo)
+        toks += L - lo_all
+    return toks, pairs
+
+
 def decode_bytes(case, lens) -> float:
-    kv = float(np.sum(lens)) * case.Hkv * case.D * 2 * 2
+    kv = float(decode_tokens(case, lens)[0]) * case.Hkv * case.D * 2 * 2
     return kv + case.B * case.Hq * case.Nq * case.D * 2 * 2 + 4 * case.B * case.Hq * case.Nq
 
 
 def decode_flops(case, lens) -> float:
-    return 4.0 * case.D * case.Hq * case.Nq * float(np.sum(lens))
+    return 4.0 * case.D * case.Hq * float(decode_tokens(case, lens)[1])
 
 
 def peaks():
@@ -407,13 +423,15 @@ def bench_decode(case, steps, warmup, flush, stream, world):
 
     def step():
         mfa.mfa_decode_splitkv(qt, kt, vt, tt, lt, out, lse, scale=scale, causal=case.causal,
-                               softcap=case.softcap, workspace=ws, stream=stream)
+                               softcap=case.softcap, workspace=ws, win_l=case.win_l,
+                               stream=stream)
 
     with torch.cuda.stream(stream):
         ms, bracket = time_steps(step, steps, warmup, flush, stream)
     return {"ms": max_over_ranks(statistics.mean(ms), world), "ms_min": min(ms),
             "bracket_ms": bracket, "bytes": decode_bytes(case, lens),
-            "flops": decode_flops(case, lens), "seq_len_sum": int(np.sum(lens))}
+            "flops": decode_flops(case, lens), "seq_len_sum": int(np.sum(lens)),
+            "visible_tokens": int(decode_tokens(case, lens)[0])}
 
 
 def run_gpu(args):
@@ -478,6 +496,9 @@ def run_gpu(args):
                                "frac_of_measured_peak": round(tb / pk["gbs"], 4),
                                "frac_of_nominal_peak": round(tb / NOMINAL_GBS, 4),
                                "seq_len_sum": r["seq_len_sum"],
+                               **({"window_left": case.win_l,
+                                   "visible_tokens": r["visible_tokens"]}
+                                  if case.win_l >= 0 else {}),
                                "traffic_phase1": ncu_traffic(name, "mfa_decode_phase1_kernel"),
                                "tflops": round(r["flops"] * world / (r["ms"] * 1e-3) / 1e12, 2)})
             else:

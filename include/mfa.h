@@ -8,7 +8,8 @@
  *   mfa_fwd_blocksparse the same forward restricted by a 128 x 128 block mask.
  *   mfa_fwd_paged      chunked prefill: packed query chunks over a paged KV cache.
  *   mfa_bwd            backward of mfa_fwd (dq, dk, dv from out and lse).
- *   mfa_decode_splitkv two-phase split-KV decode (N_q <= 4) over a paged KV cache.
+ *   mfa_decode_splitkv two-phase split-KV decode (N_q <= 4) over a paged KV cache
+ *                      (mfa_decode_splitkv_window: with a left window).
  *
  * Sources (web pages, cited by title and section):
  *   [MLXBUN]  "mlx-bun 0.4.0 -> 1.0.0, src/model/flash-attention.ts" (diffend): forward shader
@@ -251,6 +252,24 @@ int mfa_decode_splitkv(const void* q, const void* k_pages, const void* v_pages,
                        int max_pages_per_seq, int num_pages,
                        float scale, int causal, float softcap, int dtype,
                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * mfa_decode_splitkv_window -- mfa_decode_splitkv with a left window ([MFA252] Features:
+ * window_size=(left, right) for local-attention layers, here in decode): query token t (at
+ * position a = seq_lens[b] - Nq + t) sees keys j with a - win_l <= j (and j <= a when causal);
+ * win_l = -1 is mfa_decode_splitkv. Splits are counted from the first page that some query
+ * token can see, so pages wholly left of every window are never read, and the split size is
+ * chosen from the window's page span rather than max_pages_per_seq. Arguments as
+ * mfa_decode_splitkv plus win_l >= -1 (MFA_ERR_BAD_WINDOW otherwise); the workspace that
+ * mfa_decode_workspace_size reports (which has no window argument) is always sufficient.
+ */
+int mfa_decode_splitkv_window(const void* q, const void* k_pages, const void* v_pages,
+                              const int32_t* block_table, const int32_t* seq_lens,
+                              void* out, float* lse,
+                              int B, int Nq, int Hq, int Hkv, int D, int page_size,
+                              int max_pages_per_seq, int num_pages,
+                              float scale, int causal, int win_l, float softcap, int dtype,
+                              void* workspace, size_t workspace_bytes, void* stream);
 
 /* Human-readable text for a status code (static storage). */
 const char* mfa_status_string(int code);

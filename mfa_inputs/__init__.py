@@ -174,6 +174,7 @@ class DecodeCase:
     scale: float | None = None
     extra_pages: int = 0
     permute: bool = True
+    win_l: int = -1
     _cache: dict = field(default_factory=dict, repr=False)
 
     def scale_f32(self) -> float:
@@ -438,4 +439,8 @@ def workloads():
         "decode_b8_hq32_hkv8_d128_bf16_len8k_128k": DecodeCase(
             "decode_b8_hq32_hkv8_d128_bf16_len8k_128k", 8, 1, 32, 8, 128, BF16, 8192, 131072,
             seed=1005),
+        # the same cache lengths under a 4096-token left window (each query sees 4096 keys)
+        "decode_window4k_b8_hq32_hkv8_d128_bf16_len8k_128k": DecodeCase(
+            "decode_window4k_b8_hq32_hkv8_d128_bf16_len8k_128k", 8, 1, 32, 8, 128, BF16, 8192,
+            131072, win_l=4095, seed=1005),
     }

@@ -297,11 +297,12 @@ def paged_gather(k_pages, v_pages, block_table, seq_len: int, b: int, page_size:
 
 
 def decode(q, k_pages, v_pages, block_table, seq_lens, scale, causal=True, softcap=0.0,
-           page_size: int = 16):
+           page_size: int = 16, win_l: int = -1):
     """Decode over a paged cache: each sequence is gathered, then the dense definition applies
     with Nk = len_b (query t of Nq sits at position len_b - Nq + t). Split-KV is a schedule of the
     same sum (mlx-mfa 2.5.2 Features, "Flash Decode -- two-phase split-KV"), so the oracle does
-    not split. q [B,Hq,Nq,D]. Returns (o [B,Hq,Nq,D], lse [B,Hq,Nq])."""
+    not split. win_l >= 0 adds a left window (key j visible from a iff j >= a - win_l).
+    q [B,Hq,Nq,D]. Returns (o [B,Hq,Nq,D], lse [B,Hq,Nq])."""
     q = np.asarray(q, dtype=np.float64)
     B, Hq, Nq, D = q.shape
     o = np.zeros((B, Hq, Nq, D))
@@ -311,7 +312,8 @@ def decode(q, k_pages, v_pages, block_table, seq_lens, scale, causal=True, softc
         if L == 0:
             continue
         kb, vb = paged_gather(k_pages, v_pages, block_table, L, b, page_size)
-        ob, lb = attention(q[b:b + 1], kb[None], vb[None], scale, causal=causal, softcap=softcap)
+        ob, lb = attention(q[b:b + 1], kb[None], vb[None], scale, causal=causal, win_l=win_l,
+                           softcap=softcap)
         o[b], lse[b] = ob[0], lb[0]
     return o, lse
 
@@ -339,8 +341,9 @@ def attention_paged_prefill(q, k_pages, v_pages, block_table, seq_lens, cu_q, sc
 
 
 def decode_rows(q, k_pages, v_pages, block_table, seq_lens, rows, scale, causal=True,
-                softcap=0.0, page_size: int = 16, to_f64=None):
-    """Decode outputs for selected rows only, gathering just the kv head each row needs.
+                softcap=0.0, page_size: int = 16, to_f64=None, win_l: int = -1):
+    """Decode outputs for selected rows only, gathering just the kv head each row needs
+    (win_l >= 0: the left window of decode()).
 
     rows: int array [n, 3] of (b, h, t). to_f64 converts a gathered slice of the pools to fp64
     (default: numpy conversion). Returns (o [n, D], lse [n])."""
@@ -365,6 +368,8 @@ def decode_rows(q, k_pages, v_pages, block_table, seq_lens, rows, scale, causal=
         vis = np.ones(L, dtype=bool)
         if causal:
             vis &= tok <= a
+        if win_l >= 0:
+            vis &= tok >= a - win_l
         qi = conv(np.asarray(q)[b, h, t:t + 1])
         oi, li = _rows_for_head(qi, kb, vb, vis[None, :], scale, softcap)
         o[n], lse[n] = oi[0], li[0]

@@ -22,6 +22,15 @@ SMALL = [
     Dc("noncausal_nq2_bf16", 2, 2, 8, 2, 128, mi.BF16, 1, 500, causal=False, seed=58),
     Dc("softcap30_bf16", 2, 1, 16, 4, 128, mi.BF16, 100, 900, softcap=30.0, seed=59),
     Dc("more_than_8_kv_heads_fp16", 2, 1, 32, 16, 64, mi.FP16, 50, 400, seed=60),
+    # left sliding window: spans that begin mid-page and several splits into the sequence
+    Dc("window100_nq1_gqa4_bf16", 4, 1, 32, 8, 128, mi.BF16, 1, 2000, win_l=100, seed=65),
+    Dc("window30_nq4_fp16", 3, 4, 16, 4, 64, mi.FP16, 40, 900, win_l=30, seed=66),
+    Dc("window0_nq3_bf16", 2, 3, 8, 2, 128, mi.BF16, 5, 300, win_l=0, seed=67),
+    Dc("window_longer_than_seq_fp16", 3, 2, 8, 4, 128, mi.FP16, 1, 700, win_l=5000, seed=68),
+    Dc("window_noncausal_softcap_bf16", 2, 2, 16, 4, 128, mi.BF16, 200, 1500, causal=False,
+       softcap=30.0, win_l=250, seed=69),
+    Dc("window_edge_lengths_fp16", 6, 1, 8, 2, 64, mi.FP16, 0, 0,
+       fixed_lens=[1, 16, 17, 0, 33, 513], max_pages=40, win_l=16, seed=70),
 ]
 
 
@@ -33,7 +42,7 @@ def run_gpu(case, q, k, v, table, lens, split_pages=0):
         out, lse = mfa.mfa_decode_splitkv(
             to_torch(q, case.dtype), to_torch(k, case.dtype), to_torch(v, case.dtype),
             torch.from_numpy(table).cuda(), torch.from_numpy(lens).cuda(),
-            scale=case.scale_f32(), causal=case.causal, softcap=case.softcap)
+            scale=case.scale_f32(), causal=case.causal, softcap=case.softcap, win_l=case.win_l)
     finally:
         mfa.mfa_debug_set_decode_split_pages(old)
     torch.cuda.synchronize()
@@ -42,7 +51,8 @@ def run_gpu(case, q, k, v, table, lens, split_pages=0):
 
 def oracle_full(case, q, k, v, table, lens):
     w = lambda x: mi.widen(x, case.dtype)
-    return oracle.decode(w(q), w(k), w(v), table, lens, case.scale_f32(), case.causal, case.softcap)
+    return oracle.decode(w(q), w(k), w(v), table, lens, case.scale_f32(), case.causal, case.softcap,
+                         win_l=case.win_l)
 
 
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: c.name)
@@ -55,15 +65,18 @@ def test_small_cases_match_oracle(cuda_device, case):
     assert mfa.mfa_device_status() == (0, 0)
 
 
-def test_full_size_sampled_rows(cuda_device):
-    case = mi.workloads()["decode_b8_hq32_hkv8_d128_bf16_len8k_128k"]
+@pytest.mark.parametrize("name", ["decode_b8_hq32_hkv8_d128_bf16_len8k_128k",
+                                  "decode_window4k_b8_hq32_hkv8_d128_bf16_len8k_128k"])
+def test_full_size_sampled_rows(cuda_device, name):
+    case = mi.workloads()[name]
     q, k, v, table, lens = case.tensors()
     o, lse = run_gpu(case, q, k, v, table, lens)
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
     rng = np.random.default_rng(5)
     rows = np.array([(b, h, 0) for b in range(case.B) for h in sorted(rng.choice(32, 5, replace=False))])
     o_ref, l_ref = oracle.decode_rows(q, k, v, table, lens, rows, case.scale_f32(), case.causal,
-                                      case.softcap, to_f64=lambda a: mi.widen(a, case.dtype))
+                                      case.softcap, to_f64=lambda a: mi.widen(a, case.dtype),
+                                      win_l=case.win_l)
     sel = (rows[:, 0], rows[:, 1], rows[:, 2])
     check_close(o[sel], lse[sel], o_ref, l_ref, case.dtype, case.name)
     import tiled_exact_attention_mfa_b200 as mfa
@@ -135,4 +148,44 @@ def test_out_of_range_entries_are_reported_not_read(cuda_device):
     run_gpu(case, q, k, v, table, lens2)
     code, _ = mfa.mfa_device_status()
     assert code == -22
+    assert mfa.mfa_device_status() == (0, 0)
+
+
+def test_window_split_size_changes_only_rounding(cuda_device):
+    """The splits left of the window are skipped whole; the result does not depend on where the
+    split boundaries fall relative to the window's first token."""
+    case = Dc("wsplit", 2, 2, 32, 8, 128, mi.BF16, 3000, 5000, win_l=700, seed=71)
+    q, k, v, table, lens = case.tensors()
+    ref = oracle_full(case, q, k, v, table, lens)
+    for s in (1, 3, 8, 32):
+        o, lse = run_gpu(case, q, k, v, table, lens, split_pages=s)
+        check_close(o, lse, *ref, case.dtype, f"wsplit{s}")
+
+
+def test_window_minus_one_is_the_plain_decode(cuda_device):
+    """win_l = -1 through the window entry point is bitwise the plain decode; a window covering
+    the whole sequence differs from it only by rounding."""
+    import torch
+    import tiled_exact_attention_mfa_b200 as mfa
+    case = SMALL[0]
+    q, k, v, table, lens = case.tensors()
+    args = (to_torch(q, case.dtype), to_torch(k, case.dtype), to_torch(v, case.dtype),
+            torch.from_numpy(table).cuda(), torch.from_numpy(lens).cuda())
+    o1, l1 = mfa.mfa_decode_splitkv(*args, scale=case.scale_f32())
+    ws = torch.empty(mfa.mfa_decode_workspace_size(q.shape[0], q.shape[2], q.shape[1], k.shape[2], case.D,
+                                              table.shape[1]),
+                     dtype=torch.uint8, device="cuda")
+    o2 = torch.empty_like(o1)
+    l2 = torch.empty_like(l1)
+    rc = mfa.lib.mfa_decode_splitkv_window(
+        mfa._ptr(args[0]), mfa._ptr(args[1]), mfa._ptr(args[2]), mfa._ptr(args[3]),
+        mfa._ptr(args[4]), mfa._ptr(o2), mfa._ptr(l2), q.shape[0], q.shape[2], q.shape[1],
+        k.shape[2], case.D, 16, table.shape[1], k.shape[0], case.scale_f32(), 1, -1, 0.0,
+        mfa._dtype_code(args[0]), mfa._ptr(ws), ws.numel(), mfa._stream(None))
+    assert rc == 0
+    o3, l3 = mfa.mfa_decode_splitkv(*args, scale=case.scale_f32(), win_l=100000)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    assert float((o1.float() - o3.float()).abs().max()) <= 1.6e-2
+    assert float((l1 - l3).abs().max()) <= 1e-4
     assert mfa.mfa_device_status() == (0, 0)

@@ -283,6 +283,47 @@ def test_decode_gather_matches_sdpa_on_contiguous_cache(Nq):
     assert np.all(np.isfinite(o))
 
 
+@pytest.mark.parametrize("Nq", [1, 2, 4])
+def test_decode_window_matches_sdpa_band(Nq):
+    """A left window on the paged decode keeps, for query row t, the keys within win_l of its
+    bottom-right position L - Nq + t: the gathered-cache SDPA under the band mask."""
+    B, Hq, Hkv, D, win = 3, 4, 2, 8, 20
+    lens = [37, 16, 70]
+    kc = rng.standard_normal((B, Hkv, 70, D))
+    vc = rng.standard_normal((B, Hkv, 70, D))
+    q = rng.standard_normal((B, Hq, Nq, D))
+    kp, vp, table = _paged_from_contiguous(kc, vc, lens)
+    o, lse = oracle.decode(q, kp, vp, table, lens, 0.3, causal=True, win_l=win)
+    for b in range(B):
+        L = lens[b]
+        mask = band_mask_torch(Nq, L, True, win, -1)
+        ref = sdpa_ref(q[b:b + 1], kc[b:b + 1, :, :L], vc[b:b + 1, :, :L], 0.3, mask)
+        np.testing.assert_allclose(o[b], ref[0], rtol=0, atol=1e-12)
+
+
+def test_decode_window_equals_decode_of_the_cache_tail():
+    """One query with a left window of w sees exactly the last w + 1 cached tokens, so it equals
+    the unwindowed decode of a cache holding only those tokens; a window at least as long as the
+    sequence changes nothing."""
+    B, Hq, Hkv, D, w = 2, 4, 1, 8, 25
+    lens = [90, 26]
+    kc = rng.standard_normal((B, Hkv, 90, D))
+    vc = rng.standard_normal((B, Hkv, 90, D))
+    q = rng.standard_normal((B, Hq, 1, D))
+    o, lse = oracle.decode(q, *_paged_from_contiguous(kc, vc, lens), lens, 0.3, win_l=w)
+    for b in range(B):
+        L = lens[b]
+        kt = kc[b:b + 1, :, L - w - 1:L].copy()
+        vt = vc[b:b + 1, :, L - w - 1:L].copy()
+        o2, l2 = oracle.decode(q[b:b + 1], *_paged_from_contiguous(kt, vt, [w + 1]), [w + 1], 0.3)
+        np.testing.assert_allclose(o[b], o2[0], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[b], l2[0], rtol=0, atol=1e-12)
+    paged = _paged_from_contiguous(kc, vc, lens)
+    a = oracle.decode(q, *paged, lens, 0.3, win_l=90)
+    c = oracle.decode(q, *paged, lens, 0.3)
+    np.testing.assert_allclose(a[0], c[0], rtol=0, atol=1e-14)
+
+
 def test_decode_page_permutation_and_empty_sequence():
     B, Hq, Hkv, D = 2, 4, 2, 8
     lens = [50, 0]
@@ -306,6 +347,11 @@ def test_decode_rows_helper_matches_pinned_decode():
     o, lse = oracle.decode(q, kp, vp, table, lens, 0.3, causal=True, softcap=4.0)
     rows = np.array([[0, 0, 0], [1, 7, 1], [2, 3, 0], [2, 4, 1]])
     o2, l2 = oracle.decode_rows(q, kp, vp, table, lens, rows, 0.3, True, 4.0)
+    for n, (b, h, t) in enumerate(rows):
+        np.testing.assert_allclose(o2[n], o[b, h, t], rtol=0, atol=1e-14)
+        assert l2[n] == pytest.approx(lse[b, h, t], abs=1e-14)
+    o, lse = oracle.decode(q, kp, vp, table, lens, 0.3, causal=False, win_l=9)
+    o2, l2 = oracle.decode_rows(q, kp, vp, table, lens, rows, 0.3, False, win_l=9)
     for n, (b, h, t) in enumerate(rows):
         np.testing.assert_allclose(o2[n], o[b, h, t], rtol=0, atol=1e-14)
         assert l2[n] == pytest.approx(lse[b, h, t], abs=1e-14)

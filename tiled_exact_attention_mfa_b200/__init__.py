@@ -47,6 +47,9 @@ lib.mfa_decode_workspace_size.argtypes = [_i] * 7
 lib.mfa_decode_splitkv.restype = _i
 lib.mfa_decode_splitkv.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
                                    _f, _i, _f, _i, _vp, ctypes.c_size_t, _vp]
+lib.mfa_decode_splitkv_window.restype = _i
+lib.mfa_decode_splitkv_window.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                          _i, _i, _f, _i, _i, _f, _i, _vp, ctypes.c_size_t, _vp]
 lib.mfa_decode_splitkv_noalloc.restype = _i
 lib.mfa_decode_splitkv_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                            _i, _i, _f, _i, _f, _i, _vp]
@@ -76,7 +79,7 @@ lib.mfa_debug_set_decode_split_pages.restype = _i
 lib.mfa_debug_set_decode_split_pages.argtypes = [_i]
 
 EXPORTED = ("mfa_fwd", "mfa_fwd_varlen", "mfa_fwd_blocksparse", "mfa_fwd_paged", "mfa_bwd_workspace_size", "mfa_bwd",
-            "mfa_decode_workspace_size", "mfa_decode_splitkv", "mfa_status_string",
+            "mfa_decode_workspace_size", "mfa_decode_splitkv_window", "mfa_decode_splitkv", "mfa_status_string",
             "mfa_last_launch_info", "mfa_device_status", "mfa_debug_set_flags",
             "mfa_debug_tiles_visited", "mfa_debug_set_decode_split_pages",
             "mfa_decode_splitkv_noalloc")
@@ -157,9 +160,10 @@ def mfa_decode_workspace_size(B, Nq, Hq, Hkv, D, max_pages_per_seq, page_size=16
 
 def mfa_decode_splitkv(q, k_pages, v_pages, block_table, seq_lens, out=None, lse=None, *,
                        scale=None, causal=True, softcap=0.0, workspace=None, return_lse=True,
-                       stream=None):
+                       win_l=-1, stream=None):
     """Paged split-KV decode. q [B,Hq,Nq,D]; pages [num_pages,16,Hkv,D]; block_table int32
-    [B,max_pages]; seq_lens int32 [B]. Returns (out, lse or None)."""
+    [B,max_pages]; seq_lens int32 [B]. win_l >= 0 adds a left window
+    (mfa_decode_splitkv_window). Returns (out, lse or None)."""
     torch = _torch()
     B, Hq, Nq, D = q.shape
     num_pages, page, Hkv, _ = k_pages.shape
@@ -175,12 +179,22 @@ def mfa_decode_splitkv(q, k_pages, v_pages, block_table, seq_lens, out=None, lse
     need = mfa_decode_workspace_size(B, Nq, Hq, Hkv, D, max_pages, page)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
-    rc = lib.mfa_decode_splitkv(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
-                                _ptr(seq_lens), _ptr(out), _ptr(lse), B, Nq, Hq, Hkv, D, page,
-                                max_pages, num_pages, float(scale), int(bool(causal)),
-                                float(softcap), _dtype_code(q), _ptr(workspace),
-                                workspace.numel() * workspace.element_size(), _stream(stream))
-    _check(rc, "mfa_decode_splitkv")
+    if win_l == -1:
+        rc = lib.mfa_decode_splitkv(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
+                                    _ptr(seq_lens), _ptr(out), _ptr(lse), B, Nq, Hq, Hkv, D, page,
+                                    max_pages, num_pages, float(scale), int(bool(causal)),
+                                    float(softcap), _dtype_code(q), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream))
+        _check(rc, "mfa_decode_splitkv")
+    else:
+        rc = lib.mfa_decode_splitkv_window(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
+                                           _ptr(seq_lens), _ptr(out), _ptr(lse), B, Nq, Hq, Hkv, D,
+                                           page, max_pages, num_pages, float(scale),
+                                           int(bool(causal)), int(win_l), float(softcap),
+                                           _dtype_code(q), _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(),
+                                           _stream(stream))
+        _check(rc, "mfa_decode_splitkv_window")
     return out, lse
 
 

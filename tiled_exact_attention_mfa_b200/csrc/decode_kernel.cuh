@@ -17,6 +17,9 @@
 //     accumulates O += P V with mma.sync. Value rows of tokens past the length are zeroed in
 //     registers, so NaN in unused page slots never reaches the arithmetic.
 //   * it writes unnormalised O, the running max (log2 domain) and the running sum per row.
+//   * with a left window (local-attention layers, "mlx-mfa 2.5.2" Features, window_size) the
+//     splits of a sequence start at the first page some query token can see, and tokens left of
+//     a row's window are masked like those past its causal limit.
 // Phase 2 (combine): per (sequence, query head, query token): M = max_s m_s,
 //   O = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s, LSE = ln 2 * (M + log2 sum_s 2^(m_s-M) l_s).
 #pragma once
@@ -40,6 +43,7 @@ struct DecodeParams {
   int B, Nq, Hq, Hkv, G, max_pages, num_pages;
   int pages_per_split, max_splits, heads_per_cta;
   int causal;
+  int win_l;      // left window (query at position a sees keys >= a - win_l); -1: none
   float c_log2;   // scale * log2 e (no softcap) or log2 e (softcap)
   float softcap, cap_in;
 };
@@ -53,6 +57,14 @@ __device__ __forceinline__ int checked_len(const DecodeParams& p, int b, bool re
     return len < 0 ? 0 : cap;
   }
   return len;
+}
+
+// First page holding a key that some query token of the sequence can see: with a left window,
+// tokens before len - Nq - win_l are invisible to every query token. Splits are counted from this
+// page, so pages wholly left of the window are neither read nor given a split.
+__device__ __forceinline__ int dec_first_page(const DecodeParams& p, int len) {
+  if (p.win_l < 0) return 0;
+  return max(0, len - p.Nq - p.win_l) / kDecPage;
 }
 
 template <int D>
@@ -75,6 +87,9 @@ __global__ void __launch_bounds__(9 * 32) mfa_decode_phase1_kernel(const __grid_
   uint64_t* bar_empty = bar_full + kDecStages;
   int* abort_flag = reinterpret_cast<int*>(bar_empty + kDecStages);
 
+  // every CTA of this grid is resident (or done) once all have passed here, so the combine grid
+  // may be launched now; it waits for this grid's completion before reading the workspace
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int split = blockIdx.x;
   const int b = blockIdx.y;
   const int h0 = blockIdx.z * hg;  // first kv head of this CTA
@@ -83,7 +98,7 @@ __global__ void __launch_bounds__(9 * 32) mfa_decode_phase1_kernel(const __grid_
 
   const int len = checked_len(p, b, split == 0 && blockIdx.z == 0 && threadIdx.x == 0);
   const int n_pages = (len + kDecPage - 1) / kDecPage;
-  const int pg0 = split * p.pages_per_split;
+  const int pg0 = dec_first_page(p, len) + split * p.pages_per_split;
   if (pg0 >= n_pages) return;  // nothing of this sequence falls in this split
   const int pg1 = min(n_pages, pg0 + p.pages_per_split);
   const int np = pg1 - pg0;
@@ -163,14 +178,15 @@ __global__ void __launch_bounds__(9 * 32) mfa_decode_phase1_kernel(const __grid_
       qa[kk][3] = qval(qr + 8, kk * 16 + 8 + qc);
     }
   }
-  // query position of each of this thread's two rows (causal limit), and row validity
-  int lim[2];
+  // visible tokens [low, lim] of this thread's two rows: causal limit, left window, length
+  int lim[2], low[2];
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     const int r = qr + 8 * e;
     const int t = (r < R) ? (r % p.Nq) : 0;
     lim[e] = p.causal ? (len - p.Nq + t) : (len - 1);
     lim[e] = min(lim[e], len - 1);
+    low[e] = (p.win_l >= 0) ? (len - p.Nq + t - p.win_l) : 0;
   }
 
   float o[D / 8][4];
@@ -217,7 +233,7 @@ __global__ void __launch_bounds__(9 * 32) mfa_decode_phase1_kernel(const __grid_
         const int ri = e >> 1;
         float x = sc[n][e];
         if (p.softcap > 0.f) x = p.softcap * tanh_from_exp(x * p.cap_in);
-        x = (tok <= lim[ri]) ? x : -INFINITY;
+        x = (tok <= lim[ri] && tok >= low[ri]) ? x : -INFINITY;
         sc[n][e] = x;
         mx[ri] = fmaxf(mx[ri], x);
       }
@@ -300,88 +316,85 @@ __global__ void __launch_bounds__(9 * 32) mfa_decode_phase1_kernel(const __grid_
   }
 }
 
-// Threads per combine CTA: kCombineGroups groups of D threads; group q takes splits q, q + G, ...
+// Threads per combine CTA: G = kCombineThreads / D groups of D threads (one per output column);
+// group g takes splits g, g + G, g + 2G, ...
 constexpr int kCombineThreads = 512;
+// Splits a thread loads before folding them into its running statistics: all their loads are
+// issued together, so a sequence of n splits costs about n / (G * kCombineBatch) memory round trips.
+constexpr int kCombineBatch = 8;
 
-// Block-wide reductions over kCombineThreads threads.
-__device__ __forceinline__ float block_max(float v, float* red) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float r = red[0];
-#pragma unroll
-  for (int w = 1; w < kCombineThreads / 32; ++w) r = fmaxf(r, red[w]);
-  __syncthreads();
-  return r;
-}
-__device__ __forceinline__ float block_sum(float v, float* red) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  float r = red[0];
-#pragma unroll
-  for (int w = 1; w < kCombineThreads / 32; ++w) r += red[w];
-  __syncthreads();
-  return r;
-}
-
-// One CTA per (query row, sequence). The split statistics are read cooperatively; each of the
-// kCombineThreads / D groups of threads sums the weighted partial outputs of every G-th split
-// (one thread per column, two splits in flight per thread), and the groups are added in shared
-// memory.
+// One CTA per (query row, sequence). Every group merges its own splits with the usual softmax
+// rescale, a batch of loads at a time, into (m_g, l_g, acc_g), all in log2 units; the G group
+// partials are merged in shared memory. A split with m = -inf (no visible key) weighs zero.
+// Launched as a programmatic dependent of phase 1: griddepcontrol.wait holds every thread until
+// phase 1 has completed and its workspace writes are visible (a no-op on a plain launch).
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kCombineThreads) mfa_decode_combine_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int G = kCombineThreads / D;
-  __shared__ float red[kCombineThreads / 32];
   __shared__ float part[G][D];
+  __shared__ float part_m[G], part_l[G];
   const int row = blockIdx.x;  // h * Nq + t
   const int b = blockIdx.y;
   const int d = threadIdx.x % D;
   const int grp = threadIdx.x / D;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int len = checked_len(p, b, false);
   const int n_pages = (len + kDecPage - 1) / kDecPage;
-  const int n_splits = (n_pages + p.pages_per_split - 1) / p.pages_per_split;
+  const int n_splits = (n_pages - dec_first_page(p, len) + p.pages_per_split - 1) / p.pages_per_split;
   const size_t rows_all = (size_t)p.Hq * p.Nq;
   const size_t slot0 = (size_t)b * p.max_splits * rows_all + row;  // slot of split s: slot0 + s * rows_all
   const float2* ml = reinterpret_cast<const float2*>(p.ws_ml);
+  const float* o = p.ws_o + slot0 * D + d;
+  const size_t stride = rows_all * D;
 
-  float m_loc = -INFINITY;
-  for (int s = threadIdx.x; s < n_splits; s += kCombineThreads) m_loc = fmaxf(m_loc, ml[slot0 + (size_t)s * rows_all].x);
-  const float M = block_max(m_loc, red);
-  float l_loc = 0.f;
-  if (M > -INFINITY)
-    for (int s = threadIdx.x; s < n_splits; s += kCombineThreads) {
-      const float2 v = ml[slot0 + (size_t)s * rows_all];
-      l_loc += (v.x == -INFINITY) ? 0.f : fast_exp2(v.x - M) * v.y;
+  float m_g = -INFINITY, l_g = 0.f, acc = 0.f;
+  for (int s0 = grp; s0 < n_splits; s0 += G * kCombineBatch) {
+    float2 st[kCombineBatch];
+    float ov[kCombineBatch];
+#pragma unroll
+    for (int j = 0; j < kCombineBatch; ++j) {
+      const int s = s0 + j * G;
+      st[j] = make_float2(-INFINITY, 0.f);
+      ov[j] = 0.f;
+      if (s < n_splits) {
+        st[j] = ml[slot0 + (size_t)s * rows_all];
+        ov[j] = o[(size_t)s * stride];
+      }
     }
-  const float L = block_sum(l_loc, red);
-
-  float acc0 = 0.f, acc1 = 0.f;
-  if (M > -INFINITY) {
-    const float* o = p.ws_o + slot0 * D + d;
-    const size_t stride = rows_all * D;
-    int s = grp;
-    for (; s + G < n_splits; s += 2 * G) {
-      const float m0 = ml[slot0 + (size_t)s * rows_all].x;
-      const float m1 = ml[slot0 + (size_t)(s + G) * rows_all].x;
-      const float o0 = o[(size_t)s * stride];
-      const float o1 = o[(size_t)(s + G) * stride];
-      acc0 = fmaf((m0 == -INFINITY) ? 0.f : fast_exp2(m0 - M), o0, acc0);
-      acc1 = fmaf((m1 == -INFINITY) ? 0.f : fast_exp2(m1 - M), o1, acc1);
+    float m_new = m_g;
+#pragma unroll
+    for (int j = 0; j < kCombineBatch; ++j) m_new = fmaxf(m_new, st[j].x);
+    if (m_new == -INFINITY) continue;
+    const float r = (m_g == -INFINITY) ? 0.f : fast_exp2(m_g - m_new);
+    l_g *= r;
+    acc *= r;
+#pragma unroll
+    for (int j = 0; j < kCombineBatch; ++j) {
+      const float w = (st[j].x == -INFINITY) ? 0.f : fast_exp2(st[j].x - m_new);
+      l_g = fmaf(w, st[j].y, l_g);
+      acc = fmaf(w, ov[j], acc);
     }
-    if (s < n_splits) {
-      const float m0 = ml[slot0 + (size_t)s * rows_all].x;
-      acc0 = fmaf((m0 == -INFINITY) ? 0.f : fast_exp2(m0 - M), o[(size_t)s * stride], acc0);
-    }
+    m_g = m_new;
   }
-  part[grp][d] = acc0 + acc1;
+  part[grp][d] = acc;
+  if (d == 0) {
+    part_m[grp] = m_g;
+    part_l[grp] = l_g;
+  }
   __syncthreads();
   if (grp == 0) {
-    float sum = part[0][d];
+    float M = part_m[0];
 #pragma unroll
-    for (int q = 1; q < G; ++q) sum += part[q][d];
+    for (int g = 1; g < G; ++g) M = fmaxf(M, part_m[g]);
+    float L = 0.f, sum = 0.f;
+    if (M > -INFINITY) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float w = (part_m[g] == -INFINITY) ? 0.f : fast_exp2(part_m[g] - M);
+        L = fmaf(w, part_l[g], L);
+        sum = fmaf(w, part[g][d], sum);
+      }
+    }
     const float val = (L > 0.f) ? sum / L : 0.f;
     const size_t orow = (size_t)b * rows_all + row;
     uint16_t bits;

@@ -114,7 +114,12 @@ struct DecodePlan {
   int groups;
 };
 
-DecodePlan decode_plan(int B, int Hkv, int D, int max_pages) {
+// With a left window (win_l >= 0) splits are counted from each sequence's first visible page,
+// so a sequence spans at most win_pages pages. Such a grid is small and each CTA pays a fixed
+// start-up latency (block table, Q and first page in flight), so the split is halved only while
+// the halved grid still fits one wave of two CTAs per SM, and never past the split count of the
+// unwindowed plan, so the workspace that mfa_decode_workspace_size reports stays sufficient.
+DecodePlan decode_plan(int B, int Hkv, int D, int max_pages, int Nq = 1, int win_l = -1) {
   DecodePlan pl;
   // kv heads per CTA: the largest divisor of Hkv whose token row (heads x D x 2 bytes) fits in
   // 1 KB, so that a 3-stage K+V page ring stays near 100 KB and two CTAs share an SM (one
@@ -135,6 +140,19 @@ DecodePlan decode_plan(int B, int Hkv, int D, int max_pages) {
   }
   pl.pages_per_split = s;
   pl.max_splits = (max_pages + s - 1) / s;
+  if (win_l >= 0) {
+    const long long win_pages = ((long long)win_l + Nq + mfa::kDecPage - 1) / mfa::kDecPage + 1;
+    const int span = (int)std::min<long long>(max_pages, win_pages);
+    const int cap = pl.max_splits;
+    if (g_split_pages_override <= 0) {
+      s = 32;
+      while (s > 4 && (long long)B * ((span + s / 2 - 1) / (s / 2)) * pl.groups <= 296 &&
+             (span + s / 2 - 1) / (s / 2) <= cap)
+        s /= 2;
+    }
+    pl.pages_per_split = s;
+    pl.max_splits = (span + s - 1) / s;
+  }
   return pl;
 }
 
@@ -278,9 +296,21 @@ int launch_decode(const mfa::DecodeParams& p, const DecodePlan& pl, cudaStream_t
   dim3 g1(pl.max_splits, p.B, pl.groups);
   k1<<<g1, (pl.heads_per_cta + 1) * 32, smem, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
+  // the combine is a programmatic dependent of phase 1: it is launched while the last phase-1
+  // CTAs still run and waits in griddepcontrol.wait until their workspace writes are visible
   dim3 g2(p.Hq * p.Nq, p.B, 1);
-  mfa::mfa_decode_combine_kernel<D, BF16><<<g2, mfa::kCombineThreads, 0, st>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = g2;
+  cfg.blockDim = dim3(mfa::kCombineThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, mfa::mfa_decode_combine_kernel<D, BF16>, p) != cudaSuccess)
+    return MFA_ERR_CUDA;
   mfa_launch_info li = {};
   li.kernel = 2;
   li.grid_x = g1.x;
@@ -583,12 +613,14 @@ size_t mfa_decode_workspace_size(int B, int Nq, int Hq, int Hkv, int D, int max_
   return align256(rows * D * sizeof(float)) + align256(rows * 2 * sizeof(float));
 }
 
-int mfa_decode_splitkv(const void* q, const void* k_pages, const void* v_pages,
-                       const int32_t* block_table, const int32_t* seq_lens, void* out, float* lse,
-                       int B, int Nq, int Hq, int Hkv, int D, int page_size, int max_pages_per_seq,
-                       int num_pages, float scale, int causal, float softcap, int dtype,
-                       void* workspace, size_t workspace_bytes, void* stream) {
+int mfa_decode_splitkv_window(const void* q, const void* k_pages, const void* v_pages,
+                              const int32_t* block_table, const int32_t* seq_lens, void* out,
+                              float* lse, int B, int Nq, int Hq, int Hkv, int D, int page_size,
+                              int max_pages_per_seq, int num_pages, float scale, int causal,
+                              int win_l, float softcap, int dtype, void* workspace,
+                              size_t workspace_bytes, void* stream) {
   if (dtype != MFA_DTYPE_FP16 && dtype != MFA_DTYPE_BF16) return MFA_ERR_BAD_DTYPE;
+  if (win_l < -1) return MFA_ERR_BAD_WINDOW;
   int rc = validate_decode(B, Nq, Hq, Hkv, D, page_size, max_pages_per_seq);
   if (rc != MFA_OK) return rc;
   if (num_pages < 1) return MFA_ERR_BAD_SHAPE;
@@ -604,7 +636,7 @@ int mfa_decode_splitkv(const void* q, const void* k_pages, const void* v_pages,
   const size_t need = mfa_decode_workspace_size(B, Nq, Hq, Hkv, D, max_pages_per_seq, page_size);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
     return MFA_ERR_WORKSPACE;
-  DecodePlan pl = decode_plan(B, Hkv, D, max_pages_per_seq);
+  DecodePlan pl = decode_plan(B, Hkv, D, max_pages_per_seq, Nq, win_l);
   mfa::DecodeParams p;
   std::memset(&p, 0, sizeof(p));
   p.q = static_cast<const uint16_t*>(q);
@@ -628,6 +660,7 @@ int mfa_decode_splitkv(const void* q, const void* k_pages, const void* v_pages,
   p.max_splits = pl.max_splits;
   p.heads_per_cta = pl.heads_per_cta;
   p.causal = causal ? 1 : 0;
+  p.win_l = win_l;
   const float log2e = 1.4426950408889634f;
   if (softcap > 0.f) {
     p.softcap = softcap;
@@ -641,6 +674,16 @@ int mfa_decode_splitkv(const void* q, const void* k_pages, const void* v_pages,
   const bool bf = dtype == MFA_DTYPE_BF16;
   if (D == 128) return bf ? launch_decode<128, true>(p, pl, st) : launch_decode<128, false>(p, pl, st);
   return bf ? launch_decode<64, true>(p, pl, st) : launch_decode<64, false>(p, pl, st);
+}
+
+int mfa_decode_splitkv(const void* q, const void* k_pages, const void* v_pages,
+                       const int32_t* block_table, const int32_t* seq_lens, void* out, float* lse,
+                       int B, int Nq, int Hq, int Hkv, int D, int page_size, int max_pages_per_seq,
+                       int num_pages, float scale, int causal, float softcap, int dtype,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  return mfa_decode_splitkv_window(q, k_pages, v_pages, block_table, seq_lens, out, lse, B, Nq, Hq,
+                                   Hkv, D, page_size, max_pages_per_seq, num_pages, scale, causal,
+                                   -1, softcap, dtype, workspace, workspace_bytes, stream);
 }
 
 const char* mfa_status_string(int code) {
