@@ -56,7 +56,7 @@ extern "C" {
 #define MFA_ERR_NULL_POINTER        -1   /* a required pointer is NULL */
 #define MFA_ERR_MISALIGNED          -2   /* a tensor pointer is not 16-byte aligned */
 #define MFA_ERR_BAD_DTYPE           -3   /* dtype not MFA_DTYPE_FP16 / MFA_DTYPE_BF16 */
-#define MFA_ERR_BAD_HEAD_DIM        -4   /* D not in {64, 128} */
+#define MFA_ERR_BAD_HEAD_DIM        -4   /* D not in {64, 128} (decode: {64, 128, 256}) */
 #define MFA_ERR_BAD_SHAPE           -5   /* negative size, or a size whose element count overflows */
 #define MFA_ERR_GQA_GEOMETRY        -6   /* Hkv < 1 or Hq not a multiple of Hkv */
 #define MFA_ERR_BAD_WINDOW          -7   /* window bound below -1 */
@@ -239,7 +239,7 @@ size_t mfa_decode_workspace_size(int B, int Nq, int Hq, int Hkv, int D,
  *                [0, num_pages); later entries are never read    (device)
  *   seq_lens     int32 [B], each in [0, max_pages_per_seq * 16]  (device)
  *   out          [B, Hq, Nq, D] dtype; lse float32 [B, Hq, Nq] or NULL   (device)
- *   page_size must be 16; (Hq / Hkv) * Nq <= 16; D in {64, 128};
+ *   page_size must be 16; (Hq / Hkv) * Nq <= 16; D in {64, 128, 256};
  *   workspace: device scratch of at least mfa_decode_workspace_size(...) bytes, 256-byte
  *   aligned, owned by the caller; its contents need no initialisation and are overwritten.
  * Page slots at or past a sequence's length are never used in the arithmetic, so they may hold

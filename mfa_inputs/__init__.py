@@ -439,6 +439,14 @@ def workloads():
         "decode_b8_hq32_hkv8_d128_bf16_len8k_128k": DecodeCase(
             "decode_b8_hq32_hkv8_d128_bf16_len8k_128k", 8, 1, 32, 8, 128, BF16, 8192, 131072,
             seed=1005),
+        # speculative-decoding verify: 4 draft tokens per sequence against the same caches
+        "decode_verify_nq4_b8_hq32_hkv8_d128_bf16_len8k_128k": DecodeCase(
+            "decode_verify_nq4_b8_hq32_hkv8_d128_bf16_len8k_128k", 8, 4, 32, 8, 128, BF16, 8192,
+            131072, seed=1005),
+        # D = 256 heads (two kv heads per phase-1 CTA)
+        "decode_b8_hq16_hkv8_d256_bf16_len4k_32k": DecodeCase(
+            "decode_b8_hq16_hkv8_d256_bf16_len4k_32k", 8, 1, 16, 8, 256, BF16, 4096, 32768,
+            seed=1009),
         # the same cache lengths under a 4096-token left window (each query sees 4096 keys)
         "decode_window4k_b8_hq32_hkv8_d128_bf16_len8k_128k": DecodeCase(
             "decode_window4k_b8_hq32_hkv8_d128_bf16_len8k_128k", 8, 1, 32, 8, 128, BF16, 8192,

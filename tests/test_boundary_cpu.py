@@ -144,6 +144,34 @@ def test_decode_rejects_malformed(kw, code):
     assert dec(**kw) == code
 
 
+def decw(win_l, **kw):
+    ws = kw.pop("ws_bytes", 1 << 30)
+    args = dict(q=A, k=A, v=A, table=A, lens=A, out=A, lse=A, B=8, Nq=1, Hq=32, Hkv=8, D=128,
+                page=16, max_pages=8192, num_pages=40000, scale=0.088, causal=1, win_l=win_l,
+                softcap=0.0, dtype=1, ws=A, ws_bytes=ws, stream=None)
+    args.update(kw)
+    return mfa.lib.mfa_decode_splitkv_window(*args.values())
+
+
+@pytest.mark.parametrize("win_l,kw,code", [
+    (-2, {}, -7), (-100, {}, -7), (100, dict(D=80), -4), (100, dict(Nq=5), -10),
+    (100, dict(ws_bytes=1024), -12), (0, dict(table=None), -1),
+])
+@no_device
+def test_decode_window_rejects_malformed(win_l, kw, code):
+    assert decw(win_l, **kw) == code
+
+
+def test_decode_head_dims():
+    """Decode takes D = 64, 128 and 256 (two kv heads per CTA at 256); other sizes are refused
+    before anything else is looked at."""
+    for D in (64, 128, 256):
+        assert mfa.mfa_decode_workspace_size(8, 1, 32, 8, D, 8192) == \
+            8 * 256 * 32 * D * 4 + 8 * 256 * 32 * 2 * 4
+    for D in (32, 96, 192, 512):
+        assert mfa.mfa_decode_workspace_size(8, 1, 32, 8, D, 8192) == 0
+
+
 def test_decode_workspace_size_is_shape_only():
     n = mfa.mfa_decode_workspace_size(8, 1, 32, 8, 128, 8192)
     # 8 sequences x 256 splits of 32 pages x 32 rows x (128 + 2) floats

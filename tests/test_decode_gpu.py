@@ -31,6 +31,13 @@ SMALL = [
        softcap=30.0, win_l=250, seed=69),
     Dc("window_edge_lengths_fp16", 6, 1, 8, 2, 64, mi.FP16, 0, 0,
        fixed_lens=[1, 16, 17, 0, 33, 513], max_pages=40, win_l=16, seed=70),
+    # D = 256: two kv heads per CTA when Hkv is even, one otherwise
+    Dc("d256_nq1_gqa4_bf16", 3, 1, 16, 4, 256, mi.BF16, 1, 1500, seed=72),
+    Dc("d256_nq4_gqa4_window_fp16", 2, 4, 8, 2, 256, mi.FP16, 100, 900, win_l=200, seed=73),
+    Dc("d256_nq2_softcap_bf16", 2, 2, 8, 4, 256, mi.BF16, 1, 600, softcap=30.0, seed=74),
+    Dc("d256_odd_kv_heads_fp16", 2, 1, 6, 3, 256, mi.FP16, 1, 700, seed=75),
+    Dc("d256_edge_lengths_noncausal_bf16", 5, 3, 4, 4, 256, mi.BF16, 0, 0, causal=False,
+       fixed_lens=[1, 16, 0, 17, 300], max_pages=20, seed=76),
 ]
 
 
@@ -65,15 +72,16 @@ def test_small_cases_match_oracle(cuda_device, case):
     assert mfa.mfa_device_status() == (0, 0)
 
 
-@pytest.mark.parametrize("name", ["decode_b8_hq32_hkv8_d128_bf16_len8k_128k",
-                                  "decode_window4k_b8_hq32_hkv8_d128_bf16_len8k_128k"])
+@pytest.mark.parametrize("name", sorted(n for n, c in mi.workloads().items()
+                                         if isinstance(c, mi.DecodeCase)))
 def test_full_size_sampled_rows(cuda_device, name):
     case = mi.workloads()[name]
     q, k, v, table, lens = case.tensors()
     o, lse = run_gpu(case, q, k, v, table, lens)
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
     rng = np.random.default_rng(5)
-    rows = np.array([(b, h, 0) for b in range(case.B) for h in sorted(rng.choice(32, 5, replace=False))])
+    rows = np.array([(b, h, t) for b in range(case.B)
+                     for h in sorted(rng.choice(case.Hq, 5, replace=False)) for t in range(case.Nq)])
     o_ref, l_ref = oracle.decode_rows(q, k, v, table, lens, rows, case.scale_f32(), case.causal,
                                       case.softcap, to_f64=lambda a: mi.widen(a, case.dtype),
                                       win_l=case.win_l)

@@ -67,6 +67,10 @@ __device__ __forceinline__ int dec_first_page(const DecodeParams& p, int len) {
   return max(0, len - p.Nq - p.win_l) / kDecPage;
 }
 
+// kv heads per phase-1 CTA at most: a token row of all of them fits in 1 KB
+template <int D>
+constexpr int kDecMaxHeads = 1024 / (2 * D);
+
 template <int D>
 __host__ __device__ constexpr int dec_row_bytes(int hg) {
   return hg * D * 2 + 16;
@@ -78,7 +82,7 @@ __host__ __device__ constexpr int dec_smem_bytes(int hg) {
 }
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(9 * 32) mfa_decode_phase1_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__((kDecMaxHeads<D> + 1) * 32) mfa_decode_phase1_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int hg = p.heads_per_cta;
   const int row_bytes = dec_row_bytes<D>(hg);

@@ -290,9 +290,9 @@ template <int D, bool BF16>
 int launch_decode(const mfa::DecodeParams& p, const DecodePlan& pl, cudaStream_t st) {
   static bool smem_done[kMaxDevices] = {};
   const int smem = mfa::dec_smem_bytes<D>(pl.heads_per_cta);
-  // the largest plan (8 heads per CTA) sets the attribute for all
+  // the largest plan (1024 / (2 D) heads per CTA) sets the attribute for all
   auto k1 = mfa::mfa_decode_phase1_kernel<D, BF16>;
-  if (!ensure_smem(k1, mfa::dec_smem_bytes<D>(8), smem_done)) return MFA_ERR_CUDA;
+  if (!ensure_smem(k1, mfa::dec_smem_bytes<D>(mfa::kDecMaxHeads<D>), smem_done)) return MFA_ERR_CUDA;
   dim3 g1(pl.max_splits, p.B, pl.groups);
   k1<<<g1, (pl.heads_per_cta + 1) * 32, smem, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
@@ -526,7 +526,7 @@ int mfa_fwd_paged(const void* q, const void* k_pages, const void* v_pages, const
 }
 
 static int validate_decode(int B, int Nq, int Hq, int Hkv, int D, int page_size, int max_pages) {
-  if (D != 64 && D != 128) return MFA_ERR_BAD_HEAD_DIM;
+  if (D != 64 && D != 128 && D != 256) return MFA_ERR_BAD_HEAD_DIM;
   if (B < 0 || Hq < 0) return MFA_ERR_BAD_SHAPE;
   if (Nq < 1 || Nq > 4) return Nq < 1 ? MFA_ERR_BAD_SHAPE : MFA_ERR_NQ_TOO_LARGE;
   if (Hkv < 1 || Hq % Hkv != 0 || Hq < 1) return MFA_ERR_GQA_GEOMETRY;
@@ -672,6 +672,7 @@ int mfa_decode_splitkv_window(const void* q, const void* k_pages, const void* v_
   if (pl.max_splits > 0x7FFFFFFF || B > 65535 || pl.groups > 65535) return MFA_ERR_BAD_SHAPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool bf = dtype == MFA_DTYPE_BF16;
+  if (D == 256) return bf ? launch_decode<256, true>(p, pl, st) : launch_decode<256, false>(p, pl, st);
   if (D == 128) return bf ? launch_decode<128, true>(p, pl, st) : launch_decode<128, false>(p, pl, st);
   return bf ? launch_decode<64, true>(p, pl, st) : launch_decode<64, false>(p, pl, st);
 }
