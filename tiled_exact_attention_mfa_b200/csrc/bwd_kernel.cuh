@@ -129,7 +129,7 @@ struct BwdKvSmem {
   float nl[kBwdStages][kBwdBM];  // L_i log2 e of the stage's query rows (0 past Nq / no key)
   float dd[kBwdStages][kBwdBM];  // D_i of the stage's query rows
   uint64_t bar_kv, bar_full[kBwdStages], bar_empty[kBwdStages];
-  uint64_t bar_sp, bar_ds, bar_mm, bar_final;
+  uint64_t bar_sp, bar_ds[2], bar_mm, bar_final;  // bar_ds[ch]: chunk ch of every warp stored
   uint32_t tmem_base;
   int abort;
 };
@@ -181,7 +181,8 @@ __global__ void __launch_bounds__(kBwdKvThreads, 1) mfa_bwd_dkv_kernel(const __g
       mbar_init(smem_u32(&sm.bar_empty[st]), 1);
     }
     mbar_init(smem_u32(&sm.bar_sp), 1);
-    mbar_init(smem_u32(&sm.bar_ds), 8);
+    mbar_init(smem_u32(&sm.bar_ds[0]), 8);
+    mbar_init(smem_u32(&sm.bar_ds[1]), 8);
     mbar_init(smem_u32(&sm.bar_mm), 1);
     mbar_init(smem_u32(&sm.bar_final), 1);
     sm.abort = 0;
@@ -277,17 +278,31 @@ __global__ void __launch_bounds__(kBwdKvThreads, 1) mfa_bwd_dkv_kernel(const __g
         for (int kk = 0; kk < D / 16; ++kk)
           tc_mma_ss(tmem + 128, bwd_desc_k(va, kk), bwd_desc_k(oa, kk), id_s, kk > 0 ? 1u : 0u);
         tc_commit(smem_u32(&sm.bar_sp));
-        if (!(ok = mbar_wait(smem_u32(&sm.bar_ds), u & 1, abort, 1204))) break;
-        tc_fence_after();
-        // packed P^T / dS^T of query step kk (16 queries): half kk / 4 at column 64 (kk / 4)
+        // packed P^T / dS^T of query step kk (16 queries): half kk / 4 at column 64 (kk / 4),
+        // written by chunk (kk / 2) % 2 of that half's warps. The steps of chunk 0 go to the
+        // tensor pipe while the elementwise warps still work on chunk 1 (disjoint columns).
 #pragma unroll
-        for (int kk = 0; kk < kBwdBM / 16; ++kk)
-          tc_mma_ts(tmem + 256, tmem + (kk >> 2) * 64 + (kk & 3) * 8, bwd_desc_mn(oa, kk), id_o,
-                    (u > 0 || kk > 0) ? 1u : 0u);
+        for (int ch = 0; ch < 2; ++ch) {
+          if (!(ok = mbar_wait(smem_u32(&sm.bar_ds[ch]), u & 1, abort, 1204 + ch))) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kBwdBM / 16; ++kk)
-          tc_mma_ts(tmem + 256 + D, tmem + 128 + (kk >> 2) * 64 + (kk & 3) * 8, bwd_desc_mn(qa, kk),
-                    id_o, (u > 0 || kk > 0) ? 1u : 0u);
+          for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+              const int kk = hf * 4 + ch * 2 + k2;
+              tc_mma_ts(tmem + 256, tmem + (kk >> 2) * 64 + (kk & 3) * 8, bwd_desc_mn(oa, kk),
+                        id_o, (u > 0 || kk > 0) ? 1u : 0u);
+            }
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+              const int kk = hf * 4 + ch * 2 + k2;
+              tc_mma_ts(tmem + 256 + D, tmem + 128 + (kk >> 2) * 64 + (kk & 3) * 8,
+                        bwd_desc_mn(qa, kk), id_o, (u > 0 || kk > 0) ? 1u : 0u);
+            }
+        }
+        if (!ok) break;
         tc_commit(smem_u32(&sm.bar_mm));
         tc_commit(smem_u32(&sm.bar_empty[st]));
       }
@@ -368,11 +383,11 @@ __global__ void __launch_bounds__(kBwdKvThreads, 1) mfa_bwd_dkv_kernel(const __g
         // this warp has already read
         tmem_st16(tmem + lane_base + half * 64 + ch * 16, pk);
         tmem_st16(tmem + lane_base + 128 + half * 64 + ch * 16, dk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.bar_ds[ch]));
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.bar_ds));
     }
     // ---- epilogue: lower-column warps write dV, upper-column warps scale * dK, of their key rows
     bool have = false;
