@@ -78,6 +78,32 @@ def test_backward_is_deterministic_and_empty_rows_get_zero_dq(cuda_device):
     assert np.all(g1[0][:, :, :case.Nq - case.Nk] == 0)
 
 
+@pytest.mark.parametrize("idx", [0, 5, 6])
+def test_backward_repeats_bitwise(cuda_device, idx):
+    """Eight backward calls on the same inputs give the same bits: the passes have no atomics, so
+    any difference would come from a read that raced a write (an early phase wait, a buffer
+    reused before its reader finished). The capped cases take the fastest elementwise path, where
+    the dQ epilogue once read its accumulator before the last MMAs completed."""
+    import torch
+    import tiled_exact_attention_mfa_b200 as mfa
+    case = CASES[idx]
+    q, k, v = case.tensors()
+    qt, kt, vt, dot = (to_torch(x, case.dtype) for x in (q, k, v, dout_bits(case)))
+    win = (case.win_l, case.win_r)
+    out, lse = mfa.mfa_fwd(qt, kt, vt, scale=case.scale_f32(), causal=case.causal, window=win,
+                           softcap=case.softcap)
+    first = None
+    for _ in range(8):
+        g = mfa.mfa_bwd(qt, kt, vt, out, dot, lse, scale=case.scale_f32(), causal=case.causal,
+                        window=win, softcap=case.softcap)
+        torch.cuda.synchronize()
+        if first is None:
+            first = [t.clone() for t in g]
+        else:
+            for a, b in zip(first, g):
+                assert torch.equal(a, b)
+
+
 def test_backward_empty_sides(cuda_device):
     import torch
     import tiled_exact_attention_mfa_b200 as mfa

@@ -126,7 +126,7 @@ struct BwdKvSmem {
   uint8_t v[kTile];
   uint8_t q[kBwdStages][kTile];
   uint8_t dout[kBwdStages][kTile];
-  float nl[kBwdStages][kBwdBM];  // L_i log2 e of the stage's query rows (0 past Nq / no key)
+  float nl[kBwdStages][kBwdBM];  // -L_i log2 e of the stage's query rows (0 past Nq / no key)
   float dd[kBwdStages][kBwdBM];  // D_i of the stage's query rows
   uint64_t bar_kv, bar_full[kBwdStages], bar_empty[kBwdStages];
   uint64_t bar_sp, bar_ds[2], bar_mm, bar_final;  // bar_ds[ch]: chunk ch of every warp stored
@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(kBwdKvThreads, 1) mfa_bwd_dkv_kernel(const __g
         const int row0 = (qt_lo + u % n_qt) * kBwdBM;
         const bool ok = use == 0 || mbar_wait(smem_u32(&sm.bar_empty[st]), (use - 1) & 1, abort, 1101);
         if (!__all_sync(0xffffffffu, ok)) break;
-        // L (as L log2 e) and D of the tile's rows, 0 past Nq or where L = -inf (no visible key)
+        // -L log2 e and D of the tile's rows, 0 past Nq or where L = -inf (no visible key)
         const size_t base = (size_t)(b * p.Hq + h) * p.Nq;
 #pragma unroll
         for (int rr = 0; rr < kBwdBM; rr += 32) {
@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(kBwdKvThreads, 1) mfa_bwd_dkv_kernel(const __g
             d = p.dvec[base + i];
             if (!(l > -INFINITY)) l = 0.f;
           }
-          sm.nl[st][rr + lane] = l * 1.4426950408889634f;
+          sm.nl[st][rr + lane] = l * -1.4426950408889634f;
           sm.dd[st][rr + lane] = d;
         }
         __syncwarp();
@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(kBwdKvThreads, 1) mfa_bwd_dkv_kernel(const __g
         uint32_t sr[32], dr[32];
         tmem_ld32(tmem + lane_base + half * 64 + ch * 32, sr);
         tmem_ld32(tmem + lane_base + 128 + half * 64 + ch * 32, dr);
-        tmem_wait_ld();
+        tmem_wait_ld(sr, dr);
         bool poly = false;
         if (SOFTCAP) {
           float am = 0.f;
@@ -349,36 +349,51 @@ __global__ void __launch_bounds__(kBwdKvThreads, 1) mfa_bwd_dkv_kernel(const __g
           poly = __all_sync(0xffffffffu, am * p.cap_in <= kTanhPolyMax);
         }
         uint32_t pk[16], dk[16];
+        // P^T = 2^(s c - L log2 e) (scores past the row / column limits are 0 on boundary tiles)
+        // and dS^T = P^T (dP^T - D) [(1 - tanh^2) with a cap], two columns per packed f32x2 step
+        auto chunk = [&](auto interior_c) {
+          constexpr bool kInterior = decltype(interior_c)::value;
 #pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 n4 = *reinterpret_cast<const float4*>(nlp + ch * 32 + e4 * 4);
-          const float4 d4 = *reinterpret_cast<const float4*>(ddp + ch * 32 + e4 * 4);
-          const float nv[4] = {n4.x, n4.y, n4.z, n4.w};
-          const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
-          float pv[4], dsv[4];
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const ulonglong2 n2 = *reinterpret_cast<const ulonglong2*>(nlp + ch * 32 + e4 * 4);
+            const ulonglong2 d2 = *reinterpret_cast<const ulonglong2*>(ddp + ch * 32 + e4 * 4);
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int e = e4 * 4 + q4;
-            const float sv = __uint_as_float(sr[e]);
-            float x, fac = 1.f;
-            if (SOFTCAP) {
-              const float tt = bwd_tanh(sv * p.cap_in, poly);
-              x = fmaf(tt, cc, -nv[q4]);
-              fac = fmaf(-tt, tt, 1.f);
-            } else {
-              x = fmaf(sv, c, -nv[q4]);
+            for (int hp = 0; hp < 2; ++hp) {
+              const int e = e4 * 4 + hp * 2;
+              const uint64_t nn = hp ? n2.y : n2.x;
+              const uint64_t dd2 = hp ? d2.y : d2.x;
+              float p0, p1;
+              uint64_t fac2 = 0;
+              if constexpr (SOFTCAP) {
+                const float t0 = bwd_tanh(__uint_as_float(sr[e]) * p.cap_in, poly);
+                const float t1 = bwd_tanh(__uint_as_float(sr[e + 1]) * p.cap_in, poly);
+                const uint64_t t2 = f2_pack(t0, t1);
+                f2_unpack(f2_fma(t2, f2_pack(cc, cc), nn), p0, p1);
+                // 1 - t^2 with one rounding, as fmaf(-t, t, 1)
+                fac2 = f2_fma(f2_mul(t2, f2_pack(-1.f, -1.f)), t2, f2_pack(1.f, 1.f));
+              } else {
+                f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])),
+                                 f2_pack(c, c), nn), p0, p1);
+              }
+              p0 = fast_exp2(p0);
+              p1 = fast_exp2(p1);
+              if constexpr (!kInterior) {
+                const int i = col0 + ch * 32 + e;
+                if (i < ilo || i > ihi) p0 = 0.f;
+                if (i + 1 < ilo || i + 1 > ihi) p1 = 0.f;
+              }
+              uint64_t ds2 = f2_mul(f2_pack(p0, p1),
+                                    f2_sub(f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), dd2));
+              if constexpr (SOFTCAP) ds2 = f2_mul(ds2, fac2);
+              float s0, s1;
+              f2_unpack(ds2, s0, s1);
+              pk[e >> 1] = pack2<BF16>(p0, p1);
+              dk[e >> 1] = pack2<BF16>(s0, s1);
             }
-            float pe = fast_exp2(x);
-            const int i = col0 + ch * 32 + e;
-            if (!interior && (i < ilo || i > ihi)) pe = 0.f;
-            pv[q4] = pe;
-            dsv[q4] = pe * (__uint_as_float(dr[e]) - dv4[q4]) * fac;
           }
-          pk[2 * e4] = pack2<BF16>(pv[0], pv[1]);
-          pk[2 * e4 + 1] = pack2<BF16>(pv[2], pv[3]);
-          dk[2 * e4] = pack2<BF16>(dsv[0], dsv[1]);
-          dk[2 * e4 + 1] = pack2<BF16>(dsv[2], dsv[3]);
-        }
+        };
+        if (interior) chunk(std::true_type{});
+        else chunk(std::false_type{});
         // packed values of columns 64 half + 32 ch .. land on columns 64 half + 16 ch .., which
         // this warp has already read
         tmem_st16(tmem + lane_base + half * 64 + ch * 16, pk);
@@ -392,7 +407,8 @@ __global__ void __launch_bounds__(kBwdKvThreads, 1) mfa_bwd_dkv_kernel(const __g
     // ---- epilogue: lower-column warps write dV, upper-column warps scale * dK, of their key rows
     bool have = false;
     if (n_steps > 0 && !*abort) {
-      have = mbar_wait(smem_u32(&sm.bar_mm), (n_steps - 1) & 1, abort, 1302);
+      // bar_final: one commit after the MMA thread's last MMA, so a single-phase wait
+      have = mbar_wait(smem_u32(&sm.bar_final), 0, abort, 1302);
       tc_fence_after();
     }
     have = __all_sync(0xffffffffu, have);
@@ -404,7 +420,7 @@ __global__ void __launch_bounds__(kBwdKvThreads, 1) mfa_bwd_dkv_kernel(const __g
       uint32_t o[32];
       if (have) {
         tmem_ld32(tmem + lane_base + 256 + half * D + cb, o);
-        tmem_wait_ld();
+        tmem_wait_ld(o);
       } else {
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[e] = 0u;
@@ -451,7 +467,11 @@ struct BwdQSmem {
   uint8_t k[kBwdStages][kTile];
   uint8_t v[kBwdStages][kTile];
   uint64_t bar_qo, bar_full[kBwdStages], bar_empty[kBwdStages];
-  uint64_t bar_sp, bar_ld, bar_ds, bar_mm, bar_final;
+  // bar_ds[u % 2]: every elementwise warp stored dS of key tile u. S / dP of tile u + 1 are
+  // issued once every warp has loaded tile u, so a fast warp can finish tile u + 1 before a slow
+  // one finishes tile u; alternating barriers keep its arrival out of tile u's phase (it cannot
+  // get two tiles ahead: S / dP of tile u + 2 wait for every warp to load tile u + 1).
+  uint64_t bar_sp, bar_ld, bar_ds[2], bar_final;
   uint32_t tmem_base;
   int abort;
 };
@@ -494,8 +514,8 @@ __global__ void __launch_bounds__(kBwdQThreads, 1) mfa_bwd_dq_kernel(const __gri
     }
     mbar_init(smem_u32(&sm.bar_sp), 1);
     mbar_init(smem_u32(&sm.bar_ld), 8);
-    mbar_init(smem_u32(&sm.bar_ds), 8);
-    mbar_init(smem_u32(&sm.bar_mm), 1);
+    mbar_init(smem_u32(&sm.bar_ds[0]), 8);
+    mbar_init(smem_u32(&sm.bar_ds[1]), 8);
     mbar_init(smem_u32(&sm.bar_final), 1);
     sm.abort = 0;
     fence_barrier_init();
@@ -573,14 +593,13 @@ __global__ void __launch_bounds__(kBwdQThreads, 1) mfa_bwd_dq_kernel(const __gri
           if (!(ok = mbar_wait(smem_u32(&sm.bar_ld), u & 1, abort, 1503))) break;
           if (!(ok = issue_sdp(u + 1))) break;
         }
-        if (!(ok = mbar_wait(smem_u32(&sm.bar_ds), u & 1, abort, 1504))) break;
+        if (!(ok = mbar_wait(smem_u32(&sm.bar_ds[u & 1]), (u >> 1) & 1, abort, 1504))) break;
         tc_fence_after();
         const uint32_t ka = smem_u32(sm.k[u % kBwdStages]);
         const uint32_t ds_col = 384 + (u & 1) * 64;
 #pragma unroll
         for (int kk = 0; kk < kBwdBM / 16; ++kk)
           tc_mma_ts(tmem + 256, tmem + ds_col + kk * 8, bwd_desc_mn(ka, kk), id_o, (u > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(smem_u32(&sm.bar_mm));
         tc_commit(smem_u32(&sm.bar_empty[u % kBwdStages]));
       }
       tc_commit(smem_u32(&sm.bar_final));
@@ -603,7 +622,7 @@ __global__ void __launch_bounds__(kBwdQThreads, 1) mfa_bwd_dq_kernel(const __gri
       nl = p.lse[idx];
       dd = p.dvec[idx];
       if (!(nl > -INFINITY)) nl = 0.f;
-      nl *= 1.4426950408889634f;
+      nl *= -1.4426950408889634f;  // -L log2 e
     } else {
       klo = 1;
       khi = 0;
@@ -620,7 +639,7 @@ __global__ void __launch_bounds__(kBwdQThreads, 1) mfa_bwd_dq_kernel(const __gri
       tmem_ld32(tmem + lane_base + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_ld32(tmem + lane_base + 128 + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
       tmem_ld32(tmem + lane_base + 128 + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
-      tmem_wait_ld();
+      tmem_wait_ld(sr, dr);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.bar_ld));  // S / dP columns may be overwritten now
@@ -633,28 +652,44 @@ __global__ void __launch_bounds__(kBwdQThreads, 1) mfa_bwd_dq_kernel(const __gri
         poly = __all_sync(0xffffffffu, am * p.cap_in <= kTanhPolyMax);
       }
       uint32_t dk[32];
+      // dS = 2^(s c - L log2 e) (dP - D) [(1 - tanh^2) with a cap], zero past the row's key limits
+      // on boundary tiles; two columns per packed f32x2 step
+      const uint64_t nl2 = f2_pack(nl, nl), dd2 = f2_pack(dd, dd);
+      auto tile = [&](auto interior_c) {
+        constexpr bool kInterior = decltype(interior_c)::value;
 #pragma unroll
-      for (int e2 = 0; e2 < 32; ++e2) {
-        float dsv[2];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int e = 2 * e2 + h2;
-          const float sv = __uint_as_float(sr[e]);
-          float x, fac = 1.f;
-          if (SOFTCAP) {
-            const float tt = bwd_tanh(sv * p.cap_in, poly);
-            x = fmaf(tt, cc, -nl);
-            fac = fmaf(-tt, tt, 1.f);
+        for (int e2 = 0; e2 < 32; ++e2) {
+          const int e = 2 * e2;
+          float p0, p1;
+          uint64_t fac2 = 0;
+          if constexpr (SOFTCAP) {
+            const float t0 = bwd_tanh(__uint_as_float(sr[e]) * p.cap_in, poly);
+            const float t1 = bwd_tanh(__uint_as_float(sr[e + 1]) * p.cap_in, poly);
+            const uint64_t t2 = f2_pack(t0, t1);
+            f2_unpack(f2_fma(t2, f2_pack(cc, cc), nl2), p0, p1);
+            // 1 - t^2 with one rounding, as fmaf(-t, t, 1)
+            fac2 = f2_fma(f2_mul(t2, f2_pack(-1.f, -1.f)), t2, f2_pack(1.f, 1.f));
           } else {
-            x = fmaf(sv, c, -nl);
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])),
+                             f2_pack(c, c), nl2), p0, p1);
           }
-          float pe = fast_exp2(x);
-          const int j = kc0 + e;
-          if (!interior && (j < klo || j > khi)) pe = 0.f;
-          dsv[h2] = pe * (__uint_as_float(dr[e]) - dd) * fac;
+          p0 = fast_exp2(p0);
+          p1 = fast_exp2(p1);
+          if constexpr (!kInterior) {
+            const int j = kc0 + e;
+            if (j < klo || j > khi) p0 = 0.f;
+            if (j + 1 < klo || j + 1 > khi) p1 = 0.f;
+          }
+          uint64_t ds2 = f2_mul(f2_pack(p0, p1),
+                                f2_sub(f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])), dd2));
+          if constexpr (SOFTCAP) ds2 = f2_mul(ds2, fac2);
+          float s0, s1;
+          f2_unpack(ds2, s0, s1);
+          dk[e2] = pack2<BF16>(s0, s1);
         }
-        dk[e2] = pack2<BF16>(dsv[0], dsv[1]);
-      }
+      };
+      if (interior) tile(std::true_type{});
+      else tile(std::false_type{});
       // dS of tile u into buffer u % 2; the dQ MMA of tile u - 2 that read it is complete (the
       // commit that signalled S of tile u came after it)
       const uint32_t ds_col = 384 + (u & 1) * 64 + half * 32;
@@ -663,12 +698,15 @@ __global__ void __launch_bounds__(kBwdQThreads, 1) mfa_bwd_dq_kernel(const __gri
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.bar_ds));
+      if (lane == 0) mbar_arrive(smem_u32(&sm.bar_ds[u & 1]));
     }
     // ---- epilogue: scale * dQ of this query row, this warp's half of the columns
     bool have = false;
     if (n_kt > 0 && !*abort) {
-      have = mbar_wait(smem_u32(&sm.bar_mm), (n_kt - 1) & 1, abort, 1602);
+      // bar_final: one commit after the MMA thread's last dQ MMA. (A parity wait on a barrier
+      // committed once per key tile would be ambiguous here: when these warps finish their last
+      // tile the MMA thread may not yet have issued dQ of the tile before it.)
+      have = mbar_wait(smem_u32(&sm.bar_final), 0, abort, 1602);
       tc_fence_after();
     }
     have = __all_sync(0xffffffffu, have);
@@ -678,7 +716,7 @@ __global__ void __launch_bounds__(kBwdQThreads, 1) mfa_bwd_dq_kernel(const __gri
       uint32_t o[32];
       if (have) {
         tmem_ld32(tmem + lane_base + 256 + half * (D / 2) + cb, o);
-        tmem_wait_ld();
+        tmem_wait_ld(o);
       } else {
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[e] = 0u;

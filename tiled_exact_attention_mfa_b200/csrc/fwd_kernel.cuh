@@ -441,7 +441,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sraw[32]));
       tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&sraw[64]));
       tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&sraw[96]));
-      tmem_wait_ld();
+      tmem_wait_ld(sraw);
       float* s = reinterpret_cast<float*>(sraw);
 
       const int k0 = (kt_lo + tile_of(j)) * kFwdBN;
@@ -521,7 +521,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         for (int cb = 0; cb < D; cb += 32) {
           uint32_t o[32];
           tmem_ld32(t_o + cb, o);
-          tmem_wait_ld();
+          tmem_wait_ld(o);
           const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -628,7 +628,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       uint32_t o[32];
       if (have_o) {
         tmem_ld32(t_o + cb, o);
-        tmem_wait_ld();
+        tmem_wait_ld(o);
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] = 0u;

@@ -189,8 +189,33 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[15])
       : "memory");
 }
-__device__ __forceinline__ void tmem_wait_ld() {
+// tcgen05.ld fills its destination registers asynchronously: they hold the loaded values only
+// after tcgen05.wait::ld. An asm statement without register operands does not stop the compiler
+// from scheduling arithmetic on those registers above the wait, so after the wait every loaded
+// array goes through an empty asm that takes its registers as read-write operands: each later use
+// depends on that asm, and volatile asm statements keep their order.
+__device__ __forceinline__ void tmem_reg_fence32(uint32_t (&r)[32]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+template <int N>
+__device__ __forceinline__ void tmem_reg_fence(uint32_t (&r)[N]) {
+  static_assert(N % 32 == 0, "fence whole 32-register groups");
+#pragma unroll
+  for (int i = 0; i < N / 32; ++i) tmem_reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&r[32 * i]));
+}
+template <int N>
+__device__ __forceinline__ void tmem_reg_fence(float (&r)[N]) {
+  tmem_reg_fence(*reinterpret_cast<uint32_t(*)[N]>(&r[0]));
+}
+// Waits for this thread's outstanding tcgen05.ld and fences the arrays they were loaded into.
+template <typename... Arrays>
+__device__ __forceinline__ void tmem_wait_ld(Arrays&... loaded) {
+  static_assert(sizeof...(Arrays) > 0, "name the registers the loads wrote");
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  (tmem_reg_fence(loaded), ...);
 }
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
