@@ -102,6 +102,34 @@ int mfa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
             int causal, int win_l, int win_r, float softcap, int dtype, void* stream);
 
 /*
+ * mfa_fwd_host -- mfa_fwd with q, k, v, out and lse in HOST memory, for callers whose tensors
+ * live on the host (the same operation as "mlx-mfa 2.5.2" Usage, flash_attention(q, k, v,
+ * causal=...), whose arrays sit in memory the host and GPU share; here the copies to and from
+ * the device are part of the call).
+ *
+ * q, k, v, out: host buffers, layouts as mfa_fwd; lse: host float buffer [B, Hq, Nq] or NULL.
+ * Page-locked (pinned) host memory lets the copies run asynchronously; pageable memory works but
+ * each copy then blocks the calling thread until it is done.
+ * scratch: device buffer of at least mfa_fwd_host_scratch_size(...) bytes, 256-byte aligned,
+ * owned by the caller; it holds the device copies of all five tensors.
+ * The B * Hkv (batch, kv head) units are split into contiguous runs of about 12 MiB of input
+ * each (at most 8; one for small problems). Run c's inputs are
+ * copied in on an internal stream while run c - 1 computes on `stream` and run c - 2's outputs
+ * are copied out on a second internal stream; the internal streams are ordered after the work
+ * queued on `stream` before the call, and `stream` is ordered after the last copy out. The call
+ * returns once everything is queued: out and lse are complete when `stream` reaches this point
+ * (synchronize it, or record an event, before reading them). Results are bitwise those of
+ * mfa_fwd on the same data. Argument checks and error codes as mfa_fwd, plus MFA_ERR_WORKSPACE
+ * for a NULL, misaligned or too small scratch. Concurrent calls from several host threads on one
+ * device are serialised by the library while they queue their work.
+ */
+size_t mfa_fwd_host_scratch_size(int B, int Hq, int Hkv, int Nq, int Nk, int D);
+int mfa_fwd_host(const void* q, const void* k, const void* v, void* out, float* lse,
+                 int B, int Hq, int Hkv, int Nq, int Nk, int D, float scale,
+                 int causal, int win_l, int win_r, float softcap, int dtype,
+                 void* scratch, size_t scratch_bytes, void* stream);
+
+/*
  * mfa_fwd_varlen -- the same forward over a packed batch of variable-length sequences
  * ([MFA252] Features "Variable-length -- packed sequences with cu_seqlens"; [MXFA15] README
  * public entry point flash_attn_varlen_func; [MFA261] 2.61.0 notes that varlen causal with

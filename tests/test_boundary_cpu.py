@@ -190,3 +190,40 @@ def test_decode_workspace_size_is_shape_only():
 def test_debug_flags_roundtrip():
     old = mfa.mfa_debug_set_flags(3)
     assert mfa.mfa_debug_set_flags(old) == 3
+
+
+def fwdh(**kw):
+    ws = kw.pop("ws_bytes", 1 << 30)
+    args = dict(q=A, k=A, v=A, out=A, lse=A, B=2, Hq=8, Hkv=2, Nq=64, Nk=64, D=128, scale=0.125,
+                causal=1, win_l=-1, win_r=-1, softcap=0.0, dtype=1, ws=A, ws_bytes=ws, stream=None)
+    args.update(kw)
+    return mfa.lib.mfa_fwd_host(*args.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=7), -3), (dict(D=96), -4), (dict(B=-1), -5), (dict(Hkv=3), -6),
+    (dict(win_l=-3), -7), (dict(softcap=-1.0), -8), (dict(scale=0.0), -9),
+    (dict(q=None), -1), (dict(k=None), -1), (dict(out=None), -1),
+    (dict(ws=None), -12), (dict(ws=A + 128), -12), (dict(ws_bytes=4096), -12),
+])
+@no_device
+def test_fwd_host_rejects_malformed(kw, code):
+    assert fwdh(**kw) == code
+
+
+def test_fwd_host_scratch_size():
+    """Device copies of q, k, v, out and lse, each region rounded up to 256 bytes."""
+    r = lambda x: (x + 255) // 256 * 256
+    B, Hq, Hkv, Nq, Nk, D = 2, 8, 2, 100, 300, 64
+    q = B * Hq * Nq * D * 2
+    kv = B * Hkv * Nk * D * 2
+    lse = B * Hq * Nq * 4
+    assert mfa.mfa_fwd_host_scratch_size(B, Hq, Hkv, Nq, Nk, D) == 2 * r(q) + 2 * r(kv) + r(lse)
+    assert mfa.mfa_fwd_host_scratch_size(B, Hq, 3, Nq, Nk, D) == 0
+    assert mfa.mfa_fwd_host_scratch_size(B, Hq, Hkv, Nq, Nk, 96) == 0
+    assert mfa.mfa_fwd_host_scratch_size(0, Hq, Hkv, Nq, Nk, D) == 0 + 0 + 0
+
+
+@no_device
+def test_fwd_host_empty_problem_is_a_no_op():
+    assert fwdh(B=0, q=None, k=None, v=None, out=None, lse=None, ws=None) == 0

@@ -50,6 +50,10 @@ lib.mfa_decode_splitkv.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i
 lib.mfa_decode_splitkv_window.restype = _i
 lib.mfa_decode_splitkv_window.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                           _i, _i, _f, _i, _i, _f, _i, _vp, ctypes.c_size_t, _vp]
+lib.mfa_fwd_host_scratch_size.restype = ctypes.c_size_t
+lib.mfa_fwd_host_scratch_size.argtypes = [_i] * 6
+lib.mfa_fwd_host.restype = _i
+lib.mfa_fwd_host.argtypes = [_vp] * 5 + [_i] * 6 + [_f, _i, _i, _i, _f, _i, _vp, ctypes.c_size_t, _vp]
 lib.mfa_decode_splitkv_noalloc.restype = _i
 lib.mfa_decode_splitkv_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                            _i, _i, _f, _i, _f, _i, _vp]
@@ -82,7 +86,7 @@ EXPORTED = ("mfa_fwd", "mfa_fwd_varlen", "mfa_fwd_blocksparse", "mfa_fwd_paged",
             "mfa_decode_workspace_size", "mfa_decode_splitkv_window", "mfa_decode_splitkv", "mfa_status_string",
             "mfa_last_launch_info", "mfa_device_status", "mfa_debug_set_flags",
             "mfa_debug_tiles_visited", "mfa_debug_set_decode_split_pages",
-            "mfa_decode_splitkv_noalloc")
+            "mfa_decode_splitkv_noalloc", "mfa_fwd_host_scratch_size", "mfa_fwd_host")
 
 
 class MFAError(RuntimeError):
@@ -151,6 +155,52 @@ def mfa_fwd(q, k, v, out=None, lse=None, *, scale=None, causal=False, window=(-1
                      float(scale), int(bool(causal)), int(wl), int(wr), float(softcap),
                      _dtype_code(q), _stream(stream))
     _check(rc, "mfa_fwd")
+    return out, lse
+
+
+def _host_ptr(t):
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError("mfa_fwd_host takes host (CPU) tensors")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def mfa_fwd_host_scratch_size(B, Hq, Hkv, Nq, Nk, D) -> int:
+    return int(lib.mfa_fwd_host_scratch_size(B, Hq, Hkv, Nq, Nk, D))
+
+
+def mfa_fwd_host(q, k, v, out=None, lse=None, *, scale=None, causal=False, window=(-1, -1),
+                 softcap=0.0, scratch=None, return_lse=True, stream=None):
+    """Attention forward over HOST tensors (pinned memory lets the copies overlap): q
+    [B,Hq,Nq,D], k/v [B,Hkv,Nk,D] on the CPU; the copies to and from the device and the kernels
+    are queued on `stream` and two internal copy streams. Returns (out, lse or None) as CPU
+    tensors, complete once `stream` has reached this point (synchronize before reading them).
+    scratch: a CUDA uint8 tensor of mfa_fwd_host_scratch_size(...) bytes (allocated if None)."""
+    torch = _torch()
+    B, Hq, Nq, D = q.shape
+    _, Hkv, Nk, _ = k.shape
+    if k.shape != v.shape or k.shape[0] != B or k.shape[3] != D:
+        raise ValueError("k and v must be [B, Hkv, Nk, D] matching q")
+    if q.dtype != k.dtype or q.dtype != v.dtype:
+        raise TypeError("q, k and v must share one dtype")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32).pin_memory()
+    if scratch is None:
+        n = mfa_fwd_host_scratch_size(B, Hq, Hkv, Nq, Nk, D)
+        scratch = torch.empty(max(n, 256), dtype=torch.uint8, device="cuda")
+    wl, wr = window
+    rc = lib.mfa_fwd_host(_host_ptr(q), _host_ptr(k), _host_ptr(v), _host_ptr(out), _host_ptr(lse),
+                          B, Hq, Hkv, Nq, Nk, D, float(scale), int(bool(causal)), int(wl), int(wr),
+                          float(softcap), _dtype_code(q), _ptr(scratch),
+                          scratch.numel() * scratch.element_size(), _stream(stream))
+    _check(rc, "mfa_fwd_host")
     return out, lse
 
 

@@ -808,3 +808,128 @@ extern "C" int mfa_decode_splitkv_noalloc(const void* q, const void* k_pages, co
                             D, page_size, max_pages_per_seq, num_pages, scale, causal, softcap,
                             dtype, scratch, kNoAllocScratchBytes, stream);
 }
+
+// ----------------------------------------------------------------------------------------------
+// Forward over host buffers: the batch x kv-head units are cut into up to kHostChunks contiguous
+// runs of about 12 MiB of input each; run c's inputs are copied in on an internal stream while
+// run c - 1 computes on the caller's stream and run c - 2's outputs are copied out on a second
+// internal stream, so the PCIe copies in the two directions and the kernels overlap. Each run of units [u0, u1) is the
+// forward problem B' = u1 - u0, Hq' = Hq / Hkv, Hkv' = 1 over the same memory layout.
+namespace {
+
+constexpr int kHostChunks = 8;
+
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t entry = nullptr, done = nullptr;
+  cudaEvent_t in_done[kHostChunks] = {}, comp_done[kHostChunks] = {};
+};
+HostPipe g_host_pipe[kMaxDevices];
+std::mutex g_host_mutex[kMaxDevices];
+
+bool host_pipe_init(HostPipe& hp) {
+  if (hp.ready) return true;
+  const unsigned ev = cudaEventDisableTiming;
+  if (cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) != cudaSuccess) return false;
+  if (cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) != cudaSuccess) return false;
+  if (cudaEventCreateWithFlags(&hp.entry, ev) != cudaSuccess) return false;
+  if (cudaEventCreateWithFlags(&hp.done, ev) != cudaSuccess) return false;
+  for (int c = 0; c < kHostChunks; ++c) {
+    if (cudaEventCreateWithFlags(&hp.in_done[c], ev) != cudaSuccess) return false;
+    if (cudaEventCreateWithFlags(&hp.comp_done[c], ev) != cudaSuccess) return false;
+  }
+  hp.ready = true;
+  return true;
+}
+
+struct HostLayout {
+  size_t q_bytes, kv_bytes, lse_bytes;
+  size_t off_k, off_v, off_out, off_lse, total;
+};
+HostLayout host_layout(int B, int Hq, int Hkv, int Nq, int Nk, int D) {
+  HostLayout L;
+  L.q_bytes = (size_t)B * Hq * Nq * D * 2;
+  L.kv_bytes = (size_t)B * Hkv * Nk * D * 2;
+  L.lse_bytes = (size_t)B * Hq * Nq * sizeof(float);
+  L.off_k = align256(L.q_bytes);
+  L.off_v = L.off_k + align256(L.kv_bytes);
+  L.off_out = L.off_v + align256(L.kv_bytes);
+  L.off_lse = L.off_out + align256(L.q_bytes);
+  L.total = L.off_lse + align256(L.lse_bytes);
+  return L;
+}
+
+}  // namespace
+
+extern "C" size_t mfa_fwd_host_scratch_size(int B, int Hq, int Hkv, int Nq, int Nk, int D) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || Nq < 0 || Nk < 0 || Hq % Hkv != 0) return 0;
+  if (D != 64 && D != 128) return 0;
+  if (check_sizes(B, Hq, Nq, D) != MFA_OK || check_sizes(B, Hkv, Nk, D) != MFA_OK) return 0;
+  return host_layout(B, Hq, Hkv, Nq, Nk, D).total;
+}
+
+extern "C" int mfa_fwd_host(const void* q, const void* k, const void* v, void* out, float* lse,
+                            int B, int Hq, int Hkv, int Nq, int Nk, int D, float scale, int causal,
+                            int win_l, int win_r, float softcap, int dtype, void* scratch,
+                            size_t scratch_bytes, void* stream) {
+  int rc = validate_fwd_common(Hq, Hkv, D, dtype, win_l, win_r, softcap, scale);
+  if (rc != MFA_OK) return rc;
+  if (B < 0 || Nq < 0 || Nk < 0) return MFA_ERR_BAD_SHAPE;
+  if ((rc = check_sizes(B, Hq, Nq, D)) != MFA_OK) return rc;
+  if ((rc = check_sizes(B, Hkv, Nk, D)) != MFA_OK) return rc;
+  if ((long long)B * Hq > 0x7FFFFFFFLL || (long long)B * Hkv > 0x7FFFFFFFLL) return MFA_ERR_BAD_SHAPE;
+  if (B == 0 || Hq == 0 || Nq == 0) return MFA_OK;
+  if (!q || !out || (Nk > 0 && (!k || !v))) return MFA_ERR_NULL_POINTER;
+  const HostLayout L = host_layout(B, Hq, Hkv, Nq, Nk, D);
+  if (!scratch || (reinterpret_cast<uintptr_t>(scratch) & 255u) || scratch_bytes < L.total)
+    return MFA_ERR_WORKSPACE;
+  const int dev = current_device();
+  if (dev < 0) return MFA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_host_mutex[dev]);
+  HostPipe& hp = g_host_pipe[dev];
+  if (!host_pipe_init(hp)) return MFA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* s = static_cast<char*>(scratch);
+  const int G = Hq / Hkv;
+  const long long units = (long long)B * Hkv;
+  // runs of about 12 MiB of input each (at most kHostChunks): every copy has a fixed cost, and
+  // the last run's kernel and copy out are not hidden, so a few large runs beat many small ones
+  const long long in_bytes = (long long)(L.q_bytes + 2 * L.kv_bytes);
+  const int n_chunks = (int)std::max<long long>(
+      1, std::min<long long>(units, std::min<long long>(kHostChunks, in_bytes / (12ll << 20))));
+  const size_t q_unit = (size_t)G * Nq * D * 2, kv_unit = (size_t)Nk * D * 2;
+  const size_t l_unit = (size_t)G * Nq * sizeof(float);
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+  // earlier work on the caller's stream (which may still use the scratch) precedes the copies in
+  if (!ok(cudaEventRecord(hp.entry, st)) || !ok(cudaStreamWaitEvent(hp.in, hp.entry, 0))) return MFA_ERR_CUDA;
+  rc = MFA_OK;
+  for (int c = 0; c < n_chunks && rc == MFA_OK; ++c) {
+    const long long u0 = units * c / n_chunks, u1 = units * (c + 1) / n_chunks;
+    const size_t n = (size_t)(u1 - u0);
+    const size_t oq = (size_t)u0 * q_unit, okv = (size_t)u0 * kv_unit, ol = (size_t)u0 * l_unit;
+    if (!ok(cudaMemcpyAsync(s + oq, static_cast<const char*>(q) + oq, n * q_unit,
+                            cudaMemcpyHostToDevice, hp.in)) ||
+        (Nk > 0 && !ok(cudaMemcpyAsync(s + L.off_k + okv, static_cast<const char*>(k) + okv,
+                                       n * kv_unit, cudaMemcpyHostToDevice, hp.in))) ||
+        (Nk > 0 && !ok(cudaMemcpyAsync(s + L.off_v + okv, static_cast<const char*>(v) + okv,
+                                       n * kv_unit, cudaMemcpyHostToDevice, hp.in))) ||
+        !ok(cudaEventRecord(hp.in_done[c], hp.in)) || !ok(cudaStreamWaitEvent(st, hp.in_done[c], 0))) {
+      rc = MFA_ERR_CUDA;
+      break;
+    }
+    rc = mfa_fwd(s + oq, s + L.off_k + okv, s + L.off_v + okv, s + L.off_out + oq,
+                 lse ? reinterpret_cast<float*>(s + L.off_lse + ol) : nullptr, (int)n, G, 1, Nq, Nk,
+                 D, scale, causal, win_l, win_r, softcap, dtype, stream);
+    if (rc != MFA_OK) break;
+    if (!ok(cudaEventRecord(hp.comp_done[c], st)) || !ok(cudaStreamWaitEvent(hp.out, hp.comp_done[c], 0)) ||
+        !ok(cudaMemcpyAsync(static_cast<char*>(out) + oq, s + L.off_out + oq, n * q_unit,
+                            cudaMemcpyDeviceToHost, hp.out)) ||
+        (lse && !ok(cudaMemcpyAsync(reinterpret_cast<char*>(lse) + ol, s + L.off_lse + ol, n * l_unit,
+                                    cudaMemcpyDeviceToHost, hp.out))))
+      rc = MFA_ERR_CUDA;
+  }
+  // the caller's stream (and so the next call) continues after the last copy out, also on error
+  if (!ok(cudaEventRecord(hp.done, hp.out)) || !ok(cudaStreamWaitEvent(st, hp.done, 0))) return MFA_ERR_CUDA;
+  return rc;
+}
