@@ -293,6 +293,16 @@ def bench_prefill(case, steps, warmup, flush, stream, with_e2e, world):
         if not (torch.equal(ho, out.cpu()) and torch.equal(hl, lse.cpu())):
             raise RuntimeError("host-buffer forward differs from the device forward")
         res["e2e_ms"] = max_over_ranks(statistics.mean(ems), world)
+        # the PCIe floor on this machine, same run: the step's inputs copied in alone
+        flat_h = torch.cat([hq.view(-1), hk.view(-1), hv.view(-1)]).pin_memory()
+        flat_d = torch.empty_like(flat_h, device=dev)
+
+        def h2d_only():
+            flat_d.copy_(flat_h, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            hms, _ = time_steps(h2d_only, 5, 2, flush, stream)
+        res["h2d_alone_ms"] = statistics.mean(hms)
         res["h2d"] = int(q.nbytes + k.nbytes + v.nbytes)
         res["d2h"] = int(ho.numel() * 2 + hl.numel() * 4)
     return res
@@ -558,6 +568,7 @@ def run_gpu(args):
         line["e2e"] = {"value": round(main["flops"] * world / (main["e2e_ms"] * 1e-3) / 1e12, 3),
                        "unit": "TFLOP/s", "ms_per_step": round(main["e2e_ms"], 4),
                        "h2d_bytes_per_step": main["h2d"], "d2h_bytes_per_step": main["d2h"],
+                       "h2d_alone_ms": round(main["h2d_alone_ms"], 4),
                        "call": "mfa_fwd_host (C ABI, pinned host buffers; copies in / kernels / "
                                "copies out pipelined over runs of about 12 MiB of (batch, kv-head) units)"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
