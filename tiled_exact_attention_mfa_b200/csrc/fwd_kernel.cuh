@@ -23,10 +23,10 @@
 //                 P_t (16-bit, 2 per column) overwrites the first 64 columns of S_t.
 // Ordering: QK for tile j+1 of Q tile t overwrites S_t's columns, where PV for tile j reads P_t
 // from. tcgen05 only orders MMAs that share an accumulator, so the MMA thread waits for that PV
-// to complete before issuing the QK (kQKBehindPV = 0; issuing it right behind the PV and relying
-// on in-order execution measured ~2 % faster and is not used). The commit that signals S_t
-// ready covers every earlier MMA, so when the softmax of tile j+1 starts, PV of tile j is done
-// and O_t can be rescaled in place.
+// to complete before issuing the QK (issuing it right behind the PV would rely on an execution
+// order the rules do not give; it measured ~2 % faster and is not built). The commit that
+// signals S_t ready covers every earlier MMA, so when the softmax of tile j+1 starts, PV of tile
+// j is done and O_t can be rescaled in place.
 //
 // Tile skip ("mlx-mfa 2.5.2", Features: causal tile-skip, window_size=(left,right) tile skip):
 // each CTA visits only key tiles that intersect the union of its rows' visible ranges; inside,
@@ -41,10 +41,6 @@ constexpr int kFwdBN = 128;       // keys per K/V tile
 constexpr int kFwdQT = 2;         // Q tiles per CTA
 constexpr int kFwdStages = 2;     // K ring and V ring depth
 constexpr int kFwdThreads = 384;  // 8 softmax warps + producer + MMA + 2 idle
-#ifndef MFA_QK_BEHIND_PV
-#define MFA_QK_BEHIND_PV 0
-#endif
-constexpr bool kQKBehindPV = MFA_QK_BEHIND_PV != 0;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kFwdMaxSparseTiles = 2048;  // key tiles a block-sparse row may span (262,144 keys)
 #ifndef MFA_POLY_MASK
@@ -387,7 +383,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         tc_commit(smem_u32(&sm.bar_o_done[0]));
         if (more) {
           if (!(ok = mbar_wait(smem_u32(&sm.bar_k_full[s1]), ph1, abort, 905))) break;
-          if (!kQKBehindPV && !(ok = mbar_wait(smem_u32(&sm.bar_o_done[0]), j & 1, abort, 906))) break;
+          if (!(ok = mbar_wait(smem_u32(&sm.bar_o_done[0]), j & 1, abort, 906))) break;
           tc_fence_after();
           issue_qk(0, s1);
           tc_commit(smem_u32(&sm.bar_s_full[0]));
@@ -402,7 +398,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         tc_commit(smem_u32(&sm.bar_o_done[1]));
         tc_commit(smem_u32(&sm.bar_v_empty[s]));
         if (more) {
-          if (!kQKBehindPV && !(ok = mbar_wait(smem_u32(&sm.bar_o_done[1]), j & 1, abort, 908))) break;
+          if (!(ok = mbar_wait(smem_u32(&sm.bar_o_done[1]), j & 1, abort, 908))) break;
           tc_fence_after();
           issue_qk(1, s1);
           tc_commit(smem_u32(&sm.bar_s_full[1]));
