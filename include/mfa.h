@@ -329,10 +329,15 @@ int mfa_device_status(void* stream, int* code, int* detail);
 /*
  * Debug switches (process-wide; default 0). Bit 0: the forward visits every key tile and masks
  * element-wise instead of skipping tiles. Bit 1: count the key tiles each forward CTA visits
- * into a device counter read by mfa_debug_tiles_visited. Returns the previous flags.
+ * into a device counter read by mfa_debug_tiles_visited. Bit 2: the forward's MMA thread issues
+ * nothing, so the softmax warps' first bounded wait runs out after 2 s; the kernel then records
+ * MFA_ERR_DEVICE_TIMEOUT in the device status, writes out = 0 and lse = -inf, releases TMEM and
+ * returns, leaving the context usable (for tests of the failure path). Returns the previous
+ * flags.
  */
 #define MFA_DEBUG_NO_TILE_SKIP 1
 #define MFA_DEBUG_COUNT_TILES  2
+#define MFA_DEBUG_WITHHOLD_MMA 4
 int mfa_debug_set_flags(int flags);
 
 /* Reads and resets the tile counter (synchronises `stream`). */

@@ -25,6 +25,7 @@ MFA_DTYPE_FP16 = 0
 MFA_DTYPE_BF16 = 1
 MFA_DEBUG_NO_TILE_SKIP = 1
 MFA_DEBUG_COUNT_TILES = 2
+MFA_DEBUG_WITHHOLD_MMA = 4
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int

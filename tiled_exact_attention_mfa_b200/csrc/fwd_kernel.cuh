@@ -72,7 +72,7 @@ struct FwdParams {
   int B, Hq, Hkv, Nq, Nk, G;
   int causal, win_l, win_r;
   int n_qblk;       // number of 256-row query blocks per head
-  int flags;        // bit 0: no tile skip; bit 1: count tiles
+  int flags;        // bit 0: no tile skip; bit 1: count tiles; bit 2: withhold every MMA
   float c_log2;     // factor taking the stored score to the log2 domain
   float softcap;    // 0 = off
   float cap_in;     // scale / softcap
@@ -356,7 +356,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
                     (acc || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(smem_u32(&sm.bar_q), 0, abort, 901);
+      // Debug flag bit 2 (failure-detection tests): issue no MMA at all, so the softmax warps'
+      // first wait for S runs out; the bounded waits then take the abort path below.
+      const bool withhold = (p.flags & 4) != 0;
+      bool ok = !withhold && mbar_wait(smem_u32(&sm.bar_q), 0, abort, 901);
       for (int j = 0; ok && j < n_act; ++j) {  // j counts visited tiles
         const int s = j % kFwdStages;
         const uint32_t ph = (j / kFwdStages) & 1;
