@@ -86,25 +86,28 @@ def test_all_ones_mask_is_bitwise_the_dense_forward(cuda_device):
 
 
 def tiles_closed_form(case, m, bm=256, bn=128):
-    """Key tiles a 256-row block visits: within the causal / window range of its rows, and on
-    for at least one of its two 128-row mask rows."""
+    """Key tiles a 256-row block visits: those that one of its two 128-row Q tiles both has on in
+    the mask and can see with some of its rows (causal / window)."""
     vis = oracle.visible(case.Nq, case.Nk, case.causal, case.win_l, case.win_r)
     n = 0
     for b in range(case.B):
         for h in range(case.Hq):
             for r0 in range(0, case.Nq, bm):
-                cols = vis[r0:r0 + bm].any(axis=0)
-                tiles = sorted({j // bn for j in np.nonzero(cols)[0]})
-                if not tiles:
-                    continue
-                rows = [r0 // 128 + t for t in range(2) if r0 + 128 * t < case.Nq]
-                n += sum(1 for j in range(tiles[0], tiles[-1] + 1) if any(m[b, h, r, j] for r in rows))
+                visited = set()
+                for t in range(bm // 128):
+                    rs = r0 + 128 * t
+                    if rs >= case.Nq:
+                        continue
+                    cols = vis[rs:rs + 128].any(axis=0)
+                    visited |= {j // bn for j in np.nonzero(cols)[0] if m[b, h, rs // 128, j // bn]}
+                n += len(visited)
     return n
 
 
 def test_visited_tiles_and_tile_skip_neutrality(cuda_device):
     """The visited-tile counter equals the closed form, and visiting every key tile of the mask
-    (no causal / window skip) gives bitwise the same outputs."""
+    (no causal / window skip: each Q tile then also takes part in tiles its rows cannot see,
+    which contribute exact zeros) gives bitwise the same outputs."""
     import tiled_exact_attention_mfa_b200 as mfa
     case = S("cnt", 1, 2, 2, 1100, 64, mi.FP16, True, density=0.4, win_l=300, win_r=0, seed=68)
     q, k, v, m = case.tensors()

@@ -119,7 +119,9 @@ __device__ __forceinline__ void key_range(const FwdParams& p, int Nk, int a0, in
 // (cu_q, cu_k), read through tensor maps ordered (D, head, token); lse is [Hq, total_q]. Otherwise q / out are [B, Hq, Nq, D], k / v
 // [B, Hkv, Nk, D] and lse [B, Hq, Nq].
 // SPARSE: dense layout plus a block mask; a CTA visits only key tiles whose block is on for one
-// of its Q tiles, and a Q tile whose block is off on a visited tile masks it entirely.
+// of its Q tiles and which that Q tile's rows can see (causal / window); a Q tile takes no part
+// (no MMA, no softmax) in a visited tile that is not its own, and its barriers count only the
+// tiles it takes part in.
 // SOFTCAP: compiled with the softcap transform (p.softcap > 0); without it the softmax carries
 // no softcap code at all.
 // PAGED (with VARLEN queries): K / V tiles are assembled from 16-token pages through the block
@@ -211,14 +213,30 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     const int qt0 = q0 / kFwdBM;
     const uint8_t* r0 = p.block_mask + ((size_t)(b * p.Hq + h) * p.nqt + qt0) * p.nkt + kt_lo;
     const uint8_t* r1 = (qt0 + 1 < p.nqt) ? r0 + p.nkt : nullptr;
+    // each Q tile's own visible key range: a tile it cannot see at all is not its to visit
+    int vlo[kFwdQT], vhi[kFwdQT];
+#pragma unroll
+    for (int t = 0; t < kFwdQT; ++t) {
+      const int f = q0 + t * kFwdBM, l = min(f + kFwdBM, Nq) - 1;
+      if (l < f) {
+        vlo[t] = 1;
+        vhi[t] = 0;
+      } else if (p.flags & 1) {
+        vlo[t] = 0;
+        vhi[t] = Nk;
+      } else {
+        key_range(p, Nk, f + off, l + off, vlo[t], vhi[t]);
+      }
+    }
     int count = 0;
     for (int base = 0; base < n_tiles; base += 32 * 8) {
       uint8_t a0[8], a1[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int jj = base + i * 32 + lane;
-        a0[i] = jj < n_tiles ? r0[jj] : 0;
-        a1[i] = (r1 != nullptr && jj < n_tiles) ? r1[jj] : 0;
+        const int k0 = (kt_lo + jj) * kFwdBN;
+        a0[i] = (jj < n_tiles && k0 < vhi[0] && k0 + kFwdBN > vlo[0]) ? r0[jj] : 0;
+        a1[i] = (r1 != nullptr && jj < n_tiles && k0 < vhi[1] && k0 + kFwdBN > vlo[1]) ? r1[jj] : 0;
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -360,6 +378,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       // first wait for S runs out; the bounded waits then take the abort path below.
       const bool withhold = (p.flags & 4) != 0;
       bool ok = !withhold && mbar_wait(smem_u32(&sm.bar_q), 0, abort, 901);
+      // Block-sparse: Q tile t takes part in visited tile u only where its bit is on; its MMAs
+      // are skipped elsewhere and its barriers count only the tiles it takes part in. (Dense:
+      // every Q tile takes part in every tile, and the counts below are the loop index.)
+      auto act = [&](int u, int t) -> bool {
+        if constexpr (SPARSE) return ((sm.act_bits[u] >> t) & 1) != 0; else return true;
+      };
+      int npv[kFwdQT] = {0, 0};  // PV groups issued per Q tile (SPARSE only)
       for (int j = 0; ok && j < n_act; ++j) {  // j counts visited tiles
         const int s = j % kFwdStages;
         const uint32_t ph = (j / kFwdStages) & 1;
@@ -369,42 +394,61 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         if (j == 0) {
           if (!(ok = mbar_wait(smem_u32(&sm.bar_k_full[s]), ph, abort, 902))) break;
           tc_fence_after();
-          issue_qk(0, s);
-          tc_commit(smem_u32(&sm.bar_s_full[0]));
-          issue_qk(1, s);
-          tc_commit(smem_u32(&sm.bar_s_full[1]));
+          if (act(0, 0)) {
+            issue_qk(0, s);
+            tc_commit(smem_u32(&sm.bar_s_full[0]));
+          }
+          if (act(0, 1)) {
+            issue_qk(1, s);
+            tc_commit(smem_u32(&sm.bar_s_full[1]));
+          }
           tc_commit(smem_u32(&sm.bar_k_empty[s]));
         }
         // Q tile 0: PV(j), then QK(j+1) once PV(j) is done (P_0 lives in S_0's columns)
         if (!(ok = mbar_wait(smem_u32(&sm.bar_v_full[s]), ph, abort, 903))) break;
-        if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[0][0]), j & 1, abort, 904))) break;
-        tc_fence_after();
-        issue_pv(0, s, j > 0, 0);
-        if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[0][1]), j & 1, abort, 914))) break;
-        tc_fence_after();
-        issue_pv(0, s, true, 1);
-        tc_commit(smem_u32(&sm.bar_o_done[0]));
+        if (act(j, 0)) {
+          const int c = SPARSE ? npv[0] : j;
+          if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[0][0]), c & 1, abort, 904))) break;
+          tc_fence_after();
+          issue_pv(0, s, c > 0, 0);
+          if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[0][1]), c & 1, abort, 914))) break;
+          tc_fence_after();
+          issue_pv(0, s, true, 1);
+          tc_commit(smem_u32(&sm.bar_o_done[0]));
+          ++npv[0];
+        }
         if (more) {
           if (!(ok = mbar_wait(smem_u32(&sm.bar_k_full[s1]), ph1, abort, 905))) break;
-          if (!(ok = mbar_wait(smem_u32(&sm.bar_o_done[0]), j & 1, abort, 906))) break;
-          tc_fence_after();
-          issue_qk(0, s1);
-          tc_commit(smem_u32(&sm.bar_s_full[0]));
+          if (act(j + 1, 0)) {
+            // the latest PV of Q tile 0 read P_0 from S_0's columns
+            if (!SPARSE || npv[0] > 0)
+              if (!(ok = mbar_wait(smem_u32(&sm.bar_o_done[0]), (SPARSE ? npv[0] - 1 : j) & 1, abort, 906))) break;
+            tc_fence_after();
+            issue_qk(0, s1);
+            tc_commit(smem_u32(&sm.bar_s_full[0]));
+          }
         }
         // Q tile 1
-        if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[1][0]), j & 1, abort, 907))) break;
-        tc_fence_after();
-        issue_pv(1, s, j > 0, 0);
-        if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[1][1]), j & 1, abort, 917))) break;
-        tc_fence_after();
-        issue_pv(1, s, true, 1);
-        tc_commit(smem_u32(&sm.bar_o_done[1]));
+        if (act(j, 1)) {
+          const int c = SPARSE ? npv[1] : j;
+          if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[1][0]), c & 1, abort, 907))) break;
+          tc_fence_after();
+          issue_pv(1, s, c > 0, 0);
+          if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[1][1]), c & 1, abort, 917))) break;
+          tc_fence_after();
+          issue_pv(1, s, true, 1);
+          tc_commit(smem_u32(&sm.bar_o_done[1]));
+          ++npv[1];
+        }
         tc_commit(smem_u32(&sm.bar_v_empty[s]));
         if (more) {
-          if (!(ok = mbar_wait(smem_u32(&sm.bar_o_done[1]), j & 1, abort, 908))) break;
-          tc_fence_after();
-          issue_qk(1, s1);
-          tc_commit(smem_u32(&sm.bar_s_full[1]));
+          if (act(j + 1, 1)) {
+            if (!SPARSE || npv[1] > 0)
+              if (!(ok = mbar_wait(smem_u32(&sm.bar_o_done[1]), (SPARSE ? npv[1] - 1 : j) & 1, abort, 908))) break;
+            tc_fence_after();
+            issue_qk(1, s1);
+            tc_commit(smem_u32(&sm.bar_s_full[1]));
+          }
           tc_commit(smem_u32(&sm.bar_k_empty[s1]));
         }
       }
@@ -431,8 +475,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     float m_run = -INFINITY;  // running max of the stored (scaled, capped) score
     float l_run = 0.f;
 
+    int nt = 0;  // tiles this Q tile took part in (block-sparse: its bit on); dense: nt == j
     for (int j = 0; j < n_act; ++j) {  // j counts visited tiles
-      const bool got = mbar_wait(smem_u32(&sm.bar_s_full[t]), j & 1, abort, 1001 + t);
+      if constexpr (SPARSE) {
+        if (!((sm.act_bits[j] >> t) & 1)) continue;  // not this Q tile's: no S, no P for it
+      }
+      const int c_t = SPARSE ? nt : j;
+      const bool got = mbar_wait(smem_u32(&sm.bar_s_full[t]), c_t & 1, abort, 1001 + t);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       uint32_t sraw[128];
@@ -444,8 +493,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       float* s = reinterpret_cast<float*>(sraw);
 
       const int k0 = (kt_lo + tile_of(j)) * kFwdBN;
-      // block-sparse: this Q tile's block is off on a tile visited for the other Q tile
-      const bool off_block = SPARSE && !((sm.act_bits[SPARSE ? j : 0] >> t) & 1);
       // Softcap: the capped score is cap * tanh(s * scale / cap); the value kept per key is that
       // divided by scale, so the exponent factor c = scale * log2 e is the same as without a cap.
       // When every |y| = |s| * scale / cap of this warp's rows is small, tanh(y) = y * q(y^2) is
@@ -476,12 +523,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       if (p.win_r >= 0) interior = interior && (k0 + kFwdBN - 1 <= a_lo + p.win_r);
       if (p.win_l >= 0) interior = interior && (k0 >= a_hi - p.win_l);
       if (p.flags & 1) interior = false;
-      if (off_block) interior = false;
       if (!interior) {
         int jhi = Nk - k0;                                     // keys >= Nk
         if (p.causal) jhi = min(jhi, a - k0 + 1);
         if (p.win_r >= 0) jhi = min(jhi, a + p.win_r - k0 + 1);
-        if (off_block) jhi = 0;
         const int jlo = (p.win_l >= 0) ? (a - p.win_l - k0) : -1;
 #pragma unroll
         for (int i = 0; i < 128; ++i) s[i] = (i < jhi && i >= jlo) ? s[i] : -INFINITY;
@@ -515,7 +560,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
 
       // O rescale before any PV of this tile reads P (only after the first tile: before it O
       // holds nothing). The previous PV of this Q tile has completed: its commit preceded S.
-      if (warp_rescale && j > 0) {
+      if (warp_rescale && c_t > 0) {
 #pragma unroll
         for (int cb = 0; cb < D; cb += 32) {
           uint32_t o[32];
@@ -606,13 +651,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       float sa, sb;
       f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), sa, sb);
       l_run = l_run * alpha + (sa + sb);
-
+      ++nt;
     }
 
     // ---- epilogue: O / l, LSE
     bool have_o = false;
-    if (n_act > 0 && !*abort) {
-      have_o = mbar_wait(smem_u32(&sm.bar_o_done[t]), (n_act - 1) & 1, abort, 1003 + t);
+    const int n_t = SPARSE ? nt : n_act;  // PV groups of this Q tile
+    if (n_t > 0 && !*abort) {
+      have_o = mbar_wait(smem_u32(&sm.bar_o_done[t]), (n_t - 1) & 1, abort, 1003 + t);
       tc_fence_after();
     }
     have_o = __all_sync(0xffffffffu, have_o);
