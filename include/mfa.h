@@ -73,6 +73,7 @@ extern "C" {
 #define MFA_ERR_SCRATCH_TOO_SMALL  -23   /* mfa_decode_splitkv_noalloc: shape needs more than its fixed scratch */
 #define MFA_ERR_DEVICE_BAD_SEQLENS -24   /* device status: a cu_seqlens entry was negative, decreasing or past
                                             the packed total, or a sequence was longer than max_seqlen_q */
+#define MFA_ERR_DEVICE_TILE_LIST   -25   /* device status: a key-tile list exceeded its capacity (a host check failed) */
 
 /*
  * mfa_fwd -- exact attention forward (prefill).

@@ -244,13 +244,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         const unsigned bal = __ballot_sync(0xffffffffu, act);
         if (act) {
           const int pos = count + __popc(bal & ((1u << lane) - 1u));
-          sm.act_tile[pos] = (uint16_t)(base + i * 32 + lane);
-          sm.act_bits[pos] = (uint8_t)((a0[i] != 0 ? 1 : 0) | (a1[i] != 0 ? 2 : 0));
+          if (pos < kFwdMaxSparseTiles) {  // the host keeps every list within the capacity
+            sm.act_tile[pos] = (uint16_t)(base + i * 32 + lane);
+            sm.act_bits[pos] = (uint8_t)((a0[i] != 0 ? 1 : 0) | (a1[i] != 0 ? 2 : 0));
+          }
         }
         count += __popc(bal);
       }
     }
-    if (lane == 0) sm.n_act = count;
+    if (lane == 0) {
+      if (count > kFwdMaxSparseTiles) record_status(-25, count);
+      sm.n_act = min(count, kFwdMaxSparseTiles);
+    }
   }
   if (warp == 9) {
     tmem_alloc(smem_u32(&sm.tmem_base), 512);

@@ -707,6 +707,7 @@ const char* mfa_status_string(int code) {
     case MFA_ERR_DEVICE_TIMEOUT: return "device: a bounded wait inside a kernel ran out";
     case MFA_ERR_DEVICE_BAD_PAGE: return "device: block_table or seq_lens entry out of range";
     case MFA_ERR_DEVICE_BAD_SEQLENS: return "device: cu_seqlens entry negative, decreasing, past the packed total, or a sequence longer than max_seqlen_q";
+    case MFA_ERR_DEVICE_TILE_LIST: return "device: a key-tile list exceeded its capacity (tiles past it were not visited)";
     case MFA_ERR_SCRATCH_TOO_SMALL: return "decode shape needs more workspace than the fixed 64 MiB scratch of mfa_decode_splitkv_noalloc";
     default: return "unknown status";
   }
