@@ -386,8 +386,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       // Block-sparse: Q tile t takes part in visited tile u only where its bit is on; its MMAs
       // are skipped elsewhere and its barriers count only the tiles it takes part in. (Dense:
       // every Q tile takes part in every tile, and the counts below are the loop index.)
-      auto act = [&](int u, int t) -> bool {
-        if constexpr (SPARSE) return ((sm.act_bits[u] >> t) & 1) != 0; else return true;
+      // the bits of tile j + 1 are read at the top of iteration j, ahead of the waits, and
+      // carried into iteration j + 1 (a shared load after a wait would sit on the issue path)
+      uint32_t bits_cur = SPARSE ? sm.act_bits[0] : 3u, bits_next = 3u;
+      auto act_cur = [&](int t) -> bool {  // Q tile t takes part in tile j
+        if constexpr (SPARSE) return ((bits_cur >> t) & 1u) != 0; else return true;
+      };
+      auto act_next = [&](int t) -> bool {  // ... in tile j + 1
+        if constexpr (SPARSE) return ((bits_next >> t) & 1u) != 0; else return true;
       };
       int npv[kFwdQT] = {0, 0};  // PV groups issued per Q tile (SPARSE only)
       for (int j = 0; ok && j < n_act; ++j) {  // j counts visited tiles
@@ -396,14 +402,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         const int s1 = (j + 1) % kFwdStages;
         const uint32_t ph1 = ((j + 1) / kFwdStages) & 1;
         const bool more = j + 1 < n_act;
+        if constexpr (SPARSE) {
+          if (j > 0) bits_cur = bits_next;
+          bits_next = more ? sm.act_bits[j + 1] : 0u;
+        }
         if (j == 0) {
           if (!(ok = mbar_wait(smem_u32(&sm.bar_k_full[s]), ph, abort, 902))) break;
           tc_fence_after();
-          if (act(0, 0)) {
+          if (act_cur(0)) {
             issue_qk(0, s);
             tc_commit(smem_u32(&sm.bar_s_full[0]));
           }
-          if (act(0, 1)) {
+          if (act_cur(1)) {
             issue_qk(1, s);
             tc_commit(smem_u32(&sm.bar_s_full[1]));
           }
@@ -411,7 +421,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         }
         // Q tile 0: PV(j), then QK(j+1) once PV(j) is done (P_0 lives in S_0's columns)
         if (!(ok = mbar_wait(smem_u32(&sm.bar_v_full[s]), ph, abort, 903))) break;
-        if (act(j, 0)) {
+        if (act_cur(0)) {
           const int c = SPARSE ? npv[0] : j;
           if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[0][0]), c & 1, abort, 904))) break;
           tc_fence_after();
@@ -424,7 +434,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         }
         if (more) {
           if (!(ok = mbar_wait(smem_u32(&sm.bar_k_full[s1]), ph1, abort, 905))) break;
-          if (act(j + 1, 0)) {
+          if (act_next(0)) {
             // the latest PV of Q tile 0 read P_0 from S_0's columns
             if (!SPARSE || npv[0] > 0)
               if (!(ok = mbar_wait(smem_u32(&sm.bar_o_done[0]), (SPARSE ? npv[0] - 1 : j) & 1, abort, 906))) break;
@@ -434,7 +444,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
           }
         }
         // Q tile 1
-        if (act(j, 1)) {
+        if (act_cur(1)) {
           const int c = SPARSE ? npv[1] : j;
           if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[1][0]), c & 1, abort, 907))) break;
           tc_fence_after();
@@ -447,7 +457,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         }
         tc_commit(smem_u32(&sm.bar_v_empty[s]));
         if (more) {
-          if (act(j + 1, 1)) {
+          if (act_next(1)) {
             if (!SPARSE || npv[1] > 0)
               if (!(ok = mbar_wait(smem_u32(&sm.bar_o_done[1]), (SPARSE ? npv[1] - 1 : j) & 1, abort, 908))) break;
             tc_fence_after();
