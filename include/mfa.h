@@ -345,8 +345,8 @@ int mfa_debug_set_flags(int flags);
 int mfa_debug_tiles_visited(void* stream, unsigned long long* count);
 
 /*
- * Decode split size override in pages (0 = automatic). It changes the split plan, and with it
- * mfa_decode_workspace_size. Returns the previous value.
+ * Decode split size override in pages (0 = automatic, at most 64). It changes the split plan,
+ * and with it mfa_decode_workspace_size. Returns the previous value.
  */
 int mfa_debug_set_decode_split_pages(int pages);
 

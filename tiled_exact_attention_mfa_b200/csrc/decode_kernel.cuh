@@ -28,6 +28,7 @@
 namespace mfa {
 
 constexpr int kDecPage = 16;
+constexpr int kDecMaxSplitPages = 64;  // pages per phase-1 split at most (two table entries per lane)
 constexpr int kDecStages = 3;
 
 struct DecodeParams {
@@ -120,16 +121,18 @@ __global__ void __launch_bounds__((kDecMaxHeads<D> + 1) * 32) mfa_decode_phase1_
 
   if (warp == hg) {
     // ====================================================== producer warp
-    // block_table entries of this split, one per lane (pages_per_split <= 32)
-    int page_id = -1;
-    if (lane < np) page_id = p.block_table[(size_t)b * p.max_pages + pg0 + lane];
-    const bool bad = (lane < np) && (page_id < 0 || page_id >= p.num_pages);
-    if (bad) record_status(-22, b * 65536 + pg0 + lane);
+    // block_table entries of this split, two per lane (pages_per_split <= kDecMaxSplitPages)
+    int page_lo = -1, page_hi = -1;  // entries pg0 + lane and pg0 + 32 + lane
+    if (lane < np) page_lo = p.block_table[(size_t)b * p.max_pages + pg0 + lane];
+    if (32 + lane < np) page_hi = p.block_table[(size_t)b * p.max_pages + pg0 + 32 + lane];
+    if (lane < np && (page_lo < 0 || page_lo >= p.num_pages)) record_status(-22, b * 65536 + pg0 + lane);
+    if (32 + lane < np && (page_hi < 0 || page_hi >= p.num_pages))
+      record_status(-22, b * 65536 + pg0 + 32 + lane);
     int issued[kDecStages] = {0, 0, 0};
     for (int i = 0; i < np; ++i) {
       const int s = i % kDecStages;
       const int use = i / kDecStages;
-      const int pid = __shfl_sync(0xffffffffu, page_id, i);
+      const int pid = __shfl_sync(0xffffffffu, i < 32 ? page_lo : page_hi, i & 31);
       const bool pid_ok = pid >= 0 && pid < p.num_pages;
       const int valid = min(kDecPage, len - (pg0 + i) * kDecPage);
       bool ok = true;

@@ -133,7 +133,7 @@ DecodePlan decode_plan(int B, int Hkv, int D, int max_pages, int Nq = 1, int win
   pl.groups = Hkv / pl.heads_per_cta;
   int s = 32;
   if (g_split_pages_override > 0) {
-    s = g_split_pages_override > 32 ? 32 : g_split_pages_override;
+    s = std::min(g_split_pages_override, mfa::kDecMaxSplitPages);
   } else {
     // halve the split while the grid would hold fewer than two CTAs per SM (148 SMs)
     while (s > 4 && (long long)B * ((max_pages + s - 1) / s) * pl.groups < 296) s /= 2;
