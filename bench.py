@@ -480,7 +480,9 @@ def run_gpu(args):
         import torch.distributed as dist
         dist.barrier()
     others = []
-    if not args.only_main:
+    # the secondary workloads run at N = 1 only: a scaling run measures the headline, and every
+    # rank would otherwise build all their inputs (page pools of GBs) in host memory at once
+    if not args.only_main and world == 1:
         for name, case in W.items():
             if name == args.workload:
                 continue
@@ -525,6 +527,7 @@ def run_gpu(args):
                                "frac_of_measured_tensor_peak": round(tf / pk["tflops"], 4),
                                "frac_of_nominal_tensor_peak": round(tf / NOMINAL_TFLOPS, 4),
                                "frac_of_roofline": round(t_floor / (r["ms"] * 1e-3), 4)})
+            getattr(case, "_cache", {}).clear()  # the workload's host inputs are not needed again
         for name in BACKWARD_WORKLOADS:
             sk, wu = max(3, min(args.steps, 10)), max(3, args.warmup)
             r = bench_backward(W[name], sk, wu, flush, stream, world)
