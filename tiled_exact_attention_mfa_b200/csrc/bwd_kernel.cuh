@@ -457,16 +457,24 @@ __global__ void __launch_bounds__(kBwdKvThreads, 1) mfa_bwd_dkv_kernel(const __g
 // dS goes to two spare TMEM buffers [384, 448) and [448, 512), so S / dP of key tile u + 1 are
 // computed while the elementwise warps work on tile u: the MMA thread issues them as soon as
 // every elementwise warp has read S / dP of tile u (bar_ld), then dQ += dS K for tile u.
+// K and V have rings of their own: V of tile u is read only by dP of tile u, so its slot is
+// released as soon as S / dP of tile u complete; K is read again by dQ of tile u, so its ring has
+// a third stage, and K of tile u + 1 is already in flight while dQ of tile u - 1 still reads its
+// slot (with one shared 2-stage ring the copy of tile u + 1 started only after dQ of tile u - 1
+// and sat on the critical path).
 constexpr int kBwdQThreads = 384;
+constexpr int kBwdQKStages = 3;
+constexpr int kBwdQVStages = 2;
 
 template <int D>
 struct BwdQSmem {
   static constexpr int kTile = kBwdBM * D * 2;
   uint8_t q[kTile];
   uint8_t dout[kTile];
-  uint8_t k[kBwdStages][kTile];
-  uint8_t v[kBwdStages][kTile];
-  uint64_t bar_qo, bar_full[kBwdStages], bar_empty[kBwdStages];
+  uint8_t k[kBwdQKStages][kTile];
+  uint8_t v[kBwdQVStages][kTile];
+  uint64_t bar_qo, bar_kfull[kBwdQKStages], bar_kempty[kBwdQKStages];
+  uint64_t bar_vfull[kBwdQVStages], bar_vempty[kBwdQVStages];
   // bar_ds[u % 2]: every elementwise warp stored dS of key tile u. S / dP of tile u + 1 are
   // issued once every warp has loaded tile u, so a fast warp can finish tile u + 1 before a slow
   // one finishes tile u; alternating barriers keep its arrival out of tile u's phase (it cannot
@@ -508,9 +516,13 @@ __global__ void __launch_bounds__(kBwdQThreads, 1) mfa_bwd_dq_kernel(const __gri
   constexpr uint32_t kTile = BwdQSmem<D>::kTile;
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&sm.bar_qo), 1);
-    for (int st = 0; st < kBwdStages; ++st) {
-      mbar_init(smem_u32(&sm.bar_full[st]), 1);
-      mbar_init(smem_u32(&sm.bar_empty[st]), 1);
+    for (int st = 0; st < kBwdQKStages; ++st) {
+      mbar_init(smem_u32(&sm.bar_kfull[st]), 1);
+      mbar_init(smem_u32(&sm.bar_kempty[st]), 1);
+    }
+    for (int st = 0; st < kBwdQVStages; ++st) {
+      mbar_init(smem_u32(&sm.bar_vfull[st]), 1);
+      mbar_init(smem_u32(&sm.bar_vempty[st]), 1);
     }
     mbar_init(smem_u32(&sm.bar_sp), 1);
     mbar_init(smem_u32(&sm.bar_ld), 8);
@@ -547,24 +559,30 @@ __global__ void __launch_bounds__(kBwdQThreads, 1) mfa_bwd_dq_kernel(const __gri
         tma_load_3d(smem_u32(sm.q) + sl * 128 * 128, &p.tm_q, bqo, sl * 64, q0, b * p.Hq + h);
         tma_load_3d(smem_u32(sm.dout) + sl * 128 * 128, &p.tm_do, bqo, sl * 64, q0, b * p.Hq + h);
       }
-      int issued[kBwdStages] = {};
+      int issued_k[kBwdQKStages] = {}, issued_v[kBwdQVStages] = {};
       for (int u = 0; u < n_kt; ++u) {
-        const int st = u % kBwdStages;
-        const int use = u / kBwdStages;
+        const int sk = u % kBwdQKStages, uk = u / kBwdQKStages;
+        const int sv = u % kBwdQVStages, uv = u / kBwdQVStages;
         const int row = (kt_lo + u) * kBwdBM;
-        if (use > 0 && !mbar_wait(smem_u32(&sm.bar_empty[st]), (use - 1) & 1, abort, 1401)) break;
-        const uint32_t bf = smem_u32(&sm.bar_full[st]);
-        mbar_expect_tx(bf, 2 * kTile);
-        for (int sl = 0; sl < kSlabs; ++sl) {
-          tma_load_3d(smem_u32(sm.k[st]) + sl * 128 * 128, &p.tm_k, bf, sl * 64, row, b * p.Hkv + g);
-          tma_load_3d(smem_u32(sm.v[st]) + sl * 128 * 128, &p.tm_v, bf, sl * 64, row, b * p.Hkv + g);
-        }
-        issued[st] = use + 1;
+        if (uk > 0 && !mbar_wait(smem_u32(&sm.bar_kempty[sk]), (uk - 1) & 1, abort, 1401)) break;
+        const uint32_t bk = smem_u32(&sm.bar_kfull[sk]);
+        mbar_expect_tx(bk, kTile);
+        for (int sl = 0; sl < kSlabs; ++sl)
+          tma_load_3d(smem_u32(sm.k[sk]) + sl * 128 * 128, &p.tm_k, bk, sl * 64, row, b * p.Hkv + g);
+        issued_k[sk] = uk + 1;
+        if (uv > 0 && !mbar_wait(smem_u32(&sm.bar_vempty[sv]), (uv - 1) & 1, abort, 1404)) break;
+        const uint32_t bv = smem_u32(&sm.bar_vfull[sv]);
+        mbar_expect_tx(bv, kTile);
+        for (int sl = 0; sl < kSlabs; ++sl)
+          tma_load_3d(smem_u32(sm.v[sv]) + sl * 128 * 128, &p.tm_v, bv, sl * 64, row, b * p.Hkv + g);
+        issued_v[sv] = uv + 1;
       }
       volatile int no_abort = 0;
       mbar_wait(bqo, 0, &no_abort, 1402);
-      for (int st = 0; st < kBwdStages; ++st)
-        if (issued[st] > 0) mbar_wait(smem_u32(&sm.bar_full[st]), (issued[st] - 1) & 1, &no_abort, 1403);
+      for (int st = 0; st < kBwdQKStages; ++st)
+        if (issued_k[st] > 0) mbar_wait(smem_u32(&sm.bar_kfull[st]), (issued_k[st] - 1) & 1, &no_abort, 1403);
+      for (int st = 0; st < kBwdQVStages; ++st)
+        if (issued_v[st] > 0) mbar_wait(smem_u32(&sm.bar_vfull[st]), (issued_v[st] - 1) & 1, &no_abort, 1405);
     }
    } else if (warp == 9) {
     // ================================================================ MMA issuer
@@ -573,17 +591,20 @@ __global__ void __launch_bounds__(kBwdQThreads, 1) mfa_bwd_dq_kernel(const __gri
       const uint32_t id_o = idesc_f16(BF16 ? 1 : 0, kBwdBM, D, 1);       // dQ: B MN-major
       const uint32_t qa = smem_u32(sm.q), oa = smem_u32(sm.dout);
       auto issue_sdp = [&](int u) -> bool {
-        const int st = u % kBwdStages;
-        if (!mbar_wait(smem_u32(&sm.bar_full[st]), (u / kBwdStages) & 1, abort, 1502)) return false;
+        const int sk = u % kBwdQKStages, sv = u % kBwdQVStages;
+        if (!mbar_wait(smem_u32(&sm.bar_kfull[sk]), (u / kBwdQKStages) & 1, abort, 1502)) return false;
         tc_fence_after();
-        const uint32_t ka = smem_u32(sm.k[st]), va = smem_u32(sm.v[st]);
+        const uint32_t ka = smem_u32(sm.k[sk]), va = smem_u32(sm.v[sv]);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           tc_mma_ss(tmem + 0, bwd_desc_k(qa, kk), bwd_desc_k(ka, kk), id_s, kk > 0 ? 1u : 0u);
+        if (!mbar_wait(smem_u32(&sm.bar_vfull[sv]), (u / kBwdQVStages) & 1, abort, 1506)) return false;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           tc_mma_ss(tmem + 128, bwd_desc_k(oa, kk), bwd_desc_k(va, kk), id_s, kk > 0 ? 1u : 0u);
         tc_commit(smem_u32(&sm.bar_sp));  // also covers every earlier dQ MMA
+        tc_commit(smem_u32(&sm.bar_vempty[sv]));  // V of tile u is not read again
         return true;
       };
       bool ok = mbar_wait(smem_u32(&sm.bar_qo), 0, abort, 1501) && issue_sdp(0);
@@ -595,12 +616,12 @@ __global__ void __launch_bounds__(kBwdQThreads, 1) mfa_bwd_dq_kernel(const __gri
         }
         if (!(ok = mbar_wait(smem_u32(&sm.bar_ds[u & 1]), (u >> 1) & 1, abort, 1504))) break;
         tc_fence_after();
-        const uint32_t ka = smem_u32(sm.k[u % kBwdStages]);
+        const uint32_t ka = smem_u32(sm.k[u % kBwdQKStages]);
         const uint32_t ds_col = 384 + (u & 1) * 64;
 #pragma unroll
         for (int kk = 0; kk < kBwdBM / 16; ++kk)
           tc_mma_ts(tmem + 256, tmem + ds_col + kk * 8, bwd_desc_mn(ka, kk), id_o, (u > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(smem_u32(&sm.bar_empty[u % kBwdStages]));
+        tc_commit(smem_u32(&sm.bar_kempty[u % kBwdQKStages]));
       }
       tc_commit(smem_u32(&sm.bar_final));
       volatile int no_abort = 0;
