@@ -1,0 +1,86 @@
+"""Repeated calls on the full-size workloads give the same bits, for every entry point.
+
+None of the kernels uses atomics or a data-dependent order of accumulation, so a difference
+between two calls on the same inputs can only come from a read that raced a write: a phase wait
+that returned early, a shared-memory or TMEM buffer refilled before its reader was done, an
+epilogue that read an accumulator before the last MMA completed. Such races depend on timing
+and show most at full size, where every SM holds work and the pipelines run full; each path
+runs four times here with an L2-sized buffer written between calls to vary the timing."""
+import numpy as np
+import pytest
+
+import mfa_inputs as mi
+from gpu_util import to_torch
+
+pytestmark = pytest.mark.gpu
+
+RUNS = 4
+
+
+def repeats_bitwise(fn):
+    import torch
+    import tiled_exact_attention_mfa_b200 as mfa
+    scratch = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    first = None
+    for i in range(RUNS):
+        scratch.fill_(i)  # evict L2 so each call meets a different cache state
+        got = fn()
+        torch.cuda.synchronize()
+        if first is None:
+            first = [t.clone() for t in got]
+        else:
+            for a, b in zip(first, got):
+                assert torch.equal(a, b)
+    assert mfa.mfa_device_status() == (0, 0)
+
+
+@pytest.mark.parametrize("name", ["causal_b2_h8_n4096_d128_fp16", "noncausal_b2_h8_n4096_d128_fp16",
+                                  "window512_b2_h8_n8192_d128_fp16",
+                                  "gqa_causal_b1_hq32_hkv8_n16384_d128_bf16_cap50"])
+def test_forward_and_backward_repeat(cuda_device, name):
+    import tiled_exact_attention_mfa_b200 as mfa
+    c = mi.workloads()[name]
+    q, k, v = (to_torch(x, c.dtype) for x in c.tensors())
+    kw = dict(scale=c.scale_f32(), causal=c.causal, window=(c.win_l, c.win_r), softcap=c.softcap)
+    repeats_bitwise(lambda: mfa.mfa_fwd(q, k, v, **kw))
+    out, lse = mfa.mfa_fwd(q, k, v, **kw)
+    do = to_torch(mi.normal_bits(c.seed + 500, mi.STREAM_Q, tuple(out.shape), c.dtype), c.dtype)
+    repeats_bitwise(lambda: mfa.mfa_bwd(q, k, v, out, do, lse, **kw))
+
+
+@pytest.mark.parametrize("name", ["decode_b8_hq32_hkv8_d128_bf16_len8k_128k",
+                                  "decode_verify_nq4_b8_hq32_hkv8_d128_bf16_len8k_128k",
+                                  "decode_window4k_b8_hq32_hkv8_d128_bf16_len8k_128k"])
+def test_decode_repeats(cuda_device, name):
+    import torch
+    import tiled_exact_attention_mfa_b200 as mfa
+    d = mi.workloads()[name]
+    qd, kp, vp, table, lens = d.tensors()
+    a = (to_torch(qd, d.dtype), to_torch(kp, d.dtype), to_torch(vp, d.dtype),
+         torch.from_numpy(table).cuda(), torch.from_numpy(lens).cuda())
+    repeats_bitwise(lambda: mfa.mfa_decode_splitkv(*a, scale=d.scale_f32(), causal=d.causal,
+                                                   win_l=d.win_l))
+
+
+def test_varlen_sparse_and_paged_prefill_repeat(cuda_device):
+    import torch
+    import tiled_exact_attention_mfa_b200 as mfa
+    W = mi.workloads()
+    vc = W["varlen_causal_b8_h8_d128_fp16_len512_8k"]
+    q, k, v = (to_torch(x, vc.dtype) for x in vc.tensors())
+    cq, ck = (torch.from_numpy(x).cuda() for x in vc.cu_seqlens())
+    mx = int(np.max(np.diff(vc.cu_seqlens()[0])))
+    repeats_bitwise(lambda: mfa.mfa_fwd_varlen(q, k, v, cq, ck, mx, scale=vc.scale_f32(),
+                                               causal=True))
+    sc = W["sparse_spatial2d_b1_h16_n16384_d128_fp16"]
+    q, k, v, m = sc.tensors()
+    q, k, v = (to_torch(x, sc.dtype) for x in (q, k, v))
+    m = torch.from_numpy(m).cuda()
+    repeats_bitwise(lambda: mfa.mfa_fwd_blocksparse(q, k, v, m, scale=sc.scale_f32(),
+                                                    causal=sc.causal))
+    pc = W["paged_prefill_b8_hq32_hkv8_d128_bf16_ctx4k_32k"]
+    q, kp, vp, table, lens, cq = pc.tensors()
+    a = (to_torch(q, pc.dtype), to_torch(kp, pc.dtype), to_torch(vp, pc.dtype),
+         torch.from_numpy(table).cuda(), torch.from_numpy(lens).cuda(), torch.from_numpy(cq).cuda(),
+         int(np.max(np.diff(cq))))
+    repeats_bitwise(lambda: mfa.mfa_fwd_paged(*a, scale=pc.scale_f32(), causal=True))
