@@ -233,6 +233,25 @@ def time_steps(fn, steps, warmup, flush, stream):
     return [s.elapsed_time(e) for s, e in ev], b0.elapsed_time(b1)
 
 
+def spread(ms):
+    """Median and 10th / 90th percentiles of one rank's per-step times (ms)."""
+    xs = sorted(ms)
+    if not xs:
+        return {}
+
+    def pct(q):  # linear interpolation between order statistics
+        pos = q * (len(xs) - 1)
+        lo = int(pos)
+        hi = min(lo + 1, len(xs) - 1)
+        return xs[lo] + (xs[hi] - xs[lo]) * (pos - lo)
+    return {"ms_median": round(pct(0.5), 5), "ms_p10": round(pct(0.1), 5),
+            "ms_p90": round(pct(0.9), 5)}
+
+
+def spread_of(r):
+    return {k: r[k] for k in ("ms_median", "ms_p10", "ms_p90") if k in r}
+
+
 def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
     """Largest per-rank time: every rank runs its own copy of the workload (weak scaling), so the
     job takes as long as its slowest rank."""
@@ -267,7 +286,7 @@ def bench_prefill(case, steps, warmup, flush, stream, with_e2e, world):
 
     with torch.cuda.stream(stream):
         ms, bracket = time_steps(step, steps, warmup, flush, stream)
-    res = {"ms": statistics.mean(ms), "ms_min": min(ms), "bracket_ms": bracket,
+    res = {"ms": statistics.mean(ms), "ms_min": min(ms), **spread(ms), "bracket_ms": bracket,
            "flops": prefill_flops(case), "bytes": prefill_bytes(case)}
     res["ms"] = max_over_ranks(res["ms"], world)
     if with_e2e:
@@ -328,7 +347,7 @@ def bench_varlen(case, steps, warmup, flush, stream, world):
 
     with torch.cuda.stream(stream):
         ms, bracket = time_steps(step, steps, warmup, flush, stream)
-    return {"ms": max_over_ranks(statistics.mean(ms), world), "ms_min": min(ms),
+    return {"ms": max_over_ranks(statistics.mean(ms), world), "ms_min": min(ms), **spread(ms),
             "bracket_ms": bracket, "flops": varlen_flops(case), "bytes": varlen_bytes(case),
             "total_q": int(cq[-1])}
 
@@ -353,7 +372,7 @@ def bench_sparse(case, steps, warmup, flush, stream, world):
     pairs = sparse_pairs(case, m)
     byts = 2 * case.B * case.Hq * case.Nq * case.D * 2 + 2 * 2 * case.B * case.Hkv * case.Nk * case.D \
         + 4 * case.B * case.Hq * case.Nq + m.size
-    return {"ms": max_over_ranks(statistics.mean(ms), world), "ms_min": min(ms),
+    return {"ms": max_over_ranks(statistics.mean(ms), world), "ms_min": min(ms), **spread(ms),
             "bracket_ms": bracket, "flops": 4.0 * case.D * pairs, "bytes": float(byts),
             "density": float(m.mean())}
 
@@ -382,7 +401,7 @@ def bench_backward(case, steps, warmup, flush, stream, world):
 
     with torch.cuda.stream(stream):
         ms, bracket = time_steps(step, steps, warmup, flush, stream)
-    return {"ms": max_over_ranks(statistics.mean(ms), world), "ms_min": min(ms),
+    return {"ms": max_over_ranks(statistics.mean(ms), world), "ms_min": min(ms), **spread(ms),
             "bracket_ms": bracket, "flops": 2.5 * prefill_flops(case),
             "bytes": 2.0 * prefill_bytes(case)}
 
@@ -411,7 +430,7 @@ def bench_paged(case, steps, warmup, flush, stream, world):
         ms, bracket = time_steps(step, steps, warmup, flush, stream)
     pairs = sum(visible_pairs(case_like(case), a, b) for a, b in zip(nq, lens))
     kv_bytes = float(np.sum(lens)) * case.Hkv * case.D * 2 * 2
-    return {"ms": max_over_ranks(statistics.mean(ms), world), "ms_min": min(ms),
+    return {"ms": max_over_ranks(statistics.mean(ms), world), "ms_min": min(ms), **spread(ms),
             "bracket_ms": bracket, "flops": 4.0 * case.D * case.Hq * pairs,
             "bytes": kv_bytes + 2 * 2 * float(cq[-1]) * case.Hq * case.D, "total_q": int(cq[-1])}
 
@@ -442,7 +461,7 @@ def bench_decode(case, steps, warmup, flush, stream, world):
 
     with torch.cuda.stream(stream):
         ms, bracket = time_steps(step, steps, warmup, flush, stream)
-    return {"ms": max_over_ranks(statistics.mean(ms), world), "ms_min": min(ms),
+    return {"ms": max_over_ranks(statistics.mean(ms), world), "ms_min": min(ms), **spread(ms),
             "bracket_ms": bracket, "bytes": decode_bytes(case, lens),
             "flops": decode_flops(case, lens), "seq_len_sum": int(np.sum(lens)),
             "visible_tokens": int(decode_tokens(case, lens)[0])}
@@ -497,7 +516,7 @@ def run_gpu(args):
                 tf = r["flops"] * world / (r["ms"] * 1e-3) / 1e12
                 gbs = r["bytes"] * world / (r["ms"] * 1e-3) / 1e9
                 t_floor = max(r["flops"] / (pk["tflops"] * 1e12), r["bytes"] / (pk["gbs"] * 1e9))
-                others.append({"workload": name, "ms": round(r["ms"], 4), "unit": "TFLOP/s",
+                others.append({**spread_of(r), "workload": name, "ms": round(r["ms"], 4), "unit": "TFLOP/s",
                                "value": round(tf, 1), "GB/s": round(gbs, 1),
                                **({"total_q": r["total_q"]} if "total_q" in r else
                                   {"block_density": round(r["density"], 4)}),
@@ -507,7 +526,7 @@ def run_gpu(args):
             elif isinstance(case, mi.DecodeCase):
                 r = bench_decode(case, sk, wu, flush, stream, world)
                 tb = r["bytes"] * world / (r["ms"] * 1e-3) / 1e9
-                others.append({"workload": name, "ms": round(r["ms"], 4), "unit": "GB/s",
+                others.append({**spread_of(r), "workload": name, "ms": round(r["ms"], 4), "unit": "GB/s",
                                "value": round(tb, 1), "bound": "hbm",
                                "frac_of_measured_peak": round(tb / pk["gbs"], 4),
                                "frac_of_nominal_peak": round(tb / NOMINAL_GBS, 4),
@@ -522,7 +541,7 @@ def run_gpu(args):
                 tf = r["flops"] * world / (r["ms"] * 1e-3) / 1e12
                 gbs = r["bytes"] * world / (r["ms"] * 1e-3) / 1e9
                 t_floor = max(r["flops"] / (pk["tflops"] * 1e12), r["bytes"] / (pk["gbs"] * 1e9))
-                others.append({"workload": name, "ms": round(r["ms"], 4), "unit": "TFLOP/s",
+                others.append({**spread_of(r), "workload": name, "ms": round(r["ms"], 4), "unit": "TFLOP/s",
                                "value": round(tf, 1), "GB/s": round(gbs, 1),
                                "frac_of_measured_tensor_peak": round(tf / pk["tflops"], 4),
                                "frac_of_nominal_tensor_peak": round(tf / NOMINAL_TFLOPS, 4),
@@ -532,7 +551,7 @@ def run_gpu(args):
             sk, wu = max(3, min(args.steps, 10)), max(3, args.warmup)
             r = bench_backward(W[name], sk, wu, flush, stream, world)
             tf = r["flops"] * world / (r["ms"] * 1e-3) / 1e12
-            others.append({"workload": name + ":backward", "ms": round(r["ms"], 4),
+            others.append({**spread_of(r), "workload": name + ":backward", "ms": round(r["ms"], 4),
                            "unit": "TFLOP/s", "value": round(tf, 1),
                            "frac_of_measured_tensor_peak": round(tf / pk["tflops"], 4),
                            "frac_of_nominal_tensor_peak": round(tf / NOMINAL_TFLOPS, 4),
@@ -548,6 +567,7 @@ def run_gpu(args):
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(main["ms"], 5),
+        **spread_of(main),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,

@@ -1,5 +1,6 @@
 """bench.py's reference arm (the oracle timed on the host cores) on the CPU: one JSON line with the
-contract's keys, and under torchrun only rank 0 prints it (the other ranks exit 0 without work)."""
+contract's keys, and under torchrun only rank 0 prints it (the other ranks exit 0 without work); the
+step-time spread (median, 10th / 90th percentiles) that every bench line carries."""
 import json
 import os
 import subprocess
@@ -36,3 +37,14 @@ def test_reference_arm_other_ranks_exit_quietly():
     r = run_ref({"RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def test_step_time_spread_is_median_and_deciles():
+    """The per-workload spread the bench reports: median and 10th / 90th percentiles by linear
+    interpolation between order statistics, independent of the order the steps ran in."""
+    sys.path.insert(0, ROOT)
+    import bench
+    r = bench.spread([10.0, 1.0, 9.0, 2.0, 8.0, 3.0, 7.0, 4.0, 6.0, 5.0])
+    assert r == {"ms_median": 5.5, "ms_p10": 1.9, "ms_p90": 9.1}
+    assert bench.spread([2.0]) == {"ms_median": 2.0, "ms_p10": 2.0, "ms_p90": 2.0}
+    assert bench.spread([]) == {}
