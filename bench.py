@@ -545,7 +545,8 @@ def run_gpu(args):
                                "value": round(tf, 1), "GB/s": round(gbs, 1),
                                "frac_of_measured_tensor_peak": round(tf / pk["tflops"], 4),
                                "frac_of_nominal_tensor_peak": round(tf / NOMINAL_TFLOPS, 4),
-                               "frac_of_roofline": round(t_floor / (r["ms"] * 1e-3), 4)})
+                               "frac_of_roofline": round(t_floor / (r["ms"] * 1e-3), 4),
+                               "traffic": ncu_traffic(name, "mfa_fwd_kernel")})
             getattr(case, "_cache", {}).clear()  # the workload's host inputs are not needed again
         for name in BACKWARD_WORKLOADS:
             sk, wu = max(3, min(args.steps, 10)), max(3, args.warmup)
