@@ -323,8 +323,9 @@ __global__ void __launch_bounds__((kDecMaxHeads<D> + 1) * 32) mfa_decode_phase1_
   }
 }
 
-// Threads per combine CTA: G = kCombineThreads / D groups of D threads (one per output column);
-// group g takes splits g, g + G, g + 2G, ...
+// Threads per combine CTA. Each thread owns 4 consecutive output columns (one 16-byte load per
+// split), so a group of D / 4 threads covers a row and there are G = 4 * kCombineThreads / D
+// groups; group g takes splits g, g + G, g + 2G, ...
 constexpr int kCombineThreads = 512;
 // Splits a thread loads before folding them into its running statistics: all their loads are
 // issued together, so a sequence of n splits costs about n / (G * kCombineBatch) memory round trips.
@@ -337,13 +338,14 @@ constexpr int kCombineBatch = 8;
 // phase 1 has completed and its workspace writes are visible (a no-op on a plain launch).
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kCombineThreads) mfa_decode_combine_kernel(const __grid_constant__ DecodeParams p) {
-  constexpr int G = kCombineThreads / D;
-  __shared__ float part[G][D];
+  constexpr int kRowThreads = D / 4;
+  constexpr int G = kCombineThreads / kRowThreads;
+  __shared__ __align__(16) float part[G][D];
   __shared__ float part_m[G], part_l[G];
   const int row = blockIdx.x;  // h * Nq + t
   const int b = blockIdx.y;
-  const int d = threadIdx.x % D;
-  const int grp = threadIdx.x / D;
+  const int dq = threadIdx.x % kRowThreads;  // columns 4 dq .. 4 dq + 3
+  const int grp = threadIdx.x / kRowThreads;
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int len = checked_len(p, b, false);
   const int n_pages = (len + kDecPage - 1) / kDecPage;
@@ -351,18 +353,19 @@ __global__ void __launch_bounds__(kCombineThreads) mfa_decode_combine_kernel(con
   const size_t rows_all = (size_t)p.Hq * p.Nq;
   const size_t slot0 = (size_t)b * p.max_splits * rows_all + row;  // slot of split s: slot0 + s * rows_all
   const float2* ml = reinterpret_cast<const float2*>(p.ws_ml);
-  const float* o = p.ws_o + slot0 * D + d;
-  const size_t stride = rows_all * D;
+  const float4* o = reinterpret_cast<const float4*>(p.ws_o + slot0 * D) + dq;
+  const size_t stride = rows_all * (D / 4);  // float4 steps from one split's row to the next
 
-  float m_g = -INFINITY, l_g = 0.f, acc = 0.f;
+  float m_g = -INFINITY, l_g = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s0 = grp; s0 < n_splits; s0 += G * kCombineBatch) {
     float2 st[kCombineBatch];
-    float ov[kCombineBatch];
+    float4 ov[kCombineBatch];
 #pragma unroll
     for (int j = 0; j < kCombineBatch; ++j) {
       const int s = s0 + j * G;
       st[j] = make_float2(-INFINITY, 0.f);
-      ov[j] = 0.f;
+      ov[j] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (s < n_splits) {
         st[j] = ml[slot0 + (size_t)s * rows_all];
         ov[j] = o[(size_t)s * stride];
@@ -374,22 +377,29 @@ __global__ void __launch_bounds__(kCombineThreads) mfa_decode_combine_kernel(con
     if (m_new == -INFINITY) continue;
     const float r = (m_g == -INFINITY) ? 0.f : fast_exp2(m_g - m_new);
     l_g *= r;
-    acc *= r;
+    acc.x *= r;
+    acc.y *= r;
+    acc.z *= r;
+    acc.w *= r;
 #pragma unroll
     for (int j = 0; j < kCombineBatch; ++j) {
       const float w = (st[j].x == -INFINITY) ? 0.f : fast_exp2(st[j].x - m_new);
       l_g = fmaf(w, st[j].y, l_g);
-      acc = fmaf(w, ov[j], acc);
+      acc.x = fmaf(w, ov[j].x, acc.x);
+      acc.y = fmaf(w, ov[j].y, acc.y);
+      acc.z = fmaf(w, ov[j].z, acc.z);
+      acc.w = fmaf(w, ov[j].w, acc.w);
     }
     m_g = m_new;
   }
-  part[grp][d] = acc;
-  if (d == 0) {
+  *reinterpret_cast<float4*>(&part[grp][4 * dq]) = acc;
+  if (dq == 0) {
     part_m[grp] = m_g;
     part_l[grp] = l_g;
   }
   __syncthreads();
-  if (grp == 0) {
+  if (threadIdx.x < D) {
+    const int d = threadIdx.x;
     float M = part_m[0];
 #pragma unroll
     for (int g = 1; g < G; ++g) M = fmaxf(M, part_m[g]);
