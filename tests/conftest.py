@@ -24,6 +24,6 @@ def gpu_available() -> bool:
 @pytest.fixture(scope="session")
 def cuda_device():
     if not gpu_available():
-        pytest.fail("this test needs a CUDA device; run it with -m gpu on a GPU box")
+        pytest.fail("this test needs a CUDA device (select it with -m gpu where one is present)")
     import torch
     return torch.device("cuda:0")
