@@ -312,7 +312,7 @@ def bench_prefill(case, steps, warmup, flush, stream, with_e2e, world):
         if not (torch.equal(ho, out.cpu()) and torch.equal(hl, lse.cpu())):
             raise RuntimeError("host-buffer forward differs from the device forward")
         res["e2e_ms"] = max_over_ranks(statistics.mean(ems), world)
-        # the PCIe floor on this box, same run: the step's own pinned inputs copied in alone
+        # the PCIe floor on this machine, same run: the step's own pinned inputs copied in alone
         dq_, dk_, dv_ = (torch.empty_like(x, device=dev) for x in (hq, hk, hv))
 
         def h2d_only():
