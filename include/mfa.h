@@ -249,6 +249,21 @@ size_t mfa_decode_workspace_size(int B, int Nq, int Hq, int Hkv, int D,
                                  int max_pages_per_seq, int page_size);
 
 /*
+ * mfa_decode_plan -- the split plan mfa_decode_splitkv_window (win_l >= 0) or
+ * mfa_decode_splitkv (win_l = -1) uses for this shape, computed on the host without a launch:
+ * *kv_heads_per_cta kv heads per phase-1 CTA (the most that divide Hkv with a token row of at
+ * most 1 KB), *pages_per_split 16-token pages per split and *max_splits splits per sequence
+ * (the phase-1 grid is max_splits x B x Hkv / kv_heads_per_cta). Without a window the split
+ * starts at 32 pages and halves (down to 4) while that grid would hold fewer than 296 CTAs (two
+ * per SM); with a window it is the smallest halving of 32 whose grid over the window's page
+ * span still fits in 296 CTAs, never more splits than without the window. The override of
+ * mfa_debug_set_decode_split_pages applies. Any output pointer may be NULL. Returns MFA_OK, or
+ * the error code the decode entry point would return for these arguments.
+ */
+int mfa_decode_plan(int B, int Nq, int Hq, int Hkv, int D, int max_pages_per_seq, int page_size,
+                    int win_l, int* pages_per_split, int* max_splits, int* kv_heads_per_cta);
+
+/*
  * mfa_decode_splitkv -- two-phase split-KV decode over a paged KV cache
  * ([MFA252] Features "Flash Decode -- two-phase split-KV for N_q <= 4" and "Paged KV";
  *  [MXFA15] README: paged decode with per-split (m, l) slots and a combine step).

@@ -187,6 +187,60 @@ def test_decode_workspace_size_is_shape_only():
         mfa.mfa_debug_set_decode_split_pages(old)
 
 
+def test_decode_plan_without_window():
+    """The shape-only split plan: 32-page splits while the phase-1 grid (splits x B x kv-head
+    groups) holds at least 296 CTAs, halved down to 4 pages below that; kv heads per CTA the
+    most that divide Hkv with a token row (heads x D x 2 bytes) of at most 1 KB."""
+    p = mfa.mfa_decode_plan(8, 1, 32, 8, 128, 8192)
+    assert p == {"pages_per_split": 32, "max_splits": 256, "kv_heads_per_cta": 4}
+    assert mfa.mfa_decode_workspace_size(8, 1, 32, 8, 128, 8192) == 8 * 256 * 32 * (128 + 2) * 4
+    assert mfa.mfa_decode_plan(8, 4, 32, 8, 128, 8192)["max_splits"] == 256  # N_q does not move it
+    assert mfa.mfa_decode_plan(8, 1, 16, 8, 256, 2048)["kv_heads_per_cta"] == 2
+    assert mfa.mfa_decode_plan(8, 1, 32, 8, 64, 2048)["kv_heads_per_cta"] == 8
+    assert mfa.mfa_decode_plan(8, 1, 21, 7, 128, 2048)["kv_heads_per_cta"] == 1  # 7 x 256 B > 1 KB
+    # 1 sequence of 64 pages, 2 groups: 32 -> 16 -> 8 -> 4 pages per split (16 x 1 x 2 CTAs)
+    assert mfa.mfa_decode_plan(1, 1, 32, 8, 128, 64) == \
+        {"pages_per_split": 4, "max_splits": 16, "kv_heads_per_cta": 4}
+    # 2 sequences of 2048 pages: 64 x 2 x 2 = 256 CTAs at 32 pages is below 296, 16 pages is not
+    assert mfa.mfa_decode_plan(2, 1, 32, 8, 128, 2048)["pages_per_split"] == 16
+
+
+def test_decode_plan_with_window():
+    """With a left window the splits cover only the window's page span, (win_l + N_q + 15) / 16
+    + 1 pages: the largest split that keeps the grid within 296 CTAs, never more splits than
+    the plan without the window; the split override still applies."""
+    # 4096-token window over 128k-token caches: a span of 257 pages; 16-page splits give
+    # 17 x 8 x 2 = 272 CTAs, 8-page splits would give 33 x 8 x 2 = 528
+    assert mfa.mfa_decode_plan(8, 1, 32, 8, 128, 8192, win_l=4095) == \
+        {"pages_per_split": 16, "max_splits": 17, "kv_heads_per_cta": 4}
+    assert mfa.mfa_decode_plan(8, 4, 32, 8, 128, 8192, win_l=4095)["max_splits"] == 17  # 258 pages
+    # a window wider than the cache is the plan without a window
+    assert mfa.mfa_decode_plan(8, 1, 32, 8, 128, 8192, win_l=10 ** 9) == \
+        mfa.mfa_decode_plan(8, 1, 32, 8, 128, 8192)
+    # a one-token window spans 2 pages: one split of the smallest size
+    assert mfa.mfa_decode_plan(8, 1, 32, 8, 128, 8192, win_l=0) == \
+        {"pages_per_split": 4, "max_splits": 1, "kv_heads_per_cta": 4}
+    old = mfa.mfa_debug_set_decode_split_pages(8)
+    try:
+        p = mfa.mfa_decode_plan(8, 1, 32, 8, 128, 8192, win_l=4095)
+        assert p["pages_per_split"] == 8 and p["max_splits"] == 33
+        assert mfa.mfa_decode_plan(8, 1, 32, 8, 128, 8192)["max_splits"] == 1024
+    finally:
+        mfa.mfa_debug_set_decode_split_pages(old)
+
+
+def test_decode_plan_rejects_what_decode_rejects():
+    codes = header_defines()
+    for args, name in [((8, 5, 32, 8, 128, 8192, 16, -1), "MFA_ERR_NQ_TOO_LARGE"),
+                       ((8, 1, 32, 8, 96, 8192, 16, -1), "MFA_ERR_BAD_HEAD_DIM"),
+                       ((8, 1, 30, 8, 128, 8192, 16, -1), "MFA_ERR_GQA_GEOMETRY"),
+                       ((8, 1, 32, 8, 128, 8192, 8, -1), "MFA_ERR_PAGE_SIZE"),
+                       ((8, 1, 32, 8, 128, 8192, 16, -2), "MFA_ERR_BAD_WINDOW")]:
+        with pytest.raises(mfa.MFAError) as e:
+            mfa.mfa_decode_plan(*args[:6], page_size=args[6], win_l=args[7])
+        assert e.value.code == int(codes[name]), name
+
+
 def test_debug_flags_roundtrip():
     old = mfa.mfa_debug_set_flags(3)
     assert mfa.mfa_debug_set_flags(old) == 3

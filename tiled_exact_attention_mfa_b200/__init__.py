@@ -45,6 +45,8 @@ lib.mfa_fwd_paged.restype = _i
 lib.mfa_fwd_paged.argtypes = [_vp] * 8 + [_i] * 9 + [_f, _i, _i, _i, _f, _i, _vp]
 lib.mfa_decode_workspace_size.restype = ctypes.c_size_t
 lib.mfa_decode_workspace_size.argtypes = [_i] * 7
+lib.mfa_decode_plan.restype = _i
+lib.mfa_decode_plan.argtypes = [_i] * 8 + [ctypes.POINTER(ctypes.c_int)] * 3
 lib.mfa_decode_splitkv.restype = _i
 lib.mfa_decode_splitkv.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
                                    _f, _i, _f, _i, _vp, ctypes.c_size_t, _vp]
@@ -84,7 +86,7 @@ lib.mfa_debug_set_decode_split_pages.restype = _i
 lib.mfa_debug_set_decode_split_pages.argtypes = [_i]
 
 EXPORTED = ("mfa_fwd", "mfa_fwd_varlen", "mfa_fwd_blocksparse", "mfa_fwd_paged", "mfa_bwd_workspace_size", "mfa_bwd",
-            "mfa_decode_workspace_size", "mfa_decode_splitkv_window", "mfa_decode_splitkv", "mfa_status_string",
+            "mfa_decode_workspace_size", "mfa_decode_plan", "mfa_decode_splitkv_window", "mfa_decode_splitkv", "mfa_status_string",
             "mfa_last_launch_info", "mfa_device_status", "mfa_debug_set_flags",
             "mfa_debug_tiles_visited", "mfa_debug_set_decode_split_pages",
             "mfa_decode_splitkv_noalloc", "mfa_fwd_host_scratch_size", "mfa_fwd_host")
@@ -207,6 +209,15 @@ def mfa_fwd_host(q, k, v, out=None, lse=None, *, scale=None, causal=False, windo
 
 def mfa_decode_workspace_size(B, Nq, Hq, Hkv, D, max_pages_per_seq, page_size=16) -> int:
     return int(lib.mfa_decode_workspace_size(B, Nq, Hq, Hkv, D, max_pages_per_seq, page_size))
+
+
+def mfa_decode_plan(B, Nq, Hq, Hkv, D, max_pages_per_seq, page_size=16, win_l=-1) -> dict:
+    """The decode split plan for this shape (host only, no launch): pages per split, splits per
+    sequence and kv heads per phase-1 CTA."""
+    s, n, h = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    _check(lib.mfa_decode_plan(B, Nq, Hq, Hkv, D, max_pages_per_seq, page_size, win_l,
+                               ctypes.byref(s), ctypes.byref(n), ctypes.byref(h)), "mfa_decode_plan")
+    return {"pages_per_split": s.value, "max_splits": n.value, "kv_heads_per_cta": h.value}
 
 
 def mfa_decode_splitkv(q, k_pages, v_pages, block_table, seq_lens, out=None, lse=None, *,

@@ -605,6 +605,18 @@ int mfa_bwd(const void* q, const void* k, const void* v, const void* out, const 
 #undef MFA_BWD_CAP
 }
 
+int mfa_decode_plan(int B, int Nq, int Hq, int Hkv, int D, int max_pages_per_seq, int page_size,
+                    int win_l, int* pages_per_split, int* max_splits, int* kv_heads_per_cta) {
+  if (win_l < -1) return MFA_ERR_BAD_WINDOW;
+  const int rc = validate_decode(B, Nq, Hq, Hkv, D, page_size, max_pages_per_seq);
+  if (rc != MFA_OK) return rc;
+  const DecodePlan pl = decode_plan(B, Hkv, D, max_pages_per_seq, Nq, win_l);
+  if (pages_per_split) *pages_per_split = pl.pages_per_split;
+  if (max_splits) *max_splits = pl.max_splits;
+  if (kv_heads_per_cta) *kv_heads_per_cta = pl.heads_per_cta;
+  return MFA_OK;
+}
+
 size_t mfa_decode_workspace_size(int B, int Nq, int Hq, int Hkv, int D, int max_pages_per_seq,
                                  int page_size) {
   if (validate_decode(B, Nq, Hq, Hkv, D, page_size, max_pages_per_seq) != MFA_OK) return 0;
