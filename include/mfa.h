@@ -377,13 +377,16 @@ int mfa_debug_set_decode_split_pages(int pages);
  * device array inside the library instead of taking one from the caller; every other argument
  * has the meaning given for mfa_decode_splitkv, and the computation and result are the same.
  *
- *   - The array holds MFA_NOALLOC_SCRATCH_BYTES (64 MiB). Every GPU on which the library is
- *     loaded holds it until the process exits. A shape whose workspace
+ *   - The array holds MFA_NOALLOC_SCRATCH_BYTES (64 MiB). A device takes it when the library's
+ *     code is first used there (under CUDA's lazy module loading that can be this entry point's
+ *     first call, whose address lookup loads the module) and holds it until the process exits.
+ *     A shape whose workspace
  *     (mfa_decode_workspace_size) is larger is rejected with MFA_ERR_SCRATCH_TOO_SMALL before
  *     anything runs; the paged decode of 8 sequences x 131072 tokens with 32 query heads, 8 kv
  *     heads and D = 128 needs about 34 MB.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress with
- *     that device current) and remembers it; make that first call before any stream capture.
+ *     that device current; this can also load the module and take the array) and remembers it;
+ *     make that first call before any stream capture.
  *   - No call allocates or frees memory.
  *   - All calls on a device share the one array and leave their partial results in it. Calls
  *     whose kernels overlap on the GPU (different streams without ordering, or concurrent

@@ -30,7 +30,7 @@ Sources (web pages, cited by title and section):
     block_mask, causal=...), a block mask whose zero blocks are never attended; here a block is
     `block` query rows x `block` keys and the mask further restricts the causal / window set.
 
-Readings where the pages are silent or ambiguous (each restated in the design doc):
+Readings where the pages are silent or ambiguous (the kernels and tests follow the same ones):
   * window: key j is visible from absolute query position a iff a - win_l <= j <= a + win_r
     (inclusive; -1 = unbounded on that side), ANDed with causality when both are given;
   * causal with Nq != Nk is bottom-right aligned: query i sits at absolute position

@@ -207,8 +207,9 @@ def test_decode_plan_without_window():
 
 def test_decode_plan_with_window():
     """With a left window the splits cover only the window's page span, (win_l + N_q + 15) / 16
-    + 1 pages: the largest split that keeps the grid within 296 CTAs, never more splits than
-    the plan without the window; the split override still applies."""
+    + 1 pages: the split is the smallest halving of 32 whose grid over that span still fits in
+    296 CTAs, never with more splits than the plan without the window; the split override still
+    applies."""
     # 4096-token window over 128k-token caches: a span of 257 pages; 16-page splits give
     # 17 x 8 x 2 = 272 CTAs, 8-page splits would give 33 x 8 x 2 = 528
     assert mfa.mfa_decode_plan(8, 1, 32, 8, 128, 8192, win_l=4095) == \

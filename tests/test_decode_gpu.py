@@ -31,6 +31,10 @@ SMALL = [
        softcap=30.0, win_l=250, seed=69),
     Dc("window_edge_lengths_fp16", 6, 1, 8, 2, 64, mi.FP16, 0, 0,
        fixed_lens=[1, 16, 17, 0, 33, 513], max_pages=40, win_l=16, seed=70),
+    # a window of INT_MAX (a common "no window" sentinel) over sequences shorter than N_q: the
+    # position arithmetic must not wrap around, every row sees its whole causal prefix
+    Dc("window_int_max_short_lens_bf16", 5, 4, 8, 2, 128, mi.BF16, 0, 0,
+       fixed_lens=[0, 1, 2, 3, 40], max_pages=4, win_l=2 ** 31 - 1, seed=71),
     # D = 256: two kv heads per CTA when Hkv is even, one otherwise
     Dc("d256_nq1_gqa4_bf16", 3, 1, 16, 4, 256, mi.BF16, 1, 1500, seed=72),
     Dc("d256_nq4_gqa4_window_fp16", 2, 4, 8, 2, 256, mi.FP16, 100, 900, win_l=200, seed=73),

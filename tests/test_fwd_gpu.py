@@ -30,6 +30,12 @@ SMALL = [
     # of O runs often
     P("large_logits_noncausal_fp16", 1, 2, 2, 400, 900, 128, mi.FP16, False, seed=24,
       scale=16.0 / 128 ** 0.5),
+    # windows of INT_MAX on both sides (a common "unbounded" sentinel) with Nq > Nk: the same
+    # visible set as no window, and no wrap-around in the position arithmetic
+    P("window_int_max_nq_gt_nk_fp16", 1, 2, 2, 300, 200, 64, mi.FP16, True, 2 ** 31 - 1,
+      2 ** 31 - 1, seed=25),
+    P("window_int_max_noncausal_bf16", 1, 2, 1, 200, 333, 128, mi.BF16, False, 2 ** 31 - 1,
+      2 ** 31 - 1, seed=26),
 ]
 
 

@@ -1,11 +1,11 @@
-"""The allocation-free decode entry point (mfa_decode_splitkv_noalloc) against mfa_decode_splitkv.
+"""The allocation-free decode entry point (mfa_decode_splitkv_noalloc).
 
 Callers such as serving engines that reserve all of HBM for their KV pool, or code running
 inside an allocator callback, cannot allocate a decode workspace; this entry point uses a fixed
 device array inside the library instead. Here it is called through the C ABI twice in a row (two
 different shapes, so the second call reuses what the first left in the shared array) and each
-result must match the regular entry point's within the parity tolerances. This file is collected
-last so that a failure here cannot hide the rest of the suite.
+result must match both the fp64 oracle's decode and the regular entry point's within the parity
+tolerances. This file is collected last so that a failure here cannot hide the rest of the suite.
 """
 import ctypes
 
@@ -13,7 +13,8 @@ import numpy as np
 import pytest
 
 import mfa_inputs as mi
-from gpu_util import TOL_LSE, TOL_O, from_torch, to_torch
+import oracle
+from gpu_util import TOL_LSE, TOL_O, check_close, from_torch, to_torch
 
 pytestmark = pytest.mark.gpu
 
@@ -46,6 +47,10 @@ def test_noalloc_decode_matches_workspace_decode_twice_in_a_row(cuda_device):
                                               causal=case.causal, softcap=case.softcap)
         torch.cuda.synchronize()
         o, l, ro, rl = from_torch(out), from_torch(lse), from_torch(ref_o), from_torch(ref_l)
+        w = lambda x: mi.widen(x, case.dtype)
+        oo, ol = oracle.decode(w(q), w(k), w(v), table, lens, case.scale_f32(), case.causal,
+                               case.softcap)
+        check_close(o, l, oo, ol, case.dtype, case.name + " vs oracle")
         assert np.all(np.isfinite(o))
         assert np.max(np.abs(o - ro)) <= TOL_O[case.dtype], case.name
         fin = np.isfinite(rl)

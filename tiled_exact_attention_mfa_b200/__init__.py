@@ -260,24 +260,25 @@ def mfa_decode_splitkv(q, k_pages, v_pages, block_table, seq_lens, out=None, lse
     return out, lse
 
 
-def mfa_decode_splitkv_noalloc(q, k_pages, v_pages, block_table, seq_lens, out=None, lse=None, *,
-                               scale=None, causal=True, softcap=0.0, return_lse=True, stream=None):
+def mfa_decode_splitkv_noalloc(q, k_pages, v_pages, block_table, seq_lens, out, lse=None, *,
+                               scale=None, causal=True, softcap=0.0, stream=None):
     """mfa_decode_splitkv without a caller workspace, for callers that cannot allocate device
-    memory when decode runs (see include/mfa.h). The workspace is the library's fixed 64 MiB
-    device array; calls that overlap on the GPU race on it, so keep them on one stream.
-    Returns (out, lse or None)."""
+    memory when decode runs (an engine that has handed all of HBM to its KV page pool, code inside
+    an allocator callback). The workspace is the library's fixed 64 MiB device array; calls that
+    overlap on the GPU race on it, so keep them on one stream.
+
+    This wrapper allocates nothing either: the caller passes `out` (like q) and, if it wants the
+    log-sum-exp, `lse` (fp32 [B, Hq, Nq]; None skips it). Returns (out, lse)."""
     torch = _torch()
     B, Hq, Nq, D = q.shape
     num_pages, page, Hkv, _ = k_pages.shape
     max_pages = block_table.shape[1]
     if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
         raise TypeError("block_table and seq_lens must be int32")
+    if out is None:
+        raise ValueError("mfa_decode_splitkv_noalloc allocates nothing: pass `out`")
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None and return_lse:
-        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     rc = lib.mfa_decode_splitkv_noalloc(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
                                         _ptr(seq_lens), _ptr(out), _ptr(lse), B, Nq, Hq, Hkv, D,
                                         page, max_pages, num_pages, float(scale),

@@ -65,7 +65,9 @@ __device__ __forceinline__ int checked_len(const DecodeParams& p, int b, bool re
 // page, so pages wholly left of the window are neither read nor given a split.
 __device__ __forceinline__ int dec_first_page(const DecodeParams& p, int len) {
   if (p.win_l < 0) return 0;
-  return max(0, len - p.Nq - p.win_l) / kDecPage;
+  // 64-bit: a window near INT_MAX over a sequence shorter than Nq must not wrap around
+  const long long first = (long long)len - p.Nq - p.win_l;
+  return first > 0 ? (int)(first / kDecPage) : 0;
 }
 
 // kv heads per phase-1 CTA at most: a token row of all of them fits in 1 KB
@@ -193,7 +195,7 @@ __global__ void __launch_bounds__((kDecMaxHeads<D> + 1) * 32) mfa_decode_phase1_
     const int t = (r < R) ? (r % p.Nq) : 0;
     lim[e] = p.causal ? (len - p.Nq + t) : (len - 1);
     lim[e] = min(lim[e], len - 1);
-    low[e] = (p.win_l >= 0) ? (len - p.Nq + t - p.win_l) : 0;
+    low[e] = (p.win_l >= 0) ? (int)max(-1ll, (long long)len - p.Nq + t - p.win_l) : 0;
   }
 
   float o[D / 8][4];

@@ -3,6 +3,7 @@
 // that the device status word is one symbol.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -16,7 +17,10 @@ namespace {
 
 thread_local mfa_launch_info g_last = {};
 int g_debug_flags = 0;
-int g_split_pages_override = 0;
+// Debug override of the decode split size (0 = the plan's own). Every entry point reads it once
+// and passes that value down, so the size check and the launched plan of one call agree even
+// while another thread changes it.
+std::atomic<int> g_split_pages_override{0};
 std::mutex g_mutex;
 
 constexpr int kMaxDevices = 64;
@@ -119,7 +123,7 @@ struct DecodePlan {
 // start-up latency (block table, Q and first page in flight), so the split is halved only while
 // the halved grid still fits one wave of two CTAs per SM, and never past the split count of the
 // unwindowed plan, so the workspace that mfa_decode_workspace_size reports stays sufficient.
-DecodePlan decode_plan(int B, int Hkv, int D, int max_pages, int Nq = 1, int win_l = -1) {
+DecodePlan decode_plan(int B, int Hkv, int D, int max_pages, int Nq, int win_l, int override_pages) {
   DecodePlan pl;
   // kv heads per CTA: the largest divisor of Hkv whose token row (heads x D x 2 bytes) fits in
   // 1 KB, so that a 3-stage K+V page ring stays near 100 KB and two CTAs share an SM (one
@@ -132,8 +136,8 @@ DecodePlan decode_plan(int B, int Hkv, int D, int max_pages, int Nq = 1, int win
     }
   pl.groups = Hkv / pl.heads_per_cta;
   int s = 32;
-  if (g_split_pages_override > 0) {
-    s = std::min(g_split_pages_override, mfa::kDecMaxSplitPages);
+  if (override_pages > 0) {
+    s = std::min(override_pages, mfa::kDecMaxSplitPages);
   } else {
     // halve the split while the grid would hold fewer than two CTAs per SM (148 SMs)
     while (s > 4 && (long long)B * ((max_pages + s - 1) / s) * pl.groups < 296) s /= 2;
@@ -144,7 +148,7 @@ DecodePlan decode_plan(int B, int Hkv, int D, int max_pages, int Nq = 1, int win
     const long long win_pages = ((long long)win_l + Nq + mfa::kDecPage - 1) / mfa::kDecPage + 1;
     const int span = (int)std::min<long long>(max_pages, win_pages);
     const int cap = pl.max_splits;
-    if (g_split_pages_override <= 0) {
+    if (override_pages <= 0) {
       s = 32;
       while (s > 4 && (long long)B * ((span + s / 2 - 1) / (s / 2)) * pl.groups <= 296 &&
              (span + s / 2 - 1) / (s / 2) <= cap)
@@ -338,6 +342,18 @@ int validate_fwd_common(int Hq, int Hkv, int D, int dtype, int win_l, int win_r,
   return MFA_OK;
 }
 
+// A window wider than any sequence of the call is the same as no bound on that side; it is
+// replaced by -1 before launch, so the kernels' 32-bit position arithmetic (a - win_l,
+// a + win_r + 1, with positions below 2^30) cannot wrap around for windows near INT_MAX.
+// max_k bounds every key count of the call and max_q every query count.
+void clamp_window(int& win_l, int& win_r, long long max_k, long long max_q) {
+  if (win_l >= max_k) win_l = -1;
+  if (win_r >= max_q) win_r = -1;
+}
+
+// Sequence lengths the kernels index with 32-bit positions.
+constexpr long long kMaxTokens = 0x3fffffffLL;
+
 // Every row sees no key: out = 0, lse = -inf (rows = number of (query, head) pairs).
 int launch_fill_empty(void* out, float* lse, size_t rows, int D, int dtype, cudaStream_t st) {
   if (dtype == MFA_DTYPE_BF16)
@@ -437,12 +453,14 @@ int mfa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, 
   if ((rc = check_sizes(B, Hq, Nq, D)) != MFA_OK) return rc;
   if ((rc = check_sizes(B, Hkv, Nk, D)) != MFA_OK) return rc;
   if ((long long)B * Hq > 0x7FFFFFFFLL || (long long)B * Hkv > 0x7FFFFFFFLL) return MFA_ERR_BAD_SHAPE;
+  if (Nq > kMaxTokens || Nk > kMaxTokens) return MFA_ERR_BAD_SHAPE;
   if (B == 0 || Hq == 0 || Nq == 0) return MFA_OK;
   if (!q || !out || (Nk > 0 && (!k || !v))) return MFA_ERR_NULL_POINTER;
   if (!aligned16(q) || !aligned16(out) || !aligned16(lse) || (Nk > 0 && (!aligned16(k) || !aligned16(v))))
     return MFA_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (Nk == 0) return launch_fill_empty(out, lse, (size_t)B * Hq * Nq, D, dtype, st);
+  clamp_window(win_l, win_r, Nk, Nq);
   FwdCall c = {q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, scale, causal, win_l, win_r, softcap, dtype,
                nullptr, nullptr, 0, 0, nullptr, nullptr, nullptr, 0, 0};
   return dispatch_fwd<false, false>(c, D, st);
@@ -459,12 +477,14 @@ int mfa_fwd_blocksparse(const void* q, const void* k, const void* v, void* out, 
   if ((rc = check_sizes(B, Hkv, Nk, D)) != MFA_OK) return rc;
   if ((long long)B * Hq > 0x7FFFFFFFLL || (long long)B * Hkv > 0x7FFFFFFFLL) return MFA_ERR_BAD_SHAPE;
   if ((long long)(Nk + mfa::kFwdBN - 1) / mfa::kFwdBN > mfa::kFwdMaxSparseTiles) return MFA_ERR_UNSUPPORTED;
+  if (Nq > kMaxTokens || Nk > kMaxTokens) return MFA_ERR_BAD_SHAPE;
   if (B == 0 || Hq == 0 || Nq == 0) return MFA_OK;
   if (!q || !out || !block_mask || (Nk > 0 && (!k || !v))) return MFA_ERR_NULL_POINTER;
   if (!aligned16(q) || !aligned16(out) || !aligned16(lse) || (Nk > 0 && (!aligned16(k) || !aligned16(v))))
     return MFA_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (Nk == 0) return launch_fill_empty(out, lse, (size_t)B * Hq * Nq, D, dtype, st);
+  clamp_window(win_l, win_r, Nk, Nq);
   FwdCall c = {q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, scale, causal, win_l, win_r, softcap, dtype,
                nullptr, nullptr, 0, 0, block_mask, nullptr, nullptr, 0, 0};
   return dispatch_fwd<false, true>(c, D, st);
@@ -481,6 +501,7 @@ int mfa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float
   if ((rc = check_sizes(total_q, Hq, D, 1)) != MFA_OK) return rc;
   if ((rc = check_sizes(total_k, Hkv, D, 1)) != MFA_OK) return rc;
   if ((long long)B * Hq > 0x7FFFFFFFLL) return MFA_ERR_BAD_SHAPE;
+  if (total_q > kMaxTokens || total_k > kMaxTokens) return MFA_ERR_BAD_SHAPE;
   if (B == 0 || Hq == 0 || total_q == 0 || max_seqlen_q == 0) return MFA_OK;
   if (!q || !out || !cu_seqlens_q || !cu_seqlens_k || (total_k > 0 && (!k || !v)))
     return MFA_ERR_NULL_POINTER;
@@ -490,6 +511,7 @@ int mfa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float
     return MFA_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (total_k == 0) return launch_fill_empty(out, lse, (size_t)total_q * Hq, D, dtype, st);
+  clamp_window(win_l, win_r, total_k, total_q);
   FwdCall c = {q, k, v, out, lse, B, Hq, Hkv, max_seqlen_q, 0, scale, causal, win_l, win_r, softcap,
                dtype, cu_seqlens_q, cu_seqlens_k, total_q, total_k, nullptr, nullptr, nullptr, 0, 0};
   return dispatch_fwd<true, false>(c, D, st);
@@ -510,7 +532,7 @@ int mfa_fwd_paged(const void* q, const void* k_pages, const void* v_pages, const
   if ((rc = check_sizes(num_pages, page_size, Hkv, D)) != MFA_OK) return rc;
   if ((long long)max_pages_per_seq * 16 > 0x3fffffffLL || (long long)num_pages * 16 > 0x3fffffffLL)
     return MFA_ERR_BAD_SHAPE;
-  if ((long long)B * Hq > 0x7FFFFFFFLL) return MFA_ERR_BAD_SHAPE;
+  if ((long long)B * Hq > 0x7FFFFFFFLL || total_q > kMaxTokens) return MFA_ERR_BAD_SHAPE;
   if (B == 0 || Hq == 0 || total_q == 0 || max_seqlen_q == 0) return MFA_OK;
   if (!q || !out || !k_pages || !v_pages || !block_table || !seq_lens || !cu_seqlens_q)
     return MFA_ERR_NULL_POINTER;
@@ -519,6 +541,7 @@ int mfa_fwd_paged(const void* q, const void* k_pages, const void* v_pages, const
       (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u))
     return MFA_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  clamp_window(win_l, win_r, (long long)max_pages_per_seq * 16, total_q);
   FwdCall c = {q, k_pages, v_pages, out, lse, B, Hq, Hkv, max_seqlen_q, 0, scale, causal, win_l, win_r,
                softcap, dtype, cu_seqlens_q, nullptr, total_q, 0, nullptr, block_table, seq_lens,
                max_pages_per_seq, num_pages};
@@ -553,7 +576,9 @@ int mfa_bwd(const void* q, const void* k, const void* v, const void* out, const 
   if ((rc = check_sizes(B, Hq, Nq, D)) != MFA_OK) return rc;
   if ((rc = check_sizes(B, Hkv, Nk, D)) != MFA_OK) return rc;
   if ((long long)B * Hq > 0x7FFFFFFFLL || (long long)B * Hkv > 0x7FFFFFFFLL) return MFA_ERR_BAD_SHAPE;
+  if (Nq > kMaxTokens || Nk > kMaxTokens) return MFA_ERR_BAD_SHAPE;
   if (B == 0 || Hq == 0 || (Nq == 0 && Nk == 0)) return MFA_OK;
+  clamp_window(win_l, win_r, Nk, Nq);
   const bool need_q = Nq > 0, need_k = Nk > 0;
   if ((need_q && (!q || !out || !dout || !lse || !dq)) || (need_k && (!k || !v || !dk || !dv)))
     return MFA_ERR_NULL_POINTER;
@@ -610,27 +635,32 @@ int mfa_decode_plan(int B, int Nq, int Hq, int Hkv, int D, int max_pages_per_seq
   if (win_l < -1) return MFA_ERR_BAD_WINDOW;
   const int rc = validate_decode(B, Nq, Hq, Hkv, D, page_size, max_pages_per_seq);
   if (rc != MFA_OK) return rc;
-  const DecodePlan pl = decode_plan(B, Hkv, D, max_pages_per_seq, Nq, win_l);
+  const DecodePlan pl = decode_plan(B, Hkv, D, max_pages_per_seq, Nq, win_l, g_split_pages_override.load());
   if (pages_per_split) *pages_per_split = pl.pages_per_split;
   if (max_splits) *max_splits = pl.max_splits;
   if (kv_heads_per_cta) *kv_heads_per_cta = pl.heads_per_cta;
   return MFA_OK;
 }
 
-size_t mfa_decode_workspace_size(int B, int Nq, int Hq, int Hkv, int D, int max_pages_per_seq,
-                                 int page_size) {
+}  // extern "C"
+
+namespace {
+
+size_t decode_workspace_size(int B, int Nq, int Hq, int Hkv, int D, int max_pages_per_seq,
+                             int page_size, int override_pages) {
   if (validate_decode(B, Nq, Hq, Hkv, D, page_size, max_pages_per_seq) != MFA_OK) return 0;
-  DecodePlan pl = decode_plan(B, Hkv, D, max_pages_per_seq);
+  DecodePlan pl = decode_plan(B, Hkv, D, max_pages_per_seq, 1, -1, override_pages);
   const size_t rows = (size_t)B * pl.max_splits * Hq * Nq;
   return align256(rows * D * sizeof(float)) + align256(rows * 2 * sizeof(float));
 }
 
-int mfa_decode_splitkv_window(const void* q, const void* k_pages, const void* v_pages,
-                              const int32_t* block_table, const int32_t* seq_lens, void* out,
-                              float* lse, int B, int Nq, int Hq, int Hkv, int D, int page_size,
-                              int max_pages_per_seq, int num_pages, float scale, int causal,
-                              int win_l, float softcap, int dtype, void* workspace,
-                              size_t workspace_bytes, void* stream) {
+// The decode entry points after their override read: override_pages is the split-size override
+// this call uses for both the workspace check and the launched plan.
+int decode_splitkv(const void* q, const void* k_pages, const void* v_pages,
+                   const int32_t* block_table, const int32_t* seq_lens, void* out, float* lse,
+                   int B, int Nq, int Hq, int Hkv, int D, int page_size, int max_pages_per_seq,
+                   int num_pages, float scale, int causal, int win_l, float softcap, int dtype,
+                   void* workspace, size_t workspace_bytes, cudaStream_t st, int override_pages) {
   if (dtype != MFA_DTYPE_FP16 && dtype != MFA_DTYPE_BF16) return MFA_ERR_BAD_DTYPE;
   if (win_l < -1) return MFA_ERR_BAD_WINDOW;
   int rc = validate_decode(B, Nq, Hq, Hkv, D, page_size, max_pages_per_seq);
@@ -645,10 +675,10 @@ int mfa_decode_splitkv_window(const void* q, const void* k_pages, const void* v_
   if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(block_table) ||
       !aligned16(seq_lens) || !aligned16(out) || !aligned16(lse))
     return MFA_ERR_MISALIGNED;
-  const size_t need = mfa_decode_workspace_size(B, Nq, Hq, Hkv, D, max_pages_per_seq, page_size);
+  const size_t need = decode_workspace_size(B, Nq, Hq, Hkv, D, max_pages_per_seq, page_size, override_pages);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
     return MFA_ERR_WORKSPACE;
-  DecodePlan pl = decode_plan(B, Hkv, D, max_pages_per_seq, Nq, win_l);
+  DecodePlan pl = decode_plan(B, Hkv, D, max_pages_per_seq, Nq, win_l, override_pages);
   mfa::DecodeParams p;
   std::memset(&p, 0, sizeof(p));
   p.q = static_cast<const uint16_t*>(q);
@@ -682,11 +712,32 @@ int mfa_decode_splitkv_window(const void* q, const void* k_pages, const void* v_
     p.c_log2 = scale * log2e;
   }
   if (pl.max_splits > 0x7FFFFFFF || B > 65535 || pl.groups > 65535) return MFA_ERR_BAD_SHAPE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool bf = dtype == MFA_DTYPE_BF16;
   if (D == 256) return bf ? launch_decode<256, true>(p, pl, st) : launch_decode<256, false>(p, pl, st);
   if (D == 128) return bf ? launch_decode<128, true>(p, pl, st) : launch_decode<128, false>(p, pl, st);
   return bf ? launch_decode<64, true>(p, pl, st) : launch_decode<64, false>(p, pl, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mfa_decode_workspace_size(int B, int Nq, int Hq, int Hkv, int D, int max_pages_per_seq,
+                                 int page_size) {
+  return decode_workspace_size(B, Nq, Hq, Hkv, D, max_pages_per_seq, page_size,
+                               g_split_pages_override.load());
+}
+
+int mfa_decode_splitkv_window(const void* q, const void* k_pages, const void* v_pages,
+                              const int32_t* block_table, const int32_t* seq_lens, void* out,
+                              float* lse, int B, int Nq, int Hq, int Hkv, int D, int page_size,
+                              int max_pages_per_seq, int num_pages, float scale, int causal,
+                              int win_l, float softcap, int dtype, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  return decode_splitkv(q, k_pages, v_pages, block_table, seq_lens, out, lse, B, Nq, Hq, Hkv, D,
+                        page_size, max_pages_per_seq, num_pages, scale, causal, win_l, softcap,
+                        dtype, workspace, workspace_bytes, static_cast<cudaStream_t>(stream),
+                        g_split_pages_override.load());
 }
 
 int mfa_decode_splitkv(const void* q, const void* k_pages, const void* v_pages,
@@ -768,9 +819,7 @@ int mfa_debug_tiles_visited(void* stream, unsigned long long* count) {
 }
 
 int mfa_debug_set_decode_split_pages(int pages) {
-  int old = g_split_pages_override;
-  g_split_pages_override = pages < 0 ? 0 : pages;
-  return old;
+  return g_split_pages_override.exchange(pages < 0 ? 0 : pages);
 }
 
 }  // extern "C"
@@ -805,21 +854,24 @@ extern "C" int mfa_decode_splitkv_noalloc(const void* q, const void* k_pages, co
                                           int D, int page_size, int max_pages_per_seq,
                                           int num_pages, float scale, int causal, float softcap,
                                           int dtype, void* stream) {
-  // Every argument check of mfa_decode_splitkv runs first; with no workspace it returns before
-  // any launch, and MFA_ERR_WORKSPACE then means that everything else is valid.
-  int rc = mfa_decode_splitkv(q, k_pages, v_pages, block_table, seq_lens, out, lse, B, Nq, Hq,
-                              Hkv, D, page_size, max_pages_per_seq, num_pages, scale, causal,
-                              softcap, dtype, nullptr, 0, stream);
+  // one read of the split-size override serves the size check and the launch
+  const int ovr = g_split_pages_override.load();
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Every argument check of the decode runs first; with no workspace it returns before any
+  // launch, and MFA_ERR_WORKSPACE then means that everything else is valid.
+  int rc = decode_splitkv(q, k_pages, v_pages, block_table, seq_lens, out, lse, B, Nq, Hq, Hkv, D,
+                          page_size, max_pages_per_seq, num_pages, scale, causal, -1, softcap,
+                          dtype, nullptr, 0, st, ovr);
   if (rc != MFA_ERR_WORKSPACE) return rc;
-  const size_t need = mfa_decode_workspace_size(B, Nq, Hq, Hkv, D, max_pages_per_seq, page_size);
+  const size_t need = decode_workspace_size(B, Nq, Hq, Hkv, D, max_pages_per_seq, page_size, ovr);
   if (need > kNoAllocScratchBytes) return MFA_ERR_SCRATCH_TOO_SMALL;
   const int dev = current_device();
   if (dev < 0) return MFA_ERR_CUDA;
   void* scratch = noalloc_scratch(dev);
   if (scratch == nullptr) return MFA_ERR_CUDA;
-  return mfa_decode_splitkv(q, k_pages, v_pages, block_table, seq_lens, out, lse, B, Nq, Hq, Hkv,
-                            D, page_size, max_pages_per_seq, num_pages, scale, causal, softcap,
-                            dtype, scratch, kNoAllocScratchBytes, stream);
+  return decode_splitkv(q, k_pages, v_pages, block_table, seq_lens, out, lse, B, Nq, Hq, Hkv, D,
+                        page_size, max_pages_per_seq, num_pages, scale, causal, -1, softcap, dtype,
+                        scratch, kNoAllocScratchBytes, st, ovr);
 }
 
 // ----------------------------------------------------------------------------------------------
