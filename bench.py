@@ -31,6 +31,16 @@ sys.path.insert(0, ROOT)
 import mfa_inputs as mi  # noqa: E402
 
 MAIN = "causal_b2_h8_n4096_d128_fp16"
+# The pages' own forward timings on an Apple M1 Max (f16, "mlx-mfa 2.5.2", Performance tables:
+# the dense causal table and the sliding-window table), for the workloads of the same shape.
+# Context only: another machine, another kernel.
+PAGES_M1_MAX_MS = {
+    "causal_b2_h8_n4096_d128_fp16": 11.5,
+    "causal_b2_h8_n8192_d128_fp16": 44.1,
+    "window512_b2_h8_n8192_d128_fp16": 6.2,
+    "window256_b2_h8_n8192_d128_fp16": 3.6,
+}
+PAGES_SOURCE = "mlx-mfa 2.5.2, Performance tables (Apple M1 Max, f16, ms per forward)"
 METRIC = "attention TFLOP/s (prefill) and KV GB/s (split-KV decode) vs B200 peak"
 NOMINAL_TFLOPS = 2250.0
 NOMINAL_GBS = 8000.0
@@ -205,6 +215,23 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
+def main_config(name: str, world: int) -> dict:
+    """The `config` of the headline line, shared by the GPU arm and the reference arm."""
+    c = mi.workloads()[name]
+    return {"workload": name, "B": c.B, "Hq": c.Hq, "Hkv": c.Hkv, "N": c.Nq, "D": c.D,
+            "causal": c.causal, "window": [c.win_l, c.win_r], "softcap": c.softcap,
+            "dtype": mi.DTYPE_NAMES[c.dtype],
+            "l2": "flushed before every timed step (256 MiB write)",
+            "parallelism": f"replica per GPU x{world}"}
+
+
+def pages_context(name: str) -> dict:
+    """The pages' M1 Max time for this workload's shape, when they print one."""
+    if name not in PAGES_M1_MAX_MS:
+        return {}
+    return {"pages_m1_max_ms": PAGES_M1_MAX_MS[name], "pages_source": PAGES_SOURCE}
+
+
 # --------------------------------------------------------------------------- GPU arm
 def upload(bits, dtype, dev):
     import torch
@@ -328,6 +355,28 @@ def bench_prefill(case, steps, warmup, flush, stream, with_e2e, world):
     return res
 
 
+def host_call_us(case, stream, calls=2000):
+    """Host time of one forward call through the Python binding and the C ABI (argument checks,
+    tensor maps from the library's cache, the launch), averaged over back-to-back calls."""
+    import torch
+    import tiled_exact_attention_mfa_b200 as mfa
+    dev = torch.device("cuda")
+    qt, kt, vt = (upload(x, case.dtype, dev) for x in case.tensors())
+    out = torch.empty_like(qt)
+    lse = torch.empty(case.B, case.Hq, case.Nq, dtype=torch.float32, device=dev)
+    kw = dict(scale=case.scale_f32(), causal=case.causal, window=(case.win_l, case.win_r),
+              softcap=case.softcap, stream=stream)
+    for _ in range(20):
+        mfa.mfa_fwd(qt, kt, vt, out, lse, **kw)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(calls):
+        mfa.mfa_fwd(qt, kt, vt, out, lse, **kw)
+    dt = time.perf_counter() - t0
+    torch.cuda.synchronize()
+    return round(dt / calls * 1e6, 2)
+
+
 def bench_varlen(case, steps, warmup, flush, stream, world):
     import torch
     import tiled_exact_attention_mfa_b200 as mfa
@@ -388,7 +437,7 @@ def bench_backward(case, steps, warmup, flush, stream, world):
     win = (case.win_l, case.win_r)
     out, lse = mfa.mfa_fwd(qt, kt, vt, scale=case.scale_f32(), causal=case.causal, window=win,
                            softcap=case.softcap, stream=stream)
-    dout = upload(mi.normal_bits(case.seed + 500, mi.STREAM_Q, tuple(qt.shape), case.dtype),
+    dout = upload(case.dout(),
                   case.dtype, dev)
     dq, dk, dv = torch.empty_like(qt), torch.empty_like(kt), torch.empty_like(vt)
     ws = torch.empty(max(mfa.mfa_bwd_workspace_size(case.B, case.Hq, case.Nq), 256),
@@ -538,6 +587,8 @@ def run_gpu(args):
                                "tflops": round(r["flops"] * world / (r["ms"] * 1e-3) / 1e12, 2)})
             else:
                 r = bench_prefill(case, sk, wu, flush, stream, False, world)
+                if name == "causal_b1_h2_n128_d64_fp16":
+                    r["host_us"] = host_call_us(case, stream)
                 tf = r["flops"] * world / (r["ms"] * 1e-3) / 1e12
                 gbs = r["bytes"] * world / (r["ms"] * 1e-3) / 1e9
                 t_floor = max(r["flops"] / (pk["tflops"] * 1e12), r["bytes"] / (pk["gbs"] * 1e9))
@@ -546,7 +597,9 @@ def run_gpu(args):
                                "frac_of_measured_tensor_peak": round(tf / pk["tflops"], 4),
                                "frac_of_nominal_tensor_peak": round(tf / NOMINAL_TFLOPS, 4),
                                "frac_of_roofline": round(t_floor / (r["ms"] * 1e-3), 4),
-                               "traffic": ncu_traffic(name, "mfa_fwd_kernel")})
+                               "traffic": ncu_traffic(name, "mfa_fwd_kernel"),
+                               **({"host_us_per_call": r["host_us"]} if "host_us" in r else {}),
+                               **pages_context(name)})
             getattr(case, "_cache", {}).clear()  # the workload's host inputs are not needed again
         for name in BACKWARD_WORKLOADS:
             sk, wu = max(3, min(args.steps, 10)), max(3, args.warmup)
@@ -574,10 +627,9 @@ def run_gpu(args):
         "vs_baseline": None,
         "dtype": mi.DTYPE_NAMES[main_case.dtype],
         "data": "synthetic (seeded N(0,1) Q/K/V, SplitMix64 + Box-Muller)",
-        "config": {"workload": args.workload, "B": main_case.B, "Hq": main_case.Hq,
-                   "Hkv": main_case.Hkv, "N": main_case.Nq, "D": main_case.D,
-                   "causal": main_case.causal, "l2": "flushed before every timed step (256 MiB write)",
-                   "parallelism": f"replica per GPU x{world}"},
+        "config": main_config(args.workload, world),
+        "context": {**pages_context(args.workload),
+                    "note": "the pages' own timing on Apple hardware, for context; not a target"},
         "roofline": {"bound": "tensor", "achieved": round(per_gpu_tflops, 2),
                      "peak": pk["tflops"], "unit": "TFLOP/s",
                      "frac": round(per_gpu_tflops / pk["tflops"], 4),
@@ -644,29 +696,41 @@ def cpu_baseline(case, budget_s: float = 15.0):
 
 
 def run_reference(args):
+    """The reference arm: the fp64 oracle as it stands, timed over whole steps of the named
+    workload (every head, every row) on the host cores. Rank 0 alone runs it."""
+    import oracle
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     case = mi.workloads()[args.workload]
-    budget = max(1.0, min(20.0, args.cpu_seconds / max(1, args.steps)))
+    q, k, v = case.tensors()
+    w = lambda x: mi.widen(x, case.dtype)
+    qd, kd, vd = w(q), w(k), w(v)
+
+    def step():
+        oracle.attention(qd, kd, vd, case.scale_f32(), case.causal, case.win_l, case.win_r,
+                         case.softcap)
+
     for _ in range(args.warmup):
-        cpu_baseline(case, budget_s=0.1)
-    vals = []
-    last = None
+        step()
+    ms = []
     for _ in range(args.steps):
-        last = cpu_baseline(case, budget_s=budget)
-        vals.append(last["value"])
-    value = statistics.mean(vals)
-    ms = 4.0 * case.D * visible_pairs(case) * case.B * case.Hq / (value * 1e12) * 1e3
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        t0 = time.perf_counter()
+        step()
+        ms.append((time.perf_counter() - t0) * 1e3)
+    mean_ms = statistics.mean(ms)
+    value = prefill_flops(case) / (mean_ms * 1e-3) / 1e12
+    sample = (f"whole steps: all {case.B * case.Hq} (b,h) heads x {case.Nq} rows of {case.name} "
+              f"per step, fp64 numpy, {mean_ms / 1e3:.2f} s per step")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload},
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": last["cores"],
-                             "kind": "oracle", "sample": last["sample"]},
-            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+            "ms_per_step": round(mean_ms, 3), **spread(ms), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": main_config(args.workload, world),
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 

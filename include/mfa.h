@@ -36,6 +36,12 @@
  *     or approximate answer.
  *   - Kernels bound every internal wait; a wait that runs out, or an out-of-range block_table
  *     entry, records a device status that mfa_device_status() returns.
+ *   - The TMA tensor maps a launch needs are cached inside the library per device, keyed by
+ *     (base pointer, data type, layout, extents), 256 of them with the least recently used one
+ *     replaced; repeated calls over the same buffers encode no map (mfa_debug_tmap_stats).
+ *   - Windows (win_l, win_r) at least as wide as every sequence of the call mean the same as -1
+ *     and are treated as -1, so INT_MAX is a valid "unbounded" value; sequence lengths are below
+ *     2^30.
  */
 #ifndef MFA_H_
 #define MFA_H_
@@ -358,6 +364,23 @@ int mfa_debug_set_flags(int flags);
 
 /* Reads and resets the tile counter (synchronises `stream`). */
 int mfa_debug_tiles_visited(void* stream, unsigned long long* count);
+
+/*
+ * Tensor-map cache counters: map lookups made by launches so far and how many of them had to
+ * encode a map (cuTensorMapEncodeTiled) because no map of the same (device, base pointer, data
+ * type, layout, extents) was cached. A second call over the same buffers encodes nothing.
+ */
+int mfa_debug_tmap_stats(unsigned long long* lookups, unsigned long long* encodes);
+
+/*
+ * Host-only check of the tensor-map cache (no GPU or driver needed): looks up the key (base,
+ * kind 0 dense / 1 packed / 2 pages, dtype, outer, n, D) under a device number no launch uses,
+ * encoding a placeholder map on a miss. *encoded = 1 on a miss, 0 on a hit; the counters of
+ * mfa_debug_tmap_stats include these lookups. Returns MFA_OK, or MFA_ERR_CUDA if a hit returned
+ * a map built for another key.
+ */
+int mfa_debug_tmap_probe(const void* base, int kind, int dtype, long long outer, long long n, int D,
+                         int* encoded);
 
 /*
  * Decode split size override in pages (0 = automatic, at most 64). It changes the split plan,

@@ -140,6 +140,11 @@ class PrefillCase:
         s = self.scale if self.scale is not None else 1.0 / np.sqrt(self.D)
         return float(np.float32(s))
 
+    def dout(self):
+        """The output gradient dO for the backward, [B,Hq,Nq,D] bit patterns: N(0,1) from seed + 500
+        (stream 0)."""
+        return normal_bits(self.seed + 500, STREAM_Q, (self.B, self.Hq, self.Nq, self.D), self.dtype)
+
     def tensors(self):
         """(q, k, v) as uint16 bit patterns."""
         q = normal_bits(self.seed, STREAM_Q, (self.B, self.Hq, self.Nq, self.D), self.dtype, self.mul)
@@ -418,6 +423,9 @@ def workloads():
             "causal_b2_h8_n4096_d128_fp16", 2, 8, 8, 4096, 4096, 128, FP16, True, seed=1002),
         "noncausal_b2_h8_n4096_d128_fp16": PrefillCase(
             "noncausal_b2_h8_n4096_d128_fp16", 2, 8, 8, 4096, 4096, 128, FP16, False, seed=1002),
+        # the causal shape of the window workloads (and their inputs), without a window
+        "causal_b2_h8_n8192_d128_fp16": PrefillCase(
+            "causal_b2_h8_n8192_d128_fp16", 2, 8, 8, 8192, 8192, 128, FP16, True, seed=1003),
         "window512_b2_h8_n8192_d128_fp16": PrefillCase(
             "window512_b2_h8_n8192_d128_fp16", 2, 8, 8, 8192, 8192, 128, FP16, True, 512, 0,
             seed=1003),

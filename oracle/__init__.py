@@ -192,10 +192,12 @@ def _block_visibility(block_mask, b, h, Nq, Nk, block):
 
 
 def attention_blocksparse(q, k, v, block_mask, scale, causal=False, win_l=-1, win_r=-1,
-                          softcap=0.0, block=128):
+                          softcap=0.0, block=128, row_block=512):
     """Block-sparse forward: the dense definition with visibility vis(i, j) AND
     block_mask[b, h, i // block, j // block] != 0. q [B,Hq,Nq,D], k/v [B,Hkv,Nk,D],
-    block_mask [B, Hq, ceil(Nq/block), ceil(Nk/block)]. Returns (o [B,Hq,Nq,D], lse [B,Hq,Nq])."""
+    block_mask [B, Hq, ceil(Nq/block), ceil(Nk/block)]. Returns (o [B,Hq,Nq,D], lse [B,Hq,Nq]).
+    Rows are independent; they are taken row_block at a time (as in attention) so that the
+    score block stays row_block x Nk."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -208,8 +210,10 @@ def attention_blocksparse(q, k, v, block_mask, scale, causal=False, win_l=-1, wi
     for b in range(B):
         for h in range(Hq):
             vb = vis & _block_visibility(block_mask, b, h, Nq, Nk, block)
-            o[b, h], lse[b, h] = _rows_for_head(q[b, h], k[b, h // G], v[b, h // G], vb, scale,
-                                                softcap)
+            for r0 in range(0, Nq, row_block):
+                r1 = min(Nq, r0 + row_block)
+                o[b, h, r0:r1], lse[b, h, r0:r1] = _rows_for_head(
+                    q[b, h, r0:r1], k[b, h // G], v[b, h // G], vb[r0:r1], scale, softcap)
     return o, lse
 
 

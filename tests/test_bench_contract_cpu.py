@@ -13,12 +13,20 @@ def run_ref(extra_env=None):
     env = dict(os.environ)
     env.update(extra_env or {})
     return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                           "--steps", "1", "--warmup", "3", "--cpu-seconds", "1"],
+                           "--steps", "2", "--warmup", "3", "--workload", SMALL],
                           capture_output=True, text=True, env=env, cwd=ROOT, timeout=600)
 
 
+SMALL = "causal_b1_h2_n128_d64_fp16"
+
+
 def test_reference_arm_prints_one_contract_line():
+    """Whole steps of the named workload are timed, so steps x ms_per_step fits inside the run,
+    and the line carries the same config as the GPU arm's."""
+    import time
+    t0 = time.perf_counter()
     r = run_ref({"RANK": "0", "WORLD_SIZE": "1"})
+    wall_ms = (time.perf_counter() - t0) * 1e3
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
     assert len(lines) == 1
@@ -30,7 +38,11 @@ def test_reference_arm_prints_one_contract_line():
     assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "TFLOP/s"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
-    assert d["config"]["workload"] == "causal_b2_h8_n4096_d128_fp16"
+    sys.path.insert(0, ROOT)
+    import bench
+    assert d["config"] == bench.main_config(SMALL, 1)
+    assert d["steps"] * d["ms_per_step"] < wall_ms
+    assert "whole steps" in d["cpu_baseline"]["sample"]
 
 
 def test_reference_arm_other_ranks_exit_quietly():

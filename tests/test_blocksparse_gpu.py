@@ -127,16 +127,10 @@ def test_visited_tiles_and_tile_skip_neutrality(cuda_device):
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
 
 
-def test_full_size_spatial_workload_sampled_rows(cuda_device):
+def test_full_size_spatial_workload_every_element(cuda_device):
+    from oracle import cache
     case = mi.workloads()["sparse_spatial2d_b1_h16_n16384_d128_fp16"]
     q, k, v, m = case.tensors()
     o, lse = run_gpu(case, q, k, v, m)
-    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
-    rng = np.random.default_rng(1)
-    rows = np.array([(0, h, int(i)) for h in range(case.Hq)
-                     for i in sorted({0, 127, 128, 8191, 16383} | set(rng.integers(0, case.N, 10).tolist()))])
-    w = lambda x: mi.widen(x, case.dtype)
-    o_ref, l_ref = oracle.attention_blocksparse_rows(w(q), w(k), w(v), m, rows, case.scale_f32(),
-                                                     case.causal)
-    sel = (rows[:, 0], rows[:, 1], rows[:, 2])
-    check_close(o[sel], lse[sel], o_ref, l_ref, case.dtype, case.name)
+    ref = cache.reference(case.name, (q, k, v, m))
+    check_close(o, lse, ref["o"], ref["lse"], case.dtype, case.name)

@@ -282,3 +282,26 @@ def test_fwd_host_scratch_size():
 @no_device
 def test_fwd_host_empty_problem_is_a_no_op():
     assert fwdh(B=0, q=None, k=None, v=None, out=None, lse=None, ws=None) == 0
+
+
+def test_tensor_map_cache_hits_the_second_time():
+    """The tensor-map cache, host only (placeholder maps): a key's first lookup encodes, the
+    second with the same key encodes nothing, any changed field is a new key, and after more
+    than the cache's 256 distinct keys the least recently used one has been replaced."""
+    base = 0x7F0000100000
+    before = mfa.mfa_debug_tmap_stats()
+    assert mfa.mfa_debug_tmap_probe(base, 0, 0, 16, 4096, 128)
+    assert not mfa.mfa_debug_tmap_probe(base, 0, 0, 16, 4096, 128)
+    after = mfa.mfa_debug_tmap_stats()
+    assert after["lookups"] - before["lookups"] == 2
+    assert after["encodes"] - before["encodes"] == 1
+    for changed in ((base + 256, 0, 0, 16, 4096, 128), (base, 1, 0, 16, 4096, 128),
+                    (base, 0, 1, 16, 4096, 128), (base, 0, 0, 8, 4096, 128),
+                    (base, 0, 0, 16, 4095, 128), (base, 0, 0, 16, 4096, 64)):
+        assert mfa.mfa_debug_tmap_probe(*changed), changed
+        assert not mfa.mfa_debug_tmap_probe(*changed), changed
+    # keep the first key recently used while 300 other keys pass through: it stays, the oldest go
+    for i in range(300):
+        mfa.mfa_debug_tmap_probe(base + 4096 * (i + 1), 2, 1, 8, 16 * 1024, 128)
+        assert not mfa.mfa_debug_tmap_probe(base, 0, 0, 16, 4096, 128)
+    assert mfa.mfa_debug_tmap_probe(base + 4096, 2, 1, 8, 16 * 1024, 128)  # evicted long ago

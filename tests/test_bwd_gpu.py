@@ -32,7 +32,7 @@ CASES = [
 
 
 def dout_bits(case):
-    return mi.normal_bits(case.seed + 500, mi.STREAM_Q, (case.B, case.Hq, case.Nq, case.D), case.dtype)
+    return case.dout()
 
 
 def run(case):
@@ -67,6 +67,24 @@ def check(case, inputs, grads):
 def test_backward_matches_oracle(cuda_device, case):
     inputs, grads = run(case)
     check(case, inputs, grads)
+
+
+@pytest.mark.parametrize("name", ["causal_b2_h8_n4096_d128_fp16",
+                                  "noncausal_b2_h8_n4096_d128_fp16"])
+def test_full_size_backward_every_element(cuda_device, name):
+    """The backward of the B=2 H=8 N=4096 D=128 workloads, every element of dq / dk / dv against
+    the oracle's gradients (cached), at the bound above."""
+    from oracle import cache
+    case = mi.workloads()[name]
+    inputs, grads = run(case)
+    ref = cache.reference(name + ":backward", inputs[:3])
+    for gname, g in zip(("dq", "dk", "dv"), grads):
+        r = ref[gname]
+        assert np.all(np.isfinite(g)), f"{name}: non-finite {gname}"
+        err = float(np.max(np.abs(g - r)))
+        bound = TOL[case.dtype] * max(float(np.max(np.abs(r))), 1e-6)
+        print(f"{name} {gname}: max err {err:.3e}  max |ref| {np.max(np.abs(r)):.3e}  bound {bound:.3e}")
+        assert err <= bound, f"{name}: max |{gname} - oracle| = {err:.3e} > {bound:.3e}"
 
 
 def test_backward_is_deterministic_and_empty_rows_get_zero_dq(cuda_device):

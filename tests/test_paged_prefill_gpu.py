@@ -51,6 +51,19 @@ def test_paged_prefill_matches_oracle(cuda_device, case):
     assert mfa.mfa_device_status() == (0, 0)
 
 
+def test_full_size_paged_prefill_every_element(cuda_device):
+    """The chunked-prefill workload (8 sequences, 4k-32k cached keys in a permuted page pool,
+    chunks of up to 2048 queries) against the oracle, every element (cached)."""
+    import tiled_exact_attention_mfa_b200 as mfa
+    from oracle import cache
+    case = mi.workloads()["paged_prefill_b8_hq32_hkv8_d128_bf16_ctx4k_32k"]
+    q, kp, vp, table, lens, cq = case.tensors()
+    o, lse = run_gpu(case, q, kp, vp, table, lens, cq)
+    ref = cache.reference(case.name, (q, kp, vp, table, lens, cq))
+    check_close(o, lse, ref["o"], ref["lse"], case.dtype, case.name)
+    assert mfa.mfa_device_status() == (0, 0)
+
+
 def test_short_chunks_equal_split_kv_decode(cuda_device):
     """With 1-4 queries per sequence, the paged prefill and the split-KV decode compute the same
     definition: both within the tolerance of the oracle and of each other."""

@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(_HERE, "libmfa.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it first (python -m tiled_exact_attention_mfa_b200.build "
+        f"{LIB_PATH} is missing: build it first (python tiled_exact_attention_mfa_b200/build.py "
         "or __graft_entry__.build()). There is no fallback implementation.")
 
 lib = ctypes.CDLL(LIB_PATH)
@@ -82,6 +82,11 @@ lib.mfa_debug_set_flags.restype = _i
 lib.mfa_debug_set_flags.argtypes = [_i]
 lib.mfa_debug_tiles_visited.restype = _i
 lib.mfa_debug_tiles_visited.argtypes = [_vp, ctypes.POINTER(ctypes.c_ulonglong)]
+lib.mfa_debug_tmap_stats.restype = _i
+lib.mfa_debug_tmap_stats.argtypes = [ctypes.POINTER(ctypes.c_ulonglong)] * 2
+lib.mfa_debug_tmap_probe.restype = _i
+lib.mfa_debug_tmap_probe.argtypes = [_vp, _i, _i, ctypes.c_longlong, ctypes.c_longlong, _i,
+                                     ctypes.POINTER(_i)]
 lib.mfa_debug_set_decode_split_pages.restype = _i
 lib.mfa_debug_set_decode_split_pages.argtypes = [_i]
 
@@ -89,7 +94,8 @@ EXPORTED = ("mfa_fwd", "mfa_fwd_varlen", "mfa_fwd_blocksparse", "mfa_fwd_paged",
             "mfa_decode_workspace_size", "mfa_decode_plan", "mfa_decode_splitkv_window", "mfa_decode_splitkv", "mfa_status_string",
             "mfa_last_launch_info", "mfa_device_status", "mfa_debug_set_flags",
             "mfa_debug_tiles_visited", "mfa_debug_set_decode_split_pages",
-            "mfa_decode_splitkv_noalloc", "mfa_fwd_host_scratch_size", "mfa_fwd_host")
+            "mfa_decode_splitkv_noalloc", "mfa_fwd_host_scratch_size", "mfa_fwd_host",
+            "mfa_debug_tmap_stats", "mfa_debug_tmap_probe")
 
 
 class MFAError(RuntimeError):
@@ -309,6 +315,21 @@ def mfa_debug_tiles_visited(stream=None) -> int:
     n = ctypes.c_ulonglong(0)
     _check(lib.mfa_debug_tiles_visited(_stream(stream), ctypes.byref(n)), "mfa_debug_tiles_visited")
     return n.value
+
+
+def mfa_debug_tmap_stats() -> dict:
+    """Tensor-map cache counters: lookups made by launches (and probes) and encodes done."""
+    a, b = ctypes.c_ulonglong(0), ctypes.c_ulonglong(0)
+    _check(lib.mfa_debug_tmap_stats(ctypes.byref(a), ctypes.byref(b)), "mfa_debug_tmap_stats")
+    return {"lookups": a.value, "encodes": b.value}
+
+
+def mfa_debug_tmap_probe(base: int, kind: int, dtype: int, outer: int, n: int, D: int) -> bool:
+    """Host-only lookup in the tensor-map cache (placeholder maps, no driver): True if it encoded."""
+    enc = _i(0)
+    _check(lib.mfa_debug_tmap_probe(_vp(base), kind, dtype, outer, n, D, ctypes.byref(enc)),
+           "mfa_debug_tmap_probe")
+    return bool(enc.value)
 
 
 def mfa_debug_set_decode_split_pages(pages: int) -> int:

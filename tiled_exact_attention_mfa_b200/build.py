@@ -1,4 +1,8 @@
-"""Builds libmfa.so (the C-ABI CUDA library) in-tree for sm_100a with nvcc."""
+"""Builds libmfa.so (the C-ABI CUDA library) in-tree for sm_100a with nvcc.
+
+Run it as a script (python tiled_exact_attention_mfa_b200/build.py) or load it by path, as
+__graft_entry__.build() does: importing it as a submodule first imports the package, which loads
+libmfa.so."""
 from __future__ import annotations
 
 import glob

@@ -48,51 +48,116 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 3-D map over a [rows_outer][n][D] 16-bit tensor, box 64 x 128 x 1, 128-byte swizzle.
+// Encodes one 3-D map over a 16-bit tensor with a 128-byte swizzle:
+//   kind 0: [outer][n][D] (dense q / k / v / out), box 64 x 128 x 1: one box is one 128-row x
+//           128-byte slab of one head, so tails past n are zero-filled per head;
+//   kind 1: packed variable-length [n = total][outer = H][D], ordered (D, head, token), box
+//           64 x 1 x 128: the same 128-row x 128-byte slab as kind 0;
+//   kind 2: page pools [num_pages * 16 = n tokens][outer = H][D], ordered (D, head, token), box
+//           64 x 1 x 16: one box is one page of one head, 16 rows of a slab.
+bool encode_map(CUtensorMap* m, const void* base, int dtype, int kind, long long outer, long long n, int D) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3], strides[2];
+  cuuint32_t box[3];
+  if (kind == 0) {
+    dims[0] = (cuuint64_t)D; dims[1] = (cuuint64_t)n; dims[2] = (cuuint64_t)outer;
+    strides[0] = (cuuint64_t)D * 2; strides[1] = (cuuint64_t)n * D * 2;
+    box[0] = 64; box[1] = 128; box[2] = 1;
+  } else {
+    dims[0] = (cuuint64_t)D; dims[1] = (cuuint64_t)outer; dims[2] = (cuuint64_t)n;
+    strides[0] = (cuuint64_t)D * 2; strides[1] = (cuuint64_t)outer * D * 2;
+    box[0] = 64; box[1] = 1; box[2] = kind == 1 ? 128 : 16;
+  }
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dtype == MFA_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ tensor-map cache
+// A map depends only on (base pointer, data type, layout kind, extents); repeated calls over the
+// same buffers (a serving loop, a training step) would re-encode identical maps every time, each
+// a driver call of about a microsecond on the host. Encoded maps are therefore kept per device
+// under that key: kTmapCacheEntries entries, the least recently used one replaced, one mutex
+// (calls may come from several host threads). A map stays correct for any later allocation at
+// the same address with the same extents, since it describes addresses, not an allocation.
+struct TmapKey {
+  int dev, kind, dtype, D;
+  const void* base;
+  long long outer, n;
+  bool operator==(const TmapKey& o) const {
+    return dev == o.dev && kind == o.kind && dtype == o.dtype && D == o.D && base == o.base &&
+           outer == o.outer && n == o.n;
+  }
+};
+
+constexpr int kTmapCacheEntries = 256;
+// Keys of the fake encoder of mfa_debug_tmap_probe live under this device number, so they never
+// match a key of a real launch.
+constexpr int kTmapFakeDevice = -2;
+
+struct TmapCache {
+  struct Entry {
+    CUtensorMap map;
+    TmapKey key;
+    unsigned long long stamp;  // 0 = empty
+  };
+  std::mutex mu;
+  Entry e[kTmapCacheEntries] = {};
+  unsigned long long clock = 0, lookups = 0, encodes = 0;
+
+  // Copies the map of `k` into *out, encoding (and inserting) it on a miss. `encoded` tells which.
+  template <typename Enc>
+  bool get(const TmapKey& k, CUtensorMap* out, Enc&& encode, bool* encoded) {
+    std::lock_guard<std::mutex> lk(mu);
+    ++lookups;
+    int victim = 0;
+    for (int i = 0; i < kTmapCacheEntries; ++i) {
+      if (e[i].stamp != 0 && e[i].key == k) {
+        e[i].stamp = ++clock;
+        *out = e[i].map;
+        if (encoded) *encoded = false;
+        return true;
+      }
+      if (e[i].stamp < e[victim].stamp) victim = i;
+    }
+    CUtensorMap m;
+    if (!encode(&m)) return false;
+    ++encodes;
+    e[victim].map = m;
+    e[victim].key = k;
+    e[victim].stamp = ++clock;
+    *out = m;
+    if (encoded) *encoded = true;
+    return true;
+  }
+};
+TmapCache g_tmaps;
+
+bool cached_map(CUtensorMap* m, const void* base, int dtype, int kind, long long outer, long long n, int D) {
+  const int dev = current_device();
+  if (dev < 0) return false;
+  const TmapKey k = {dev, kind, dtype, D, base, outer, n};
+  return g_tmaps.get(k, m, [&](CUtensorMap* dst) { return encode_map(dst, base, dtype, kind, outer, n, D); },
+                     nullptr);
+}
+
+// 3-D map over a [rows_outer][n][D] 16-bit tensor (kind 0).
 bool make_map(CUtensorMap* m, const void* base, int dtype, long long outer, long long n, int D) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)n, (cuuint64_t)outer};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)n * D * 2};
-  cuuint32_t box[3] = {64, 128, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, dtype == MFA_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
-                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return cached_map(m, base, dtype, 0, outer, n, D);
 }
 
-// Packed variable-length layout [total, H, D]: a 3-D map ordered (D, head, token) so that one
-// box (64 elements x 1 head x 128 tokens) is the same 128-row x 128-byte slab as in make_map.
+// Packed variable-length layout [total, H, D] (kind 1).
 bool make_map_packed(CUtensorMap* m, const void* base, int dtype, long long total, int H, int D) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)total};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-  cuuint32_t box[3] = {64, 1, 128};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, dtype == MFA_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
-                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return cached_map(m, base, dtype, 1, H, total, D);
 }
 
-// Page pools [num_pages, 16, H, D] seen as [num_pages * 16 tokens, H, D], ordered (D, head,
-// token) with a 64 x 1 x 16 box: one box is one page of one head, 16 rows of a 128-byte slab.
+// Page pools [num_pages, 16, H, D] seen as [num_pages * 16 tokens, H, D] (kind 2).
 bool make_map_pages(CUtensorMap* m, const void* base, int dtype, long long tokens, int H, int D) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)tokens};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-  cuuint32_t box[3] = {64, 1, 16};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, dtype == MFA_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
-                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return cached_map(m, base, dtype, 2, H, tokens, D);
 }
 
 // Opt a kernel into its dynamic shared memory size once per device.
@@ -815,6 +880,37 @@ int mfa_debug_tiles_visited(void* stream, unsigned long long* count) {
     return MFA_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return MFA_ERR_CUDA;
   *count = h;
+  return MFA_OK;
+}
+
+int mfa_debug_tmap_stats(unsigned long long* lookups, unsigned long long* encodes) {
+  if (!lookups || !encodes) return MFA_ERR_NULL_POINTER;
+  std::lock_guard<std::mutex> lk(g_tmaps.mu);
+  *lookups = g_tmaps.lookups;
+  *encodes = g_tmaps.encodes;
+  return MFA_OK;
+}
+
+int mfa_debug_tmap_probe(const void* base, int kind, int dtype, long long outer, long long n, int D,
+                         int* encoded) {
+  if (!encoded) return MFA_ERR_NULL_POINTER;
+  if (kind < 0 || kind > 2) return MFA_ERR_BAD_SHAPE;
+  const TmapKey k = {kTmapFakeDevice, kind, dtype, D, base, outer, n};
+  CUtensorMap m;
+  bool enc = false;
+  // the fake encoder writes the key's fields into the map and needs no driver
+  auto fake = [&](CUtensorMap* dst) {
+    std::memset(dst, 0, sizeof(*dst));
+    long long f[4] = {(long long)(uintptr_t)base, outer, n, (long long)kind * 1000 + D};
+    std::memcpy(dst, f, sizeof(f));
+    return true;
+  };
+  if (!g_tmaps.get(k, &m, fake, &enc)) return MFA_ERR_CUDA;
+  long long f[4];
+  std::memcpy(f, &m, sizeof(f));
+  if (f[0] != (long long)(uintptr_t)base || f[1] != outer || f[2] != n || f[3] != (long long)kind * 1000 + D)
+    return MFA_ERR_CUDA;  // a hit returned another key's map
+  *encoded = enc ? 1 : 0;
   return MFA_OK;
 }
 
