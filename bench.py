@@ -8,8 +8,11 @@ workloads (non-causal, sliding window, GQA + softcap prefill, packed variable-le
 block-sparse prefill, chunked prefill over a paged cache, paged split-KV decode, and the backward
 of the two B=2 H=8 N=4096 workloads), each timed the same way. Inputs are seeded synthetic tensors resident in HBM; L2 is flushed (a 256 MiB
 write) before every timed step, outside the timed kernel. Times are CUDA events on the launching
-stream; with N > 1 (torchrun) every rank runs its own copy of the workload (weak scaling) and the
-max over ranks is reported.
+stream; with N > 1 (torchrun, one process per GPU) the problem is sharded by (sequence, kv-head)
+units with no exchange -- by default a batch N times the workload's, each GPU owning its slice
+(weak scaling; --scaling strong splits the workload's own units instead) -- the max over ranks is
+reported, and a decode line spreads every sequence's splits over the GPUs with one NCCL
+all-gather of the partial results before the combine.
 """
 from __future__ import annotations
 
@@ -215,14 +218,24 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
-def main_config(name: str, world: int) -> dict:
+def parallelism(name: str, world: int, scaling: str) -> str:
+    c = mi.workloads()[name]
+    units = c.B * c.Hkv
+    if scaling == "strong":
+        return (f"sharded: the {units} (sequence, kv-head) units of the workload split over "
+                f"{world} GPU(s), no exchange")
+    return (f"sharded: a batch of {world} x {c.B} sequences, {units} (sequence, kv-head) units "
+            f"per GPU on {world} GPU(s), no exchange")
+
+
+def main_config(name: str, world: int, scaling: str = "weak") -> dict:
     """The `config` of the headline line, shared by the GPU arm and the reference arm."""
     c = mi.workloads()[name]
     return {"workload": name, "B": c.B, "Hq": c.Hq, "Hkv": c.Hkv, "N": c.Nq, "D": c.D,
             "causal": c.causal, "window": [c.win_l, c.win_r], "softcap": c.softcap,
             "dtype": mi.DTYPE_NAMES[c.dtype],
             "l2": "flushed before every timed step (256 MiB write)",
-            "parallelism": f"replica per GPU x{world}"}
+            "parallelism": parallelism(name, world, scaling)}
 
 
 def pages_context(name: str) -> dict:
@@ -280,8 +293,7 @@ def spread_of(r):
 
 
 def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
-    """Largest per-rank time: every rank runs its own copy of the workload (weak scaling), so the
-    job takes as long as its slowest rank."""
+    """Largest per-rank time: the job takes as long as its slowest rank."""
     if world <= 1:
         return x
     import torch
@@ -296,26 +308,39 @@ def job_throughput(units_per_rank: float, world: int, max_ms: float) -> float:
     return units_per_rank * world / (max_ms * 1e-3)
 
 
-def bench_prefill(case, steps, warmup, flush, stream, with_e2e, world):
+def bench_prefill(case, steps, warmup, flush, stream, with_e2e, world, rank=0, scaling="weak"):
+    """One prefill workload. With N > 1 ranks the problem is sharded by (sequence, kv head)
+    units with no exchange: scaling "weak" makes the job N x the workload's batch, rank r owning
+    batch rows [r B, (r + 1) B) (its own slice of the seeded inputs); "strong" splits the
+    workload itself, rank r running its contiguous range of units. res["job_flops"] is the work of
+    the whole job."""
     import torch
     import tiled_exact_attention_mfa_b200 as mfa
+    from tiled_exact_attention_mfa_b200 import shard
     dev = torch.device("cuda")
-    q, k, v = case.tensors()
+    weak = scaling == "weak"
+    q, k, v = case.batch_slice_tensors(rank) if (world > 1 and weak) else case.tensors()
     qt, kt, vt = (upload(x, case.dtype, dev) for x in (q, k, v))
     out = torch.empty_like(qt)
     lse = torch.empty(case.B, case.Hq, case.Nq, dtype=torch.float32, device=dev)
     scale = case.scale_f32()
     win = (case.win_l, case.win_r)
+    kw = dict(scale=scale, causal=case.causal, window=win, softcap=case.softcap, stream=stream)
 
-    def step():
-        mfa.mfa_fwd(qt, kt, vt, out, lse, scale=scale, causal=case.causal, window=win,
-                    softcap=case.softcap, stream=stream)
+    if weak or world == 1:
+        def step():
+            mfa.mfa_fwd(qt, kt, vt, out, lse, **kw)
+    else:
+        def step():
+            shard.fwd_sharded(qt, kt, vt, out, lse, world, rank, **kw)
 
     with torch.cuda.stream(stream):
         ms, bracket = time_steps(step, steps, warmup, flush, stream)
     res = {"ms": statistics.mean(ms), "ms_min": min(ms), **spread(ms), "bracket_ms": bracket,
            "flops": prefill_flops(case), "bytes": prefill_bytes(case)}
+    res["job_flops"] = res["flops"] * (world if weak else 1)
     res["ms"] = max_over_ranks(res["ms"], world)
+
     if with_e2e:
         # the C-ABI call with host buffers (mfa_fwd_host): every step copies q, k, v from pinned
         # host memory, runs the forward and copies out and lse back, all inside the timed region
@@ -329,14 +354,30 @@ def bench_prefill(case, steps, warmup, flush, stream, with_e2e, world):
                                                             case.Nk, case.D),
                               dtype=torch.uint8, device=dev)
 
+        if weak or world == 1:
+            e_in = (hq, hk, hv, ho, hl)
+        else:  # this rank's units: contiguous slices of the host tensors
+            e_in = shard.prefill_shard_views(hq, hk, hv, ho, hl, world, rank)
+            eq = e_in[0]
+            scratch = torch.empty(mfa.mfa_fwd_host_scratch_size(eq.shape[0], eq.shape[1], 1,
+                                                                case.Nq, case.Nk, case.D),
+                                  dtype=torch.uint8, device=dev)
+
         def e2e_step():
-            mfa.mfa_fwd_host(hq, hk, hv, ho, hl, scale=scale, causal=case.causal, window=win,
+            mfa.mfa_fwd_host(*e_in, scale=scale, causal=case.causal, window=win,
                              softcap=case.softcap, scratch=scratch, stream=stream)
 
         with torch.cuda.stream(stream):
             ems, _ = time_steps(e2e_step, max(3, steps // 2), 2, flush, stream)
         torch.cuda.synchronize()
-        if not (torch.equal(ho, out.cpu()) and torch.equal(hl, lse.cpu())):
+        dev_parts = (out.cpu(), lse.cpu())
+        if not (weak or world == 1):  # compare this rank's slices only
+            dev_parts = shard.prefill_shard_views(qt.cpu(), kt.cpu(), vt.cpu(), *dev_parts, world,
+                                                  rank)[3:]
+            host_parts = e_in[3:]
+        else:
+            host_parts = (ho, hl)
+        if not all(torch.equal(a, b) for a, b in zip(host_parts, dev_parts)):
             raise RuntimeError("host-buffer forward differs from the device forward")
         res["e2e_ms"] = max_over_ranks(statistics.mean(ems), world)
         # the PCIe floor on this machine, same run: the step's own pinned inputs copied in alone
@@ -350,9 +391,41 @@ def bench_prefill(case, steps, warmup, flush, stream, with_e2e, world):
         with torch.cuda.stream(stream):
             hms, _ = time_steps(h2d_only, 5, 2, flush, stream)
         res["h2d_alone_ms"] = statistics.mean(hms)
-        res["h2d"] = int(q.nbytes + k.nbytes + v.nbytes)
-        res["d2h"] = int(ho.numel() * 2 + hl.numel() * 4)
+        res["h2d"] = int(sum(t.numel() * t.element_size() for t in e_in[:3]))
+        res["d2h"] = int(sum(t.numel() * t.element_size() for t in e_in[3:]))
     return res
+
+
+def bench_decode_sharded(case, steps, warmup, flush, stream, world, rank):
+    """Split-KV decode with each sequence's splits spread over the ranks: rank r computes phase 1
+    for its block of splits (it reads only those pages), the partial blocks are all-gathered over
+    NCCL, and every rank runs the combine. The time of a step includes the exchange."""
+    import torch
+    import tiled_exact_attention_mfa_b200 as mfa
+    from tiled_exact_attention_mfa_b200 import shard
+    dev = torch.device("cuda")
+    q, kp, vp, table, lens = case.tensors()
+    qt, kt, vt = (upload(x, case.dtype, dev) for x in (q, kp, vp))
+    tt, lt = torch.from_numpy(table).to(dev), torch.from_numpy(lens).to(dev)
+    out = torch.empty_like(qt)
+    lse = torch.empty(case.B, case.Hq, case.Nq, dtype=torch.float32, device=dev)
+    plan = mfa.mfa_decode_plan(case.B, case.Nq, case.Hq, case.Hkv, case.D, table.shape[1], 16,
+                               case.win_l)
+    so, sm = shard.decode_partial_shapes(case.B, case.Nq, case.Hq, case.D, plan["max_splits"], world)
+    po = torch.empty(so, dtype=torch.float32, device=dev)
+    pm = torch.empty(sm, dtype=torch.float32, device=dev)
+
+    def step():
+        shard.decode_sharded(qt, kt, vt, tt, lt, out, lse, po, pm, world, rank,
+                             scale=case.scale_f32(), causal=case.causal, softcap=case.softcap,
+                             win_l=case.win_l)
+
+    with torch.cuda.stream(stream):
+        ms, bracket = time_steps(step, steps, warmup, flush, stream)
+    return {"ms": max_over_ranks(statistics.mean(ms), world), "ms_min": min(ms), **spread(ms),
+            "bracket_ms": bracket, "bytes": decode_bytes(case, lens),
+            "exchange_bytes": int(4 * case.B * case.Hq * case.Nq * (case.D + 2) *
+                                  shard.split_chunk(plan["max_splits"], world) * (world - 1))}
 
 
 def host_call_us(case, stream, calls=2000):
@@ -543,7 +616,8 @@ def run_gpu(args):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    main = bench_prefill(main_case, args.steps, args.warmup, flush, stream, not args.no_e2e, world)
+    main = bench_prefill(main_case, args.steps, args.warmup, flush, stream, not args.no_e2e, world,
+                         rank, args.scaling)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -601,6 +675,19 @@ def run_gpu(args):
                                **({"host_us_per_call": r["host_us"]} if "host_us" in r else {}),
                                **pages_context(name)})
             getattr(case, "_cache", {}).clear()  # the workload's host inputs are not needed again
+    if not args.only_main and world > 1:
+        # the decode workload with every sequence's splits spread over the GPUs (strong
+        # scaling of one decode step, with its one exchange: the all-gather of the partials)
+        name = "decode_b8_hq32_hkv8_d128_bf16_len8k_128k"
+        sk, wu = max(3, min(args.steps, 10)), max(3, args.warmup)
+        r = bench_decode_sharded(W[name], sk, wu, flush, stream, world, rank)
+        tb = r["bytes"] / (r["ms"] * 1e-3) / 1e9
+        others.append({**spread_of(r), "workload": name + ":splits_over_gpus", "ms": round(r["ms"], 4),
+                       "unit": "GB/s", "value": round(tb, 1), "bound": "hbm",
+                       "frac_of_measured_peak_x_gpus": round(tb / (pk["gbs"] * world), 4),
+                       "exchange_bytes_per_gpu": r["exchange_bytes"], "scaling": "strong",
+                       "parallelism": f"splits of every sequence over {world} GPUs, NCCL all-gather "
+                                      "of the (o, m, l) partials, combine on every GPU"})
         for name in BACKWARD_WORKLOADS:
             sk, wu = max(3, min(args.steps, 10)), max(3, args.warmup)
             r = bench_backward(W[name], sk, wu, flush, stream, world)
@@ -611,8 +698,8 @@ def run_gpu(args):
                            "frac_of_nominal_tensor_peak": round(tf / NOMINAL_TFLOPS, 4),
                            "flops_convention": "2.5 x forward (S, dP, dV, dK, dQ over visible pairs)"})
     clk = clocks.stop()
-    tflops = job_throughput(main["flops"], world, main["ms"]) / 1e12
-    per_gpu_tflops = main["flops"] / (main["ms"] * 1e-3) / 1e12
+    tflops = main["job_flops"] / (main["ms"] * 1e-3) / 1e12
+    per_gpu_tflops = tflops / world
     line = {
         "metric": METRIC,
         "value": round(tflops, 2),
@@ -623,11 +710,11 @@ def run_gpu(args):
         "ms_per_step": round(main["ms"], 5),
         **spread_of(main),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": args.scaling,
         "vs_baseline": None,
         "dtype": mi.DTYPE_NAMES[main_case.dtype],
         "data": "synthetic (seeded N(0,1) Q/K/V, SplitMix64 + Box-Muller)",
-        "config": main_config(args.workload, world),
+        "config": main_config(args.workload, world, args.scaling),
         "context": {**pages_context(args.workload),
                     "note": "the pages' own timing on Apple hardware, for context; not a target"},
         "roofline": {"bound": "tensor", "achieved": round(per_gpu_tflops, 2),
@@ -642,7 +729,7 @@ def run_gpu(args):
         "workloads": others,
     }
     if "e2e_ms" in main:
-        line["e2e"] = {"value": round(main["flops"] * world / (main["e2e_ms"] * 1e-3) / 1e12, 3),
+        line["e2e"] = {"value": round(main["job_flops"] / (main["e2e_ms"] * 1e-3) / 1e12, 3),
                        "unit": "TFLOP/s", "ms_per_step": round(main["e2e_ms"], 4),
                        "h2d_bytes_per_step": main["h2d"], "d2h_bytes_per_step": main["d2h"],
                        "h2d_alone_ms": round(main["h2d_alone_ms"], 4),
@@ -726,8 +813,8 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(mean_ms, 3), **spread(ms), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": main_config(args.workload, world),
+            "scaling": args.scaling, "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": main_config(args.workload, world, args.scaling),
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -769,6 +856,9 @@ def main():
                     choices=sorted(n for n, c in mi.workloads().items() if isinstance(c, mi.PrefillCase)))
     ap.add_argument("--only-main", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--scaling", choices=["weak", "strong"], default="weak",
+                    help="N > 1: weak = a batch N times the workload's, sharded by (sequence, "
+                         "kv-head) units; strong = the workload's own units split over the GPUs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--profile", default=None,

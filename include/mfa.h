@@ -366,6 +366,49 @@ int mfa_debug_set_flags(int flags);
 int mfa_debug_tiles_visited(void* stream, unsigned long long* count);
 
 /*
+ * mfa_decode_phase1 / mfa_decode_combine -- the two phases of mfa_decode_splitkv_window as
+ * separate calls, for a decode whose splits are spread over several GPUs (each GPU holds the
+ * pages of some splits of every sequence). Source: [MFA252] Features (Flash Decode: two-phase
+ * split-KV) and [MXFA15] README (per-split (m, l) slots merged by a combine step); spreading the
+ * splits over GPUs is this library's use of the same two phases.
+ *
+ * The split plan is mfa_decode_plan's for the shape and win_l: splits s = 0 .. max_splits - 1,
+ * split s of a sequence covering pages [first + s * pages_per_split, first + (s + 1) *
+ * pages_per_split) of it (first = 0 without a window).
+ *
+ * Partial results are split-major, so a range of splits is one contiguous block of each array:
+ *   part_o   float [split_capacity][B][Hq * Nq][D]   unnormalised O of the split's keys
+ *   part_ml  float [split_capacity][B][Hq * Nq][2]   (running max in log2 units, running sum)
+ * (row index (h * Nq + t)); split_capacity >= max_splits; both 16-byte aligned device buffers
+ * owned by the caller.
+ *
+ * mfa_decode_phase1 computes the partials of splits [split_lo, split_hi) (0 <= split_lo <=
+ * split_hi <= max_splits) of every sequence and kv head into their slots; it reads only the
+ * block_table entries and pages of those splits, so a GPU's pool need hold only those pages.
+ * Slots of splits past a sequence's end are left untouched. Arguments as mfa_decode_splitkv_window.
+ *
+ * mfa_decode_combine merges, for every (sequence, query head, token), the slots of splits
+ * 0 .. n_splits(b) - 1 of part_o / part_ml (every one must have been written, by some GPU's
+ * phase 1, and be visible on this stream) into out and lse, as mfa_decode_splitkv does.
+ *
+ * Gathering: with the splits cut into equal ranges of c splits per GPU (split_capacity = c x
+ * number of GPUs), GPU r's block of each array starts at split r * c, so one all-gather of the
+ * blocks in rank order leaves every GPU with the arrays a single GPU computing all splits writes.
+ * Returns MFA_OK after the launch was queued, or a negative status (MFA_ERR_WORKSPACE when
+ * split_capacity < max_splits or a partial pointer is NULL).
+ */
+int mfa_decode_phase1(const void* q, const void* k_pages, const void* v_pages,
+                      const int32_t* block_table, const int32_t* seq_lens, int B, int Nq, int Hq,
+                      int Hkv, int D, int page_size, int max_pages_per_seq, int num_pages,
+                      float scale, int causal, int win_l, float softcap, int dtype, int split_lo,
+                      int split_hi, float* part_o, float* part_ml, int split_capacity,
+                      void* stream);
+int mfa_decode_combine(const int32_t* seq_lens, void* out, float* lse, int B, int Nq, int Hq,
+                       int Hkv, int D, int page_size, int max_pages_per_seq, int win_l, int dtype,
+                       const float* part_o, const float* part_ml, int split_capacity,
+                       void* stream);
+
+/*
  * Tensor-map cache counters: map lookups made by launches so far and how many of them had to
  * encode a map (cuTensorMapEncodeTiled) because no map of the same (device, base pointer, data
  * type, layout, extents) was cached. A second call over the same buffers encodes nothing.

@@ -147,9 +147,21 @@ class PrefillCase:
 
     def tensors(self):
         """(q, k, v) as uint16 bit patterns."""
-        q = normal_bits(self.seed, STREAM_Q, (self.B, self.Hq, self.Nq, self.D), self.dtype, self.mul)
-        k = normal_bits(self.seed, STREAM_K, (self.B, self.Hkv, self.Nk, self.D), self.dtype, self.mul)
-        v = normal_bits(self.seed, STREAM_V, (self.B, self.Hkv, self.Nk, self.D), self.dtype, self.mul)
+        return self.batch_slice_tensors(0)
+
+    def batch_slice_tensors(self, index: int):
+        """(q, k, v) of batch rows [index * B, (index + 1) * B) of the same workload with a batch
+        of any larger multiple of B: the draws continue the streams at those rows' offsets, so
+        the slices of consecutive indices are pieces of one larger seeded problem (index 0 is
+        tensors())."""
+        qn = self.B * self.Hq * self.Nq * self.D
+        kn = self.B * self.Hkv * self.Nk * self.D
+        q = normal_bits(self.seed, STREAM_Q, (self.B, self.Hq, self.Nq, self.D), self.dtype, self.mul,
+                        offset=index * qn)
+        k = normal_bits(self.seed, STREAM_K, (self.B, self.Hkv, self.Nk, self.D), self.dtype, self.mul,
+                        offset=index * kn)
+        v = normal_bits(self.seed, STREAM_V, (self.B, self.Hkv, self.Nk, self.D), self.dtype, self.mul,
+                        offset=index * kn)
         return q, k, v
 
 

@@ -53,6 +53,10 @@ lib.mfa_decode_splitkv.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i
 lib.mfa_decode_splitkv_window.restype = _i
 lib.mfa_decode_splitkv_window.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                           _i, _i, _f, _i, _i, _f, _i, _vp, ctypes.c_size_t, _vp]
+lib.mfa_decode_phase1.restype = _i
+lib.mfa_decode_phase1.argtypes = [_vp] * 5 + [_i] * 8 + [_f, _i, _i, _f, _i, _i, _i, _vp, _vp, _i, _vp]
+lib.mfa_decode_combine.restype = _i
+lib.mfa_decode_combine.argtypes = [_vp] * 3 + [_i] * 9 + [_vp, _vp, _i, _vp]
 lib.mfa_fwd_host_scratch_size.restype = ctypes.c_size_t
 lib.mfa_fwd_host_scratch_size.argtypes = [_i] * 6
 lib.mfa_fwd_host.restype = _i
@@ -95,7 +99,8 @@ EXPORTED = ("mfa_fwd", "mfa_fwd_varlen", "mfa_fwd_blocksparse", "mfa_fwd_paged",
             "mfa_last_launch_info", "mfa_device_status", "mfa_debug_set_flags",
             "mfa_debug_tiles_visited", "mfa_debug_set_decode_split_pages",
             "mfa_decode_splitkv_noalloc", "mfa_fwd_host_scratch_size", "mfa_fwd_host",
-            "mfa_debug_tmap_stats", "mfa_debug_tmap_probe")
+            "mfa_debug_tmap_stats", "mfa_debug_tmap_probe", "mfa_decode_phase1",
+            "mfa_decode_combine")
 
 
 class MFAError(RuntimeError):
@@ -291,6 +296,49 @@ def mfa_decode_splitkv_noalloc(q, k_pages, v_pages, block_table, seq_lens, out, 
                                         int(bool(causal)), float(softcap), _dtype_code(q),
                                         _stream(stream))
     _check(rc, "mfa_decode_splitkv_noalloc")
+    return out, lse
+
+
+def _check_partials(part_o, part_ml, D):
+    torch = _torch()
+    if part_o.dtype != torch.float32 or part_ml.dtype != torch.float32:
+        raise TypeError("partial buffers must be float32")
+    if part_o.dim() != 4 or part_ml.dim() != 4 or part_o.shape[3] != D or part_ml.shape[3] != 2 \
+            or part_o.shape[:3] != part_ml.shape[:3]:
+        raise ValueError("partials must be [splits, B, Hq*Nq, D] and [splits, B, Hq*Nq, 2]")
+    return part_o.shape[0]
+
+
+def mfa_decode_phase1(q, k_pages, v_pages, block_table, seq_lens, part_o, part_ml, split_lo,
+                      split_hi, *, scale=None, causal=True, softcap=0.0, win_l=-1, stream=None):
+    """Phase 1 of the split-KV decode for splits [split_lo, split_hi) of every sequence, into
+    the split-major partial buffers part_o [cap, B, Hq*Nq, D] / part_ml [cap, B, Hq*Nq, 2]."""
+    torch = _torch()
+    B, Hq, Nq, D = q.shape
+    num_pages, page, Hkv, _ = k_pages.shape
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("block_table and seq_lens must be int32")
+    cap = _check_partials(part_o, part_ml, D)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    rc = lib.mfa_decode_phase1(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
+                               _ptr(seq_lens), B, Nq, Hq, Hkv, D, page, block_table.shape[1],
+                               num_pages, float(scale), int(bool(causal)), int(win_l),
+                               float(softcap), _dtype_code(q), int(split_lo), int(split_hi),
+                               _ptr(part_o), _ptr(part_ml), cap, _stream(stream))
+    _check(rc, "mfa_decode_phase1")
+
+
+def mfa_decode_combine(seq_lens, part_o, part_ml, out, lse=None, *, Hkv, max_pages_per_seq,
+                       win_l=-1, stream=None):
+    """The combine of the split-KV decode over every split's partials, into out [B, Hq, Nq, D]
+    (and lse [B, Hq, Nq] fp32 unless None). Hkv and max_pages_per_seq fix the split plan."""
+    B, Hq, Nq, D = out.shape
+    cap = _check_partials(part_o, part_ml, D)
+    rc = lib.mfa_decode_combine(_ptr(seq_lens), _ptr(out), _ptr(lse), B, Nq, Hq, int(Hkv), D, 16,
+                                int(max_pages_per_seq), int(win_l), _dtype_code(out),
+                                _ptr(part_o), _ptr(part_ml), cap, _stream(stream))
+    _check(rc, "mfa_decode_combine")
     return out, lse
 
 

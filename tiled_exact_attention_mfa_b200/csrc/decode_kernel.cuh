@@ -39,10 +39,13 @@ struct DecodeParams {
   const int32_t* seq_lens;
   void* out;
   float* lse;
-  float* ws_o;    // [B][max_splits][Hq*Nq][D]
-  float* ws_ml;   // [B][max_splits][Hq*Nq][2]  (m in log2 units, l)
+  // partial results, split-major so that a range of splits is one contiguous block (the unit a
+  // GPU contributes when the splits of a sequence are spread over GPUs):
+  float* ws_o;    // [splits][B][Hq*Nq][D]  unnormalised O
+  float* ws_ml;   // [splits][B][Hq*Nq][2]  (m in log2 units, l)
   int B, Nq, Hq, Hkv, G, max_pages, num_pages;
   int pages_per_split, max_splits, heads_per_cta;
+  int split_lo;   // phase 1 computes splits split_lo + blockIdx.x
   int causal;
   int win_l;      // left window (query at position a sees keys >= a - win_l); -1: none
   float c_log2;   // scale * log2 e (no softcap) or log2 e (softcap)
@@ -97,7 +100,7 @@ __global__ void __launch_bounds__((kDecMaxHeads<D> + 1) * 32) mfa_decode_phase1_
   // every CTA of this grid is resident (or done) once all have passed here, so the combine grid
   // may be launched now; it waits for this grid's completion before reading the workspace
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int split = blockIdx.x;
+  const int split = p.split_lo + blockIdx.x;
   const int b = blockIdx.y;
   const int h0 = blockIdx.z * hg;  // first kv head of this CTA
   const int warp = threadIdx.x >> 5;
@@ -308,7 +311,7 @@ __global__ void __launch_bounds__((kDecMaxHeads<D> + 1) * 32) mfa_decode_phase1_
 
   // ---- partial results (rows < R only)
   const size_t rows_all = (size_t)p.Hq * p.Nq;
-  const size_t slot = ((size_t)b * p.max_splits + split) * rows_all;
+  const size_t slot = ((size_t)split * p.B + b) * rows_all;
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     const int r = qr + 8 * e;
@@ -353,10 +356,11 @@ __global__ void __launch_bounds__(kCombineThreads) mfa_decode_combine_kernel(con
   const int n_pages = (len + kDecPage - 1) / kDecPage;
   const int n_splits = (n_pages - dec_first_page(p, len) + p.pages_per_split - 1) / p.pages_per_split;
   const size_t rows_all = (size_t)p.Hq * p.Nq;
-  const size_t slot0 = (size_t)b * p.max_splits * rows_all + row;  // slot of split s: slot0 + s * rows_all
+  const size_t slot0 = (size_t)b * rows_all + row;  // slot of split s: slot0 + s * B * rows_all
+  const size_t split_step = (size_t)p.B * rows_all;
   const float2* ml = reinterpret_cast<const float2*>(p.ws_ml);
   const float4* o = reinterpret_cast<const float4*>(p.ws_o + slot0 * D) + dq;
-  const size_t stride = rows_all * (D / 4);  // float4 steps from one split's row to the next
+  const size_t stride = split_step * (D / 4);  // float4 steps from one split's row to the next
 
   float m_g = -INFINITY, l_g = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -369,7 +373,7 @@ __global__ void __launch_bounds__(kCombineThreads) mfa_decode_combine_kernel(con
       st[j] = make_float2(-INFINITY, 0.f);
       ov[j] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (s < n_splits) {
-        st[j] = ml[slot0 + (size_t)s * rows_all];
+        st[j] = ml[slot0 + (size_t)s * split_step];
         ov[j] = o[(size_t)s * stride];
       }
     }

@@ -355,43 +355,69 @@ int launch_fwd(const FwdCall& c, cudaStream_t st) {
   return MFA_OK;
 }
 
+// Parts of the decode a launch runs.
+constexpr int kDecPhase1 = 1;
+constexpr int kDecCombine = 2;
+
+// Phase 1 over splits [p.split_lo, split_hi) and / or the combine. With both, the combine is a
+// programmatic dependent of phase 1: it is launched while the last phase-1 CTAs still run and
+// waits in griddepcontrol.wait until their workspace writes are visible. Alone, it is a plain
+// launch ordered after earlier work on the stream (its wait is then a no-op).
 template <int D, bool BF16>
-int launch_decode(const mfa::DecodeParams& p, const DecodePlan& pl, cudaStream_t st) {
+int launch_decode(const mfa::DecodeParams& p, const DecodePlan& pl, int split_hi, int parts,
+                  cudaStream_t st) {
   static bool smem_done[kMaxDevices] = {};
   const int smem = mfa::dec_smem_bytes<D>(pl.heads_per_cta);
-  // the largest plan (1024 / (2 D) heads per CTA) sets the attribute for all
-  auto k1 = mfa::mfa_decode_phase1_kernel<D, BF16>;
-  if (!ensure_smem(k1, mfa::dec_smem_bytes<D>(mfa::kDecMaxHeads<D>), smem_done)) return MFA_ERR_CUDA;
-  dim3 g1(pl.max_splits, p.B, pl.groups);
-  k1<<<g1, (pl.heads_per_cta + 1) * 32, smem, st>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
-  // the combine is a programmatic dependent of phase 1: it is launched while the last phase-1
-  // CTAs still run and waits in griddepcontrol.wait until their workspace writes are visible
-  dim3 g2(p.Hq * p.Nq, p.B, 1);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = g2;
-  cfg.blockDim = dim3(mfa::kCombineThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, mfa::mfa_decode_combine_kernel<D, BF16>, p) != cudaSuccess)
-    return MFA_ERR_CUDA;
   mfa_launch_info li = {};
   li.kernel = 2;
-  li.grid_x = g1.x;
-  li.grid_y = g1.y;
-  li.grid_z = g1.z;
-  li.block_threads = (pl.heads_per_cta + 1) * 32;
-  li.smem_bytes = smem;
+  const bool phase1 = (parts & kDecPhase1) && split_hi > p.split_lo;
+  if (phase1) {
+    // the largest plan (1024 / (2 D) heads per CTA) sets the attribute for all
+    auto k1 = mfa::mfa_decode_phase1_kernel<D, BF16>;
+    if (!ensure_smem(k1, mfa::dec_smem_bytes<D>(mfa::kDecMaxHeads<D>), smem_done)) return MFA_ERR_CUDA;
+    dim3 g1(split_hi - p.split_lo, p.B, pl.groups);
+    k1<<<g1, (pl.heads_per_cta + 1) * 32, smem, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
+    li.grid_x = g1.x;
+    li.grid_y = g1.y;
+    li.grid_z = g1.z;
+    li.block_threads = (pl.heads_per_cta + 1) * 32;
+    li.smem_bytes = smem;
+  }
+  if (parts & kDecCombine) {
+    dim3 g2(p.Hq * p.Nq, p.B, 1);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = g2;
+    cfg.blockDim = dim3(mfa::kCombineThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = phase1 ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, mfa::mfa_decode_combine_kernel<D, BF16>, p) != cudaSuccess)
+      return MFA_ERR_CUDA;
+  }
   li.pages_per_split = pl.pages_per_split;
   li.max_splits = pl.max_splits;
   li.kv_heads_per_cta = pl.heads_per_cta;
   g_last = li;
   return MFA_OK;
+}
+
+template <int D>
+int dispatch_decode_d(const mfa::DecodeParams& p, const DecodePlan& pl, int split_hi, int parts,
+                      bool bf, cudaStream_t st) {
+  return bf ? launch_decode<D, true>(p, pl, split_hi, parts, st)
+            : launch_decode<D, false>(p, pl, split_hi, parts, st);
+}
+
+int dispatch_decode(const mfa::DecodeParams& p, const DecodePlan& pl, int D, int split_hi, int parts,
+                    bool bf, cudaStream_t st) {
+  if (D == 256) return dispatch_decode_d<256>(p, pl, split_hi, parts, bf, st);
+  if (D == 128) return dispatch_decode_d<128>(p, pl, split_hi, parts, bf, st);
+  return dispatch_decode_d<64>(p, pl, split_hi, parts, bf, st);
 }
 
 // Checks shared by the dense and the packed forward.
@@ -719,32 +745,32 @@ size_t decode_workspace_size(int B, int Nq, int Hq, int Hkv, int D, int max_page
   return align256(rows * D * sizeof(float)) + align256(rows * 2 * sizeof(float));
 }
 
-// The decode entry points after their override read: override_pages is the split-size override
-// this call uses for both the workspace check and the launched plan.
-int decode_splitkv(const void* q, const void* k_pages, const void* v_pages,
-                   const int32_t* block_table, const int32_t* seq_lens, void* out, float* lse,
-                   int B, int Nq, int Hq, int Hkv, int D, int page_size, int max_pages_per_seq,
-                   int num_pages, float scale, int causal, int win_l, float softcap, int dtype,
-                   void* workspace, size_t workspace_bytes, cudaStream_t st, int override_pages) {
+// Checks every argument of a decode call that phase 1 needs (pointers may be NULL only where
+// the caller passes nullptr for `need_kv`), derives the plan and fills the kernel parameters
+// (partial-result pointers left to the caller).
+int decode_params(mfa::DecodeParams& p, DecodePlan& pl, const void* q, const void* k_pages,
+                  const void* v_pages, const int32_t* block_table, const int32_t* seq_lens,
+                  void* out, float* lse, int B, int Nq, int Hq, int Hkv, int D, int page_size,
+                  int max_pages_per_seq, int num_pages, float scale, int causal, int win_l,
+                  float softcap, int dtype, int override_pages, bool need_kv, bool need_out) {
   if (dtype != MFA_DTYPE_FP16 && dtype != MFA_DTYPE_BF16) return MFA_ERR_BAD_DTYPE;
   if (win_l < -1) return MFA_ERR_BAD_WINDOW;
   int rc = validate_decode(B, Nq, Hq, Hkv, D, page_size, max_pages_per_seq);
   if (rc != MFA_OK) return rc;
-  if (num_pages < 1) return MFA_ERR_BAD_SHAPE;
+  if (need_kv && num_pages < 1) return MFA_ERR_BAD_SHAPE;
   if (!std::isfinite(softcap) || softcap < 0.f) return MFA_ERR_BAD_SOFTCAP;
   if (!std::isfinite(scale) || !(scale > 0.f)) return MFA_ERR_BAD_SCALE;
-  if ((rc = check_sizes(num_pages, page_size, Hkv, D)) != MFA_OK) return rc;
+  if (need_kv && (rc = check_sizes(num_pages, page_size, Hkv, D)) != MFA_OK) return rc;
   if ((rc = check_sizes(B, Hq, Nq, D)) != MFA_OK) return rc;
   if (B == 0) return MFA_OK;
-  if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !out) return MFA_ERR_NULL_POINTER;
-  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(block_table) ||
-      !aligned16(seq_lens) || !aligned16(out) || !aligned16(lse))
+  if (!seq_lens || (need_kv && (!q || !k_pages || !v_pages || !block_table)) || (need_out && !out))
+    return MFA_ERR_NULL_POINTER;
+  if (!aligned16(seq_lens) || (need_kv && (!aligned16(q) || !aligned16(k_pages) ||
+                                           !aligned16(v_pages) || !aligned16(block_table))) ||
+      (need_out && (!aligned16(out) || !aligned16(lse))))
     return MFA_ERR_MISALIGNED;
-  const size_t need = decode_workspace_size(B, Nq, Hq, Hkv, D, max_pages_per_seq, page_size, override_pages);
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
-    return MFA_ERR_WORKSPACE;
-  DecodePlan pl = decode_plan(B, Hkv, D, max_pages_per_seq, Nq, win_l, override_pages);
-  mfa::DecodeParams p;
+  pl = decode_plan(B, Hkv, D, max_pages_per_seq, Nq, win_l, override_pages);
+  if (pl.max_splits > 0x7FFFFFFF || B > 65535 || pl.groups > 65535) return MFA_ERR_BAD_SHAPE;
   std::memset(&p, 0, sizeof(p));
   p.q = static_cast<const uint16_t*>(q);
   p.k_pages = static_cast<const uint16_t*>(k_pages);
@@ -753,9 +779,6 @@ int decode_splitkv(const void* q, const void* k_pages, const void* v_pages,
   p.seq_lens = seq_lens;
   p.out = out;
   p.lse = lse;
-  const size_t rows = (size_t)B * pl.max_splits * Hq * Nq;
-  p.ws_o = static_cast<float*>(workspace);
-  p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(rows * D * sizeof(float)));
   p.B = B;
   p.Nq = Nq;
   p.Hq = Hq;
@@ -776,11 +799,33 @@ int decode_splitkv(const void* q, const void* k_pages, const void* v_pages,
   } else {
     p.c_log2 = scale * log2e;
   }
-  if (pl.max_splits > 0x7FFFFFFF || B > 65535 || pl.groups > 65535) return MFA_ERR_BAD_SHAPE;
-  const bool bf = dtype == MFA_DTYPE_BF16;
-  if (D == 256) return bf ? launch_decode<256, true>(p, pl, st) : launch_decode<256, false>(p, pl, st);
-  if (D == 128) return bf ? launch_decode<128, true>(p, pl, st) : launch_decode<128, false>(p, pl, st);
-  return bf ? launch_decode<64, true>(p, pl, st) : launch_decode<64, false>(p, pl, st);
+  return MFA_OK;
+}
+
+// The decode entry points after their override read: override_pages is the split-size override
+// this call uses for both the workspace check and the launched plan.
+int decode_splitkv(const void* q, const void* k_pages, const void* v_pages,
+                   const int32_t* block_table, const int32_t* seq_lens, void* out, float* lse,
+                   int B, int Nq, int Hq, int Hkv, int D, int page_size, int max_pages_per_seq,
+                   int num_pages, float scale, int causal, int win_l, float softcap, int dtype,
+                   void* workspace, size_t workspace_bytes, cudaStream_t st, int override_pages) {
+  mfa::DecodeParams p;
+  DecodePlan pl;
+  int rc = decode_params(p, pl, q, k_pages, v_pages, block_table, seq_lens, out, lse, B, Nq, Hq,
+                         Hkv, D, page_size, max_pages_per_seq, num_pages, scale, causal, win_l,
+                         softcap, dtype, override_pages, true, true);
+  if (rc != MFA_OK || B == 0) return rc;
+  const size_t need = decode_workspace_size(B, Nq, Hq, Hkv, D, max_pages_per_seq, page_size, override_pages);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
+    return MFA_ERR_WORKSPACE;
+  // the unwindowed plan sizes the workspace; a window's plan never has more splits
+  const DecodePlan full = decode_plan(B, Hkv, D, max_pages_per_seq, 1, -1, override_pages);
+  const size_t rows = (size_t)B * full.max_splits * Hq * Nq;
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(rows * D * sizeof(float)));
+  p.split_lo = 0;
+  return dispatch_decode(p, pl, D, pl.max_splits, kDecPhase1 | kDecCombine,
+                         dtype == MFA_DTYPE_BF16, st);
 }
 
 }  // namespace
@@ -803,6 +848,48 @@ int mfa_decode_splitkv_window(const void* q, const void* k_pages, const void* v_
                         page_size, max_pages_per_seq, num_pages, scale, causal, win_l, softcap,
                         dtype, workspace, workspace_bytes, static_cast<cudaStream_t>(stream),
                         g_split_pages_override.load());
+}
+
+int mfa_decode_phase1(const void* q, const void* k_pages, const void* v_pages,
+                      const int32_t* block_table, const int32_t* seq_lens, int B, int Nq, int Hq,
+                      int Hkv, int D, int page_size, int max_pages_per_seq, int num_pages,
+                      float scale, int causal, int win_l, float softcap, int dtype, int split_lo,
+                      int split_hi, float* part_o, float* part_ml, int split_capacity,
+                      void* stream) {
+  const int ovr = g_split_pages_override.load();
+  mfa::DecodeParams p;
+  DecodePlan pl;
+  int rc = decode_params(p, pl, q, k_pages, v_pages, block_table, seq_lens, nullptr, nullptr, B,
+                         Nq, Hq, Hkv, D, page_size, max_pages_per_seq, num_pages, scale, causal,
+                         win_l, softcap, dtype, ovr, true, false);
+  if (rc != MFA_OK || B == 0) return rc;
+  if (split_lo < 0 || split_hi < split_lo || split_hi > pl.max_splits) return MFA_ERR_BAD_SHAPE;
+  if (split_capacity < pl.max_splits || !part_o || !part_ml) return MFA_ERR_WORKSPACE;
+  if (!aligned16(part_o) || !aligned16(part_ml)) return MFA_ERR_MISALIGNED;
+  p.ws_o = part_o;
+  p.ws_ml = part_ml;
+  p.split_lo = split_lo;
+  return dispatch_decode(p, pl, D, split_hi, kDecPhase1, dtype == MFA_DTYPE_BF16,
+                         static_cast<cudaStream_t>(stream));
+}
+
+int mfa_decode_combine(const int32_t* seq_lens, void* out, float* lse, int B, int Nq, int Hq,
+                       int Hkv, int D, int page_size, int max_pages_per_seq, int win_l, int dtype,
+                       const float* part_o, const float* part_ml, int split_capacity,
+                       void* stream) {
+  const int ovr = g_split_pages_override.load();
+  mfa::DecodeParams p;
+  DecodePlan pl;
+  int rc = decode_params(p, pl, nullptr, nullptr, nullptr, nullptr, seq_lens, out, lse, B, Nq, Hq,
+                         Hkv, D, page_size, max_pages_per_seq, 1, 1.0f, 1, win_l, 0.f, dtype, ovr,
+                         false, true);
+  if (rc != MFA_OK || B == 0) return rc;
+  if (split_capacity < pl.max_splits || !part_o || !part_ml) return MFA_ERR_WORKSPACE;
+  if (!aligned16(part_o) || !aligned16(part_ml)) return MFA_ERR_MISALIGNED;
+  p.ws_o = const_cast<float*>(part_o);
+  p.ws_ml = const_cast<float*>(part_ml);
+  return dispatch_decode(p, pl, D, 0, kDecCombine, dtype == MFA_DTYPE_BF16,
+                         static_cast<cudaStream_t>(stream));
 }
 
 int mfa_decode_splitkv(const void* q, const void* k_pages, const void* v_pages,
