@@ -359,24 +359,36 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     if (lane == 0 && n_act > 0) {
       const uint32_t idesc_qk = idesc_f16(BF16 ? 1 : 0, kFwdBM, kFwdBN, 0);
       const uint32_t idesc_pv = idesc_f16(BF16 ? 1 : 0, kFwdBM, D, 1);
+      // descriptors of the tiles' first bytes, built once (selected, not indexed, so they stay in
+      // registers); each MMA adds a constant offset
+      static_assert(kFwdQT == 2 && kFwdStages == 2, "descriptor selection assumes two of each");
+      const SmemDesc dq0 = smem_desc_sw128_split(smem_u32(sm.q[0]), 16, 1024);
+      const SmemDesc dq1 = smem_desc_sw128_split(smem_u32(sm.q[1]), 16, 1024);
+      const SmemDesc dk0 = smem_desc_sw128_split(smem_u32(sm.k[0]), 16, 1024);
+      const SmemDesc dk1 = smem_desc_sw128_split(smem_u32(sm.k[1]), 16, 1024);
+      const SmemDesc dv0 = smem_desc_sw128_split(smem_u32(sm.v[0]), kSlab, 1024);
+      const SmemDesc dv1 = smem_desc_sw128_split(smem_u32(sm.v[1]), kSlab, 1024);
       auto issue_qk = [&](int t, int s) {
-        const uint32_t qa = smem_u32(sm.q[t]);
-        const uint32_t ka = smem_u32(sm.k[s]);
+        const SmemDesc a = t ? dq1 : dq0, bk = s ? dk1 : dk0;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * kSlab + (kk & 3) * 32;
-          tc_mma_ss(tmem + t * kFwdBN, smem_desc_sw128(qa + koff, 16, 1024),
-                    smem_desc_sw128(ka + koff, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * kSlab + (kk & 3) * 32) >> 4;
+          if (kk == 0)
+            tc_mma_ss_c<0>(tmem + t * kFwdBN, a.lo + off, a.hi, bk.lo + off, bk.hi, idesc_qk);
+          else
+            tc_mma_ss_c<1>(tmem + t * kFwdBN, a.lo + off, a.hi, bk.lo + off, bk.hi, idesc_qk);
         }
       };
       // half h covers keys 64h .. 64h + 63 (P columns 32h .. 32h + 31)
       auto issue_pv = [&](int t, int s, bool acc, int h) {
-        const uint32_t va = smem_u32(sm.v[s]);
+        const SmemDesc bv = s ? dv1 : dv0;
 #pragma unroll
         for (int kk = h * 4; kk < h * 4 + 4; ++kk) {
-          tc_mma_ts(tmem + 256 + t * D, tmem + t * kFwdBN + kk * 8,
-                    smem_desc_sw128(va + kk * 16 * 128, kSlab, 1024), idesc_pv,
-                    (acc || kk > 0) ? 1u : 0u);
+          const uint32_t off = (kk * 16 * 128) >> 4;
+          if (kk == 0 && !acc)
+            tc_mma_ts_c<0>(tmem + 256 + t * D, tmem + t * kFwdBN + kk * 8, bv.lo + off, bv.hi, idesc_pv);
+          else
+            tc_mma_ts_c<1>(tmem + 256 + t * D, tmem + t * kFwdBN + kk * 8, bv.lo + off, bv.hi, idesc_pv);
         }
       };
       // Debug flag bit 2 (failure-detection tests): issue no MMA at all, so the softmax warps'

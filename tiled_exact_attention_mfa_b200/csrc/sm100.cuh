@@ -200,11 +200,22 @@ __device__ __forceinline__ void tmem_reg_fence32(uint32_t (&r)[32]) {
                :
                : "memory");
 }
+__device__ __forceinline__ void tmem_reg_fence16(uint32_t (&r)[16]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
 template <int N>
 __device__ __forceinline__ void tmem_reg_fence(uint32_t (&r)[N]) {
-  static_assert(N % 32 == 0, "fence whole 32-register groups");
+  static_assert(N % 16 == 0, "fence whole 16-register groups");
+  if constexpr (N % 32 == 0) {
 #pragma unroll
-  for (int i = 0; i < N / 32; ++i) tmem_reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&r[32 * i]));
+    for (int i = 0; i < N / 32; ++i) tmem_reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&r[32 * i]));
+  } else {
+#pragma unroll
+    for (int i = 0; i < N / 16; ++i) tmem_reg_fence16(*reinterpret_cast<uint32_t(*)[16]>(&r[16 * i]));
+  }
 }
 template <int N>
 __device__ __forceinline__ void tmem_reg_fence(float (&r)[N]) {
@@ -242,6 +253,42 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo_
 __host__ __device__ constexpr uint32_t idesc_f16(int ab_bf16, int m, int n, int b_mn_major) {
   return (1u << 4) | ((uint32_t)ab_bf16 << 7) | ((uint32_t)ab_bf16 << 10) |
          ((uint32_t)b_mn_major << 16) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+// The same MMAs with the shared-memory descriptors passed as 32-bit halves and the accumulate
+// flag fixed at compile time. A descriptor's low word holds the start address field (bits 0-13,
+// 16-byte units), so the descriptor of an address `bytes` further on is the low word plus
+// bytes >> 4 (no carry: shared-memory addresses are below 2^18); hot issue loops then add one
+// constant per operand instead of rebuilding 64-bit descriptors, and set no predicate.
+struct SmemDesc {
+  uint32_t lo, hi;
+};
+__device__ __forceinline__ SmemDesc smem_desc_sw128_split(uint32_t addr, uint32_t lbo_bytes,
+                                                          uint32_t sbo_bytes) {
+  const uint64_t d = smem_desc_sw128(addr, lbo_bytes, sbo_bytes);
+  return {(uint32_t)d, (uint32_t)(d >> 32)};
+}
+template <int ACC>
+__device__ __forceinline__ void tc_mma_ss_c(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi,
+                                            uint32_t b_lo, uint32_t b_hi, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .b64 ad, bd;\n\t.reg .pred p;\n\t"
+      "mov.b64 ad, {%1, %2};\n\tmov.b64 bd, {%3, %4};\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "n"(ACC)
+      : "memory");
+}
+template <int ACC>
+__device__ __forceinline__ void tc_mma_ts_c(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                            uint32_t b_hi, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .b64 bd;\n\t.reg .pred p;\n\t"
+      "mov.b64 bd, {%2, %3};\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "n"(ACC)
+      : "memory");
 }
 
 // ---------------------------------------------------------------- warp-level MMA (decode)
