@@ -53,6 +53,7 @@ struct FwdParams {
   CUtensorMap tm_q;  // [B*Hq][Nq][D]
   CUtensorMap tm_k;  // [B*Hkv][Nk][D]
   CUtensorMap tm_v;
+  CUtensorMap tm_o;  // out, laid out as q (the epilogue's TMA stores)
   void* out;
   float* lse;
   unsigned long long* tile_counter;
@@ -188,8 +189,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
   const int kt_lo = lo / kFwdBN;
   const int n_tiles = (hi > lo) ? ((hi + kFwdBN - 1) / kFwdBN - kt_lo) : 0;
 
-  // ---- setup
-  if (threadIdx.x == 0) {
+  // ---- setup: the producer thread initialises the barriers and starts the Q load at once, so
+  // the copy overlaps the TMEM allocation, the block-sparse tile list and the CTA barrier
+  const bool q_early = n_tiles > 0;
+  if (warp == 8 && lane == 0) {
     mbar_init(smem_u32(&sm.bar_q), 1);
     for (int s = 0; s < kFwdStages; ++s) {
       mbar_init(smem_u32(&sm.bar_k_full[s]), 1);
@@ -206,6 +209,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     mbar_init(smem_u32(&sm.bar_final), 1);
     sm.abort = 0;
     fence_barrier_init();
+    if (q_early) {
+      tma_prefetch_desc(&p.tm_q);
+      const uint32_t bq = smem_u32(&sm.bar_q);
+      mbar_expect_tx(bq, kFwdQT * (uint32_t)FwdSmem<D, SPARSE>::kTileBytes);
+      for (int t = 0; t < kFwdQT; ++t)
+        for (int sl = 0; sl < D / 64; ++sl)
+          if constexpr (VARLEN)
+            tma_load_3d(smem_u32(sm.q[t]) + sl * FwdSmem<D, SPARSE>::kSlabBytes, &p.tm_q, bq, sl * 64,
+                        h, rq + q0 + t * kFwdBM);
+          else
+            tma_load_3d(smem_u32(sm.q[t]) + sl * FwdSmem<D, SPARSE>::kSlabBytes, &p.tm_q, bq, sl * 64,
+                        q0 + t * kFwdBM, b * p.Hq + h);
+    }
   }
   if (SPARSE && warp == 0) {
     // Active key tiles of the block mask rows of this CTA's two Q tiles, compacted in order:
@@ -262,7 +278,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     tmem_relinquish();
   }
   if (warp == 8 && lane == 0) {
-    tma_prefetch_desc(&p.tm_q);
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_v);
   }
@@ -287,16 +302,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
    regs_control();
    if (warp == 8) {
     // ================================================================ TMA producer
-    if (lane == 0 && n_act > 0) {
-      const uint32_t bq = smem_u32(&sm.bar_q);
-      mbar_expect_tx(bq, kFwdQT * kTileBytes);
-      for (int t = 0; t < kFwdQT; ++t)
-        for (int sl = 0; sl < kSlabs; ++sl)
-          if constexpr (VARLEN)
-            tma_load_3d(smem_u32(sm.q[t]) + sl * kSlab, &p.tm_q, bq, sl * 64, h, rq + q0 + t * kFwdBM);
-          else
-            tma_load_3d(smem_u32(sm.q[t]) + sl * kSlab, &p.tm_q, bq, sl * 64, q0 + t * kFwdBM,
-                        b * p.Hq + h);
+    const uint32_t bq = smem_u32(&sm.bar_q);
+    if (lane == 0 && n_act > 0) {  // (the Q tiles were requested during setup)
       int issued_k[kFwdStages] = {0, 0}, issued_v[kFwdStages] = {0, 0};
       for (int u = 0; u < n_act; ++u) {
         const int s = u % kFwdStages;
@@ -348,11 +355,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       }
       // Make sure no copy into this CTA's shared memory is still in flight when it exits.
       volatile int no_abort = 0;
-      mbar_wait(bq, 0, &no_abort, 803);
       for (int s = 0; s < kFwdStages; ++s) {
         if (issued_k[s] > 0) mbar_wait(smem_u32(&sm.bar_k_full[s]), (issued_k[s] - 1) & 1, &no_abort, 804);
         if (issued_v[s] > 0) mbar_wait(smem_u32(&sm.bar_v_full[s]), (issued_v[s] - 1) & 1, &no_abort, 805);
       }
+    }
+    if (lane == 0 && q_early) {  // the Q copy, also when a block-sparse list came out empty
+      volatile int no_abort = 0;
+      mbar_wait(bq, 0, &no_abort, 803);
     }
   } else if (warp == 9) {
     // ================================================================ MMA issuer
@@ -695,6 +705,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     const size_t orow = VARLEN ? (size_t)(rq + row) * p.Hq + h : (size_t)(b * p.Hq + h) * Nq + row;
     const size_t obase = orow * D;
     const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+    // The normalised tile goes to the Q tile's own buffer (free: its last QK completed before its
+    // last scores were read) in the 128-byte-swizzled layout of the output tensor map, and one
+    // thread writes it with TMA stores: whole 128-byte lines instead of a 16-byte piece of 32
+    // rows per store instruction. Dense rows past Nq fall outside the map and are not written;
+    // a packed tile that runs past its sequence's end is stored row by row instead.
+    const bool tma_out = !VARLEN || (q0 + t * kFwdBM + kFwdBM <= Nq);
+    const uint32_t stage = smem_u32(sm.q[t]);
 #pragma unroll
     for (int cb = 0; cb < D; cb += 32) {
       uint32_t o[32];
@@ -705,17 +722,42 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] = 0u;
       }
-      if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + obase + cb);
+      uint4 w[4];
+#pragma unroll
+      for (int v4 = 0; v4 < 4; ++v4) {
+        w[v4].x = pack2<BF16>(__uint_as_float(o[v4 * 8 + 0]) * inv_l, __uint_as_float(o[v4 * 8 + 1]) * inv_l);
+        w[v4].y = pack2<BF16>(__uint_as_float(o[v4 * 8 + 2]) * inv_l, __uint_as_float(o[v4 * 8 + 3]) * inv_l);
+        w[v4].z = pack2<BF16>(__uint_as_float(o[v4 * 8 + 4]) * inv_l, __uint_as_float(o[v4 * 8 + 5]) * inv_l);
+        w[v4].w = pack2<BF16>(__uint_as_float(o[v4 * 8 + 6]) * inv_l, __uint_as_float(o[v4 * 8 + 7]) * inv_l);
+      }
+      if (tma_out) {
+        // 16-byte chunk ch of row r in a slab sits at r * 128 + (ch ^ (r % 8)) * 16
+        const uint32_t slab = stage + (cb / 64) * kSlab + r * 128;
 #pragma unroll
         for (int v4 = 0; v4 < 4; ++v4) {
-          uint4 w;
-          w.x = pack2<BF16>(__uint_as_float(o[v4 * 8 + 0]) * inv_l, __uint_as_float(o[v4 * 8 + 1]) * inv_l);
-          w.y = pack2<BF16>(__uint_as_float(o[v4 * 8 + 2]) * inv_l, __uint_as_float(o[v4 * 8 + 3]) * inv_l);
-          w.z = pack2<BF16>(__uint_as_float(o[v4 * 8 + 4]) * inv_l, __uint_as_float(o[v4 * 8 + 5]) * inv_l);
-          w.w = pack2<BF16>(__uint_as_float(o[v4 * 8 + 6]) * inv_l, __uint_as_float(o[v4 * 8 + 7]) * inv_l);
-          dst[v4] = w;
+          const int ch = (cb % 64) / 8 + v4;
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(slab + ((ch ^ (r & 7)) << 4)),
+                       "r"(w[v4].x), "r"(w[v4].y), "r"(w[v4].z), "r"(w[v4].w)
+                       : "memory");
         }
+      } else if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + obase + cb);
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) dst[v4] = w[v4];
+      }
+    }
+    if (tma_out) {
+      fence_proxy_async_smem();  // the staged tile, then the TMA engine reads it
+      if (t == 0) named_bar_sync<1, kFwdBM>(); else named_bar_sync<2, kFwdBM>();
+      if (r == 0) {
+        for (int sl = 0; sl < kSlabs; ++sl) {
+          if constexpr (VARLEN)
+            tma_store_3d(&p.tm_o, stage + sl * kSlab, sl * 64, h, rq + q0 + t * kFwdBM);
+          else
+            tma_store_3d(&p.tm_o, stage + sl * kSlab, sl * 64, q0 + t * kFwdBM, b * p.Hq + h);
+        }
+        bulk_commit_group();
+        bulk_wait_group_all();  // the staging buffer is read and the rows written before exit
       }
     }
     if (valid && p.lse != nullptr) {

@@ -279,6 +279,7 @@ int launch_fwd(const FwdCall& c, cudaStream_t st) {
   std::memset(&p, 0, sizeof(p));
   if (PAGED) {
     if (!make_map_packed(&p.tm_q, c.q, dtype, c.total_q, Hq, D)) return MFA_ERR_CUDA;
+    if (!make_map_packed(&p.tm_o, c.out, dtype, c.total_q, Hq, D)) return MFA_ERR_CUDA;
     if (!make_map_pages(&p.tm_k, c.k, dtype, (long long)c.num_pages * 16, Hkv, D)) return MFA_ERR_CUDA;
     if (!make_map_pages(&p.tm_v, c.v, dtype, (long long)c.num_pages * 16, Hkv, D)) return MFA_ERR_CUDA;
     p.cu_q = c.cu_q;
@@ -289,6 +290,7 @@ int launch_fwd(const FwdCall& c, cudaStream_t st) {
     p.num_pages = c.num_pages;
   } else if (VARLEN) {
     if (!make_map_packed(&p.tm_q, c.q, dtype, c.total_q, Hq, D)) return MFA_ERR_CUDA;
+    if (!make_map_packed(&p.tm_o, c.out, dtype, c.total_q, Hq, D)) return MFA_ERR_CUDA;
     if (!make_map_packed(&p.tm_k, c.k, dtype, c.total_k, Hkv, D)) return MFA_ERR_CUDA;
     if (!make_map_packed(&p.tm_v, c.v, dtype, c.total_k, Hkv, D)) return MFA_ERR_CUDA;
     p.cu_q = c.cu_q;
@@ -297,6 +299,7 @@ int launch_fwd(const FwdCall& c, cudaStream_t st) {
     p.total_k = c.total_k;
   } else {
     if (!make_map(&p.tm_q, c.q, dtype, (long long)B * Hq, Nq, D)) return MFA_ERR_CUDA;
+    if (!make_map(&p.tm_o, c.out, dtype, (long long)B * Hq, Nq, D)) return MFA_ERR_CUDA;
     if (!make_map(&p.tm_k, c.k, dtype, (long long)B * Hkv, Nk, D)) return MFA_ERR_CUDA;
     if (!make_map(&p.tm_v, c.v, dtype, (long long)B * Hkv, Nk, D)) return MFA_ERR_CUDA;
   }
