@@ -195,6 +195,7 @@ def test_decode_plan_without_window():
     assert p == {"pages_per_split": 32, "max_splits": 256, "kv_heads_per_cta": 4}
     assert mfa.mfa_decode_workspace_size(8, 1, 32, 8, 128, 8192) == 8 * 256 * 32 * (128 + 2) * 4
     assert mfa.mfa_decode_plan(8, 4, 32, 8, 128, 8192)["max_splits"] == 256  # N_q does not move it
+    assert mfa.mfa_decode_workspace_size(8, 4, 32, 8, 128, 8192) == 8 * 256 * 128 * (128 + 2) * 4
     assert mfa.mfa_decode_plan(8, 1, 16, 8, 256, 2048)["kv_heads_per_cta"] == 2
     assert mfa.mfa_decode_plan(8, 1, 32, 8, 64, 2048)["kv_heads_per_cta"] == 8
     assert mfa.mfa_decode_plan(8, 1, 21, 7, 128, 2048)["kv_heads_per_cta"] == 1  # 7 x 256 B > 1 KB

@@ -330,8 +330,10 @@ __global__ void __launch_bounds__((kDecMaxHeads<D> + 1) * 32) mfa_decode_phase1_
 
 // Threads per combine CTA. Each thread owns 4 consecutive output columns (one 16-byte load per
 // split), so a group of D / 4 threads covers a row and there are G = 4 * kCombineThreads / D
-// groups; group g takes splits g, g + G, g + 2G, ...
-constexpr int kCombineThreads = 512;
+// groups; group g takes splits g, g + G, g + 2G, ... At 256 threads two CTAs share an SM, so one
+// CTA's merge and store overlap the other's loads (with 512 threads, one CTA per SM, the SM had
+// no load in flight between CTAs: 32 us for the 1,024 rows of the 4-token verify workload).
+constexpr int kCombineThreads = 256;
 // Splits a thread loads before folding them into its running statistics: all their loads are
 // issued together, so a sequence of n splits costs about n / (G * kCombineBatch) memory round trips.
 constexpr int kCombineBatch = 8;

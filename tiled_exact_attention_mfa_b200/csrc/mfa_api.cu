@@ -200,7 +200,8 @@ DecodePlan decode_plan(int B, int Hkv, int D, int max_pages, int Nq, int win_l, 
       break;
     }
   pl.groups = Hkv / pl.heads_per_cta;
-  int s = 32;
+  const int s0 = 32;
+  int s = s0;
   if (override_pages > 0) {
     s = std::min(override_pages, mfa::kDecMaxSplitPages);
   } else {
@@ -214,7 +215,7 @@ DecodePlan decode_plan(int B, int Hkv, int D, int max_pages, int Nq, int win_l, 
     const int span = (int)std::min<long long>(max_pages, win_pages);
     const int cap = pl.max_splits;
     if (override_pages <= 0) {
-      s = 32;
+      s = s0;
       while (s > 4 && (long long)B * ((span + s / 2 - 1) / (s / 2)) * pl.groups <= 296 &&
              (span + s / 2 - 1) / (s / 2) <= cap)
         s /= 2;
@@ -743,7 +744,7 @@ namespace {
 size_t decode_workspace_size(int B, int Nq, int Hq, int Hkv, int D, int max_pages_per_seq,
                              int page_size, int override_pages) {
   if (validate_decode(B, Nq, Hq, Hkv, D, page_size, max_pages_per_seq) != MFA_OK) return 0;
-  DecodePlan pl = decode_plan(B, Hkv, D, max_pages_per_seq, 1, -1, override_pages);
+  DecodePlan pl = decode_plan(B, Hkv, D, max_pages_per_seq, Nq, -1, override_pages);
   const size_t rows = (size_t)B * pl.max_splits * Hq * Nq;
   return align256(rows * D * sizeof(float)) + align256(rows * 2 * sizeof(float));
 }
@@ -822,7 +823,7 @@ int decode_splitkv(const void* q, const void* k_pages, const void* v_pages,
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
     return MFA_ERR_WORKSPACE;
   // the unwindowed plan sizes the workspace; a window's plan never has more splits
-  const DecodePlan full = decode_plan(B, Hkv, D, max_pages_per_seq, 1, -1, override_pages);
+  const DecodePlan full = decode_plan(B, Hkv, D, max_pages_per_seq, Nq, -1, override_pages);
   const size_t rows = (size_t)B * full.max_splits * Hq * Nq;
   p.ws_o = static_cast<float*>(workspace);
   p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(rows * D * sizeof(float)));
