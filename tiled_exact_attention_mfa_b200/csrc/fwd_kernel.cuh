@@ -29,8 +29,10 @@
 // j is done and O_t can be rescaled in place.
 //
 // Tile skip ("mlx-mfa 2.5.2", Features: causal tile-skip, window_size=(left,right) tile skip):
-// each CTA visits only key tiles that intersect the union of its rows' visible ranges; inside,
-// masking is applied per element only on tiles that are not fully visible to all 128 rows.
+// each CTA visits only key tiles that intersect the union of its rows' visible ranges, and each
+// of its Q tiles computes only those that intersect its own rows' range (the two differ by up to
+// a tile at each end: the causal diagonal, the window's edges); inside, masking is applied per
+// element only on tiles that are not fully visible to all 128 rows.
 #pragma once
 #include "sm100.cuh"
 
@@ -130,8 +132,14 @@ __device__ __forceinline__ void key_range(const FwdParams& p, int Nk, int a0, in
 // sequence are loaded from past the pool's end, which TMA fills with zeros. Value rows at or past
 // the length inside the last page may hold anything, so before P of that tile is released the
 // first softmax warpgroup zeroes them in shared memory (P is 0 there, but 0 x NaN is NaN).
-template <int D, bool BF16, bool VARLEN, bool SPARSE, bool SOFTCAP, bool PAGED>
+// PART (dense layout): each Q tile computes only the key tiles its own rows can see, instead of
+// every tile of the CTA's range; chosen for sliding windows, where the two Q tiles' ranges
+// differ by a tile at each end (elsewhere the saving is one diagonal tile per CTA, less than what
+// the extra bookkeeping costs the plain loop).
+template <int D, bool BF16, bool VARLEN, bool SPARSE, bool SOFTCAP, bool PAGED, bool PART = false>
 __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_constant__ FwdParams p) {
+  constexpr bool kRuns = PART && !SPARSE;  // Q tile t takes part in the run [jlo_t, jhi_t)
+  constexpr bool kPart = SPARSE || kRuns;  // a Q tile may sit out some visited tiles
   static_assert(!(VARLEN && SPARSE), "block masks are defined on the dense layout");
   static_assert(!PAGED || VARLEN, "paged keys come with packed queries");
   extern __shared__ uint8_t smem_raw[];
@@ -188,6 +196,34 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
   }
   const int kt_lo = lo / kFwdBN;
   const int n_tiles = (hi > lo) ? ((hi + kFwdBN - 1) / kFwdBN - kt_lo) : 0;
+  // each Q tile's own visible key range: a key tile it cannot see at all is not its to visit
+  // (the two Q tiles' ranges differ by up to a tile at each end: causal diagonal, window edges)
+  int vlo0, vhi0, vlo1, vhi1;  // (scalars, not arrays: selected, never indexed)
+  {
+    int vlo[kFwdQT], vhi[kFwdQT];
+#pragma unroll
+    for (int t = 0; t < kFwdQT; ++t) {
+      const int f = q0 + t * kFwdBM, l = min(f + kFwdBM, Nq) - 1;
+      if (l < f) {
+        vlo[t] = 1;
+        vhi[t] = 0;
+      } else if (p.flags & 1) {
+        vlo[t] = 0;
+        vhi[t] = Nk;
+      } else {
+        key_range(p, Nk, f + off, l + off, vlo[t], vhi[t]);
+      }
+    }
+    vlo0 = vlo[0];
+    vhi0 = vhi[0];
+    vlo1 = vlo[1];
+    vhi1 = vhi[1];
+  }
+  // bit t: Q tile t takes part in key tile kt (intersects its visible range)
+  auto vis_bits = [&](int kt) -> uint32_t {
+    const int k0 = kt * kFwdBN;
+    return ((k0 < vhi0 && k0 + kFwdBN > vlo0) ? 1u : 0u) | ((k0 < vhi1 && k0 + kFwdBN > vlo1) ? 2u : 0u);
+  };
 
   // ---- setup: the producer thread initialises the barriers and starts the Q load at once, so
   // the copy overlaps the TMEM allocation, the block-sparse tile list and the CTA barrier
@@ -229,30 +265,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     const int qt0 = q0 / kFwdBM;
     const uint8_t* r0 = p.block_mask + ((size_t)(b * p.Hq + h) * p.nqt + qt0) * p.nkt + kt_lo;
     const uint8_t* r1 = (qt0 + 1 < p.nqt) ? r0 + p.nkt : nullptr;
-    // each Q tile's own visible key range: a tile it cannot see at all is not its to visit
-    int vlo[kFwdQT], vhi[kFwdQT];
-#pragma unroll
-    for (int t = 0; t < kFwdQT; ++t) {
-      const int f = q0 + t * kFwdBM, l = min(f + kFwdBM, Nq) - 1;
-      if (l < f) {
-        vlo[t] = 1;
-        vhi[t] = 0;
-      } else if (p.flags & 1) {
-        vlo[t] = 0;
-        vhi[t] = Nk;
-      } else {
-        key_range(p, Nk, f + off, l + off, vlo[t], vhi[t]);
-      }
-    }
     int count = 0;
     for (int base = 0; base < n_tiles; base += 32 * 8) {
       uint8_t a0[8], a1[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int jj = base + i * 32 + lane;
-        const int k0 = (kt_lo + jj) * kFwdBN;
-        a0[i] = (jj < n_tiles && k0 < vhi[0] && k0 + kFwdBN > vlo[0]) ? r0[jj] : 0;
-        a1[i] = (r1 != nullptr && jj < n_tiles && k0 < vhi[1] && k0 + kFwdBN > vlo[1]) ? r1[jj] : 0;
+        const uint32_t vb = vis_bits(kt_lo + jj);
+        a0[i] = (jj < n_tiles && (vb & 1u)) ? r0[jj] : 0;
+        a1[i] = (r1 != nullptr && jj < n_tiles && (vb & 2u)) ? r1[jj] : 0;
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -289,6 +310,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
   const int n_act = SPARSE ? sm.n_act : n_tiles;
   auto tile_of = [&](int u) -> int {
     if constexpr (SPARSE) return sm.act_tile[u]; else return u;
+  };
+  // bit t of visited tile u: Q tile t takes part in it (block-sparse: its block is on as well)
+  // Dense: Q tile t's visited tiles are the contiguous run [jlo_t, jhi_t) of the CTA's.
+  const int jlo0 = min(n_tiles, max(0, vlo0 / kFwdBN - kt_lo));
+  const int jhi0 = max(jlo0, min(n_tiles, (vhi0 + kFwdBN - 1) / kFwdBN - kt_lo));
+  const int jlo1 = min(n_tiles, max(0, vlo1 / kFwdBN - kt_lo));
+  const int jhi1 = max(jlo1, min(n_tiles, (vhi1 + kFwdBN - 1) / kFwdBN - kt_lo));
+  auto bits_of = [&](int u) -> uint32_t {  // bit t: Q tile t takes part in visited tile u
+    if constexpr (SPARSE) return sm.act_bits[u];
+    else if constexpr (kRuns) return ((u >= jlo0 && u < jhi0) ? 1u : 0u) | ((u >= jlo1 && u < jhi1) ? 2u : 0u);
+    else return 3u;
   };
   if (threadIdx.x == 0 && (p.flags & 2) && n_act > 0)
     atomicAdd(p.tile_counter, (unsigned long long)n_act);
@@ -405,20 +437,38 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       // first wait for S runs out; the bounded waits then take the abort path below.
       const bool withhold = (p.flags & 4) != 0;
       bool ok = !withhold && mbar_wait(smem_u32(&sm.bar_q), 0, abort, 901);
-      // Block-sparse: Q tile t takes part in visited tile u only where its bit is on; its MMAs
-      // are skipped elsewhere and its barriers count only the tiles it takes part in. (Dense:
-      // every Q tile takes part in every tile, and the counts below are the loop index.)
-      // the bits of tile j + 1 are read at the top of iteration j, ahead of the waits, and
-      // carried into iteration j + 1 (a shared load after a wait would sit on the issue path)
-      uint32_t bits_cur = SPARSE ? sm.act_bits[0] : 3u, bits_next = 3u;
+      // Q tile t takes part in visited tile u only where its bit is on; its MMAs are skipped
+      // elsewhere and its barriers count only the tiles it takes part in. The bits of tile j + 1
+      // are taken at the top of iteration j, ahead of the waits, and carried into iteration j + 1
+      // (a shared load after a wait would sit on the issue path).
+      // (Dense: the runs [jlo_t, jhi_t) give the same answers in closed form.)
+      uint32_t bits_cur = SPARSE ? sm.act_bits[0] : 0u, bits_next = 0u;
+      int j = 0;
       auto act_cur = [&](int t) -> bool {  // Q tile t takes part in tile j
-        if constexpr (SPARSE) return ((bits_cur >> t) & 1u) != 0; else return true;
+        if constexpr (!kPart) return true;
+        else if constexpr (SPARSE) return ((bits_cur >> t) & 1u) != 0;
+        else return t ? (j >= jlo1 && j < jhi1) : (j >= jlo0 && j < jhi0);
       };
       auto act_next = [&](int t) -> bool {  // ... in tile j + 1
-        if constexpr (SPARSE) return ((bits_next >> t) & 1u) != 0; else return true;
+        if constexpr (!kPart) return true;
+        else if constexpr (SPARSE) return ((bits_next >> t) & 1u) != 0;
+        else return t ? (j + 1 >= jlo1 && j + 1 < jhi1) : (j + 1 >= jlo0 && j + 1 < jhi0);
       };
-      int npv[kFwdQT] = {0, 0};  // PV groups issued per Q tile (SPARSE only)
-      for (int j = 0; ok && j < n_act; ++j) {  // j counts visited tiles
+      int npv0 = 0, npv1 = 0;  // PV groups issued so far per Q tile (block-sparse)
+      // PV groups of Q tile t issued before tile j (dense: closed form; block-sparse: the count,
+      // read before this tile's PV adds to it)
+      auto pv_before = [&](int t) -> int {
+        if constexpr (!kPart) return j;
+        else if constexpr (SPARSE) return t ? npv1 : npv0;
+        else return t ? max(0, min(j, jhi1) - jlo1) : max(0, min(j, jhi0) - jlo0);
+      };
+      // ... issued up to and including tile j (block-sparse: read after this tile's PV)
+      auto pv_through = [&](int t) -> int {
+        if constexpr (!kPart) return j + 1;
+        else if constexpr (SPARSE) return t ? npv1 : npv0;
+        else return t ? max(0, min(j + 1, jhi1) - jlo1) : max(0, min(j + 1, jhi0) - jlo0);
+      };
+      for (; ok && j < n_act; ++j) {  // j counts visited tiles
         const int s = j % kFwdStages;
         const uint32_t ph = (j / kFwdStages) & 1;
         const int s1 = (j + 1) % kFwdStages;
@@ -444,7 +494,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         // Q tile 0: PV(j), then QK(j+1) once PV(j) is done (P_0 lives in S_0's columns)
         if (!(ok = mbar_wait(smem_u32(&sm.bar_v_full[s]), ph, abort, 903))) break;
         if (act_cur(0)) {
-          const int c = SPARSE ? npv[0] : j;
+          const int c = pv_before(0);
           if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[0][0]), c & 1, abort, 904))) break;
           tc_fence_after();
           issue_pv(0, s, c > 0, 0);
@@ -452,14 +502,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
           tc_fence_after();
           issue_pv(0, s, true, 1);
           tc_commit(smem_u32(&sm.bar_o_done[0]));
-          ++npv[0];
+          ++npv0;
         }
         if (more) {
           if (!(ok = mbar_wait(smem_u32(&sm.bar_k_full[s1]), ph1, abort, 905))) break;
           if (act_next(0)) {
             // the latest PV of Q tile 0 read P_0 from S_0's columns
-            if (!SPARSE || npv[0] > 0)
-              if (!(ok = mbar_wait(smem_u32(&sm.bar_o_done[0]), (SPARSE ? npv[0] - 1 : j) & 1, abort, 906))) break;
+            const int n_pv = pv_through(0);
+            if (n_pv > 0)
+              if (!(ok = mbar_wait(smem_u32(&sm.bar_o_done[0]), (n_pv - 1) & 1, abort, 906))) break;
             tc_fence_after();
             issue_qk(0, s1);
             tc_commit(smem_u32(&sm.bar_s_full[0]));
@@ -467,7 +518,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         }
         // Q tile 1
         if (act_cur(1)) {
-          const int c = SPARSE ? npv[1] : j;
+          const int c = pv_before(1);
           if (!(ok = mbar_wait(smem_u32(&sm.bar_p_full[1][0]), c & 1, abort, 907))) break;
           tc_fence_after();
           issue_pv(1, s, c > 0, 0);
@@ -475,13 +526,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
           tc_fence_after();
           issue_pv(1, s, true, 1);
           tc_commit(smem_u32(&sm.bar_o_done[1]));
-          ++npv[1];
+          ++npv1;
         }
         tc_commit(smem_u32(&sm.bar_v_empty[s]));
         if (more) {
           if (act_next(1)) {
-            if (!SPARSE || npv[1] > 0)
-              if (!(ok = mbar_wait(smem_u32(&sm.bar_o_done[1]), (SPARSE ? npv[1] - 1 : j) & 1, abort, 908))) break;
+            const int n_pv = pv_through(1);
+            if (n_pv > 0)
+              if (!(ok = mbar_wait(smem_u32(&sm.bar_o_done[1]), (n_pv - 1) & 1, abort, 908))) break;
             tc_fence_after();
             issue_qk(1, s1);
             tc_commit(smem_u32(&sm.bar_s_full[1]));
@@ -512,12 +564,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     float m_run = -INFINITY;  // running max of the stored (scaled, capped) score
     float l_run = 0.f;
 
-    int nt = 0;  // tiles this Q tile took part in (block-sparse: its bit on); dense: nt == j
-    for (int j = 0; j < n_act; ++j) {  // j counts visited tiles
-      if constexpr (SPARSE) {
-        if (!((sm.act_bits[j] >> t) & 1)) continue;  // not this Q tile's: no S, no P for it
-      }
-      const int c_t = SPARSE ? nt : j;
+    // block-sparse: every visited tile, skipping those without this Q tile's bit; dense: the
+    // contiguous run of tiles this Q tile takes part in
+    const int j_first = kRuns ? (t ? jlo1 : jlo0) : 0;
+    const int j_end = kRuns ? (t ? jhi1 : jhi0) : n_act;
+    int nt = 0;  // tiles this Q tile took part in
+    for (int j = j_first; j < j_end; ++j) {  // j counts visited tiles
+      const uint32_t bj = bits_of(j);
+      if (SPARSE && !((bj >> t) & 1u)) continue;  // not this Q tile's: no S, no P for it
+      const int c_t = kPart ? nt : j;
       const bool got = mbar_wait(smem_u32(&sm.bar_s_full[t]), c_t & 1, abort, 1001 + t);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
@@ -617,8 +672,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       // P = exp2(s * c - m * c) on fp32 pairs, packed to the input type and stored to TMEM 16
       // columns at a time; each half of P is announced as soon as it is stored.
       if constexpr (PAGED) {
-        // the final tile: value rows at or past the length (inside the last page) become 0
-        if (t == 0 && k0 + kFwdBN > Nk) {
+        // the final tile: value rows at or past the length (inside the last page) become 0, by
+        // the first Q tile taking part in it (each PV of the tile comes after that one's P)
+        if (t == ((bj & 1u) ? 0 : 1) && k0 + kFwdBN > Nk) {
           const int vs = j % kFwdStages;
           const bool vok = mbar_wait(smem_u32(&sm.bar_v_full[vs]), (j / kFwdStages) & 1, abort, 1009);
           if (!__all_sync(0xffffffffu, vok)) break;
@@ -693,7 +749,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
 
     // ---- epilogue: O / l, LSE
     bool have_o = false;
-    const int n_t = SPARSE ? nt : n_act;  // PV groups of this Q tile
+    const int n_t = kPart ? nt : n_act;  // PV groups of this Q tile
     if (n_t > 0 && !*abort) {
       have_o = mbar_wait(smem_u32(&sm.bar_o_done[t]), (n_t - 1) & 1, abort, 1003 + t);
       tc_fence_after();
@@ -712,6 +768,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     // a packed tile that runs past its sequence's end is stored row by row instead.
     const bool tma_out = !VARLEN || (q0 + t * kFwdBM + kFwdBM <= Nq);
     const uint32_t stage = smem_u32(sm.q[t]);
+    if (tma_out && q_early && n_t == 0) {
+      // A Q tile that took part in no key tile never waited for S, so the Q load into the
+      // buffer about to be overwritten may still be landing: wait for it first.
+      volatile int no_abort = 0;
+      mbar_wait(smem_u32(&sm.bar_q), 0, &no_abort, 1010);
+    }
 #pragma unroll
     for (int cb = 0; cb < D; cb += 32) {
       uint32_t o[32];

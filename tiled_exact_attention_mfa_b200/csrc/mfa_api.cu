@@ -254,14 +254,14 @@ struct FwdCall {
   int max_pages, num_pages;
 };
 
-template <int D, bool BF16, bool VARLEN, bool SPARSE, bool SOFTCAP, bool PAGED>
+template <int D, bool BF16, bool VARLEN, bool SPARSE, bool SOFTCAP, bool PAGED, bool PART>
 int launch_fwd(const FwdCall& c, cudaStream_t st) {
   const int B = c.B, Hq = c.Hq, Hkv = c.Hkv, Nq = c.Nq, Nk = c.Nk, dtype = c.dtype;
   const float scale = c.scale, softcap = c.softcap;
   static bool smem_done[kMaxDevices] = {};
   static bool regs_ok[kMaxDevices] = {};
   constexpr int smem = mfa::fwd_smem_bytes<D, SPARSE>();
-  auto kernel = mfa::mfa_fwd_kernel<D, BF16, VARLEN, SPARSE, SOFTCAP, PAGED>;
+  auto kernel = mfa::mfa_fwd_kernel<D, BF16, VARLEN, SPARSE, SOFTCAP, PAGED, PART>;
   if (!ensure_smem(kernel, smem, smem_done)) return MFA_ERR_CUDA;
   {
     // setmaxnreg redistributes the registers the CTA launched with; refuse to launch if the
@@ -465,20 +465,21 @@ int launch_fill_empty(void* out, float* lse, size_t rows, int D, int dtype, cuda
   return MFA_OK;
 }
 
-template <bool VARLEN, bool SPARSE, bool SOFTCAP, bool PAGED>
+template <bool VARLEN, bool SPARSE, bool SOFTCAP, bool PAGED, bool PART>
 int dispatch_fwd_d(const FwdCall& c, int D, cudaStream_t st) {
   const bool bf = c.dtype == MFA_DTYPE_BF16;
   if (D == 128)
-    return bf ? launch_fwd<128, true, VARLEN, SPARSE, SOFTCAP, PAGED>(c, st)
-              : launch_fwd<128, false, VARLEN, SPARSE, SOFTCAP, PAGED>(c, st);
-  return bf ? launch_fwd<64, true, VARLEN, SPARSE, SOFTCAP, PAGED>(c, st)
-            : launch_fwd<64, false, VARLEN, SPARSE, SOFTCAP, PAGED>(c, st);
+    return bf ? launch_fwd<128, true, VARLEN, SPARSE, SOFTCAP, PAGED, PART>(c, st)
+              : launch_fwd<128, false, VARLEN, SPARSE, SOFTCAP, PAGED, PART>(c, st);
+  return bf ? launch_fwd<64, true, VARLEN, SPARSE, SOFTCAP, PAGED, PART>(c, st)
+            : launch_fwd<64, false, VARLEN, SPARSE, SOFTCAP, PAGED, PART>(c, st);
 }
 
-template <bool VARLEN, bool SPARSE, bool PAGED = false>
+// PART: each Q tile of a CTA computes only the key tiles its own rows see (dense sliding windows)
+template <bool VARLEN, bool SPARSE, bool PAGED = false, bool PART = false>
 int dispatch_fwd(const FwdCall& c, int D, cudaStream_t st) {
-  return c.softcap > 0.f ? dispatch_fwd_d<VARLEN, SPARSE, true, PAGED>(c, D, st)
-                         : dispatch_fwd_d<VARLEN, SPARSE, false, PAGED>(c, D, st);
+  return c.softcap > 0.f ? dispatch_fwd_d<VARLEN, SPARSE, true, PAGED, PART>(c, D, st)
+                         : dispatch_fwd_d<VARLEN, SPARSE, false, PAGED, PART>(c, D, st);
 }
 
 template <int D, bool BF16, bool SOFTCAP>
@@ -558,6 +559,7 @@ int mfa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, 
   clamp_window(win_l, win_r, Nk, Nq);
   FwdCall c = {q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, scale, causal, win_l, win_r, softcap, dtype,
                nullptr, nullptr, 0, 0, nullptr, nullptr, nullptr, 0, 0};
+  if (win_l >= 0 || win_r >= 0) return dispatch_fwd<false, false, false, true>(c, D, st);
   return dispatch_fwd<false, false>(c, D, st);
 }
 
