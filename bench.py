@@ -688,6 +688,7 @@ def run_gpu(args):
                        "exchange_bytes_per_gpu": r["exchange_bytes"], "scaling": "strong",
                        "parallelism": f"splits of every sequence over {world} GPUs, NCCL all-gather "
                                       "of the (o, m, l) partials, combine on every GPU"})
+    if not args.only_main:
         for name in BACKWARD_WORKLOADS:
             sk, wu = max(3, min(args.steps, 10)), max(3, args.warmup)
             r = bench_backward(W[name], sk, wu, flush, stream, world)
