@@ -19,7 +19,8 @@
 //   query tiles that can see the keys): S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = 128
 //   queries, K = D, operands K-major in smem), then dV += P^T dO and dK += dS^T Q (P^T, dS^T
 //   from TMEM; dO, Q read MN-major from the same smem tiles). TMEM: S^T [0,128), dP^T
-//   [128,256), dV [256,256+D), dK [256+D,256+2D).
+//   [128,256), dV [256,256+D), dK [256+D,256+2D); P^T and dS^T are packed over the dP^T
+//   columns, so S^T of the next query tile is computed while the warps work on this one.
 // dQ pass (CTA = 128 query rows of one head; loops over the key tiles the rows can see):
 //   S = Q K^T, dP = dO V^T, then dQ += dS K (dS from TMEM, K MN-major). TMEM: S [0,128),
 //   dP [128,256), dQ [256,256+D).
@@ -113,10 +114,11 @@ __device__ __forceinline__ float bwd_tanh(float y, bool poly) {
 // ---------------------------------------------------------------- dKV pass
 // 384 threads: warps 0-7 elementwise (warp w: key rows on TMEM lanes 32 (w % 4) .., query
 // columns 64 (w / 4) .. of each query tile), warp 8 producer, warp 9 MMA issuer, warps 10-11
-// idle; setmaxnreg as in the dQ pass. Each warp writes its 64 packed P^T (dS^T) values over
-// the first 32 of its own 64 S^T (dP^T) columns, so the two halves of a row never touch each
-// other's columns; the dV / dK MMAs take query steps 0-3 from columns 0-31 and steps 4-7 from
-// columns 64-95 of each region.
+// idle; setmaxnreg as in the dQ pass. Each warp first reads its S^T values of both 32-column
+// chunks (after which S^T of the next query tile may overwrite them), then per chunk reads the
+// chunk's 32 dP^T columns and writes the chunk's packed P^T and dS^T (16 columns each) over
+// them, so the two halves of a row never touch each other's columns; the dV / dK MMAs take
+// query steps 2 ch + {0, 1} of half hf from columns 128 + 64 hf + 32 ch (+ 16 for dS^T).
 constexpr int kBwdKvThreads = 384;
 
 template <int D>
@@ -129,7 +131,9 @@ struct BwdKvSmem {
   float nl[kBwdStages][kBwdBM];  // -L_i log2 e of the stage's query rows (0 past Nq / no key)
   float dd[kBwdStages][kBwdBM];  // D_i of the stage's query rows
   uint64_t bar_kv, bar_full[kBwdStages], bar_empty[kBwdStages];
-  uint64_t bar_sp, bar_ds[2], bar_mm, bar_final;  // bar_ds[ch]: chunk ch of every warp stored
+  // bar_sfree: every elementwise warp has read its S^T (both chunks); bar_ds[ch]: chunk ch of
+  // every warp stored; bar_sp: S^T and dP^T of the step ready; bar_mm: dV / dK of the step done
+  uint64_t bar_sp, bar_sfree, bar_ds[2], bar_mm, bar_final;
   uint32_t tmem_base;
   int abort;
 };
@@ -181,6 +185,7 @@ __global__ void __launch_bounds__(kBwdKvThreads, 1) mfa_bwd_dkv_kernel(const __g
       mbar_init(smem_u32(&sm.bar_empty[st]), 1);
     }
     mbar_init(smem_u32(&sm.bar_sp), 1);
+    mbar_init(smem_u32(&sm.bar_sfree), 8);
     mbar_init(smem_u32(&sm.bar_ds[0]), 8);
     mbar_init(smem_u32(&sm.bar_ds[1]), 8);
     mbar_init(smem_u32(&sm.bar_mm), 1);
@@ -263,24 +268,42 @@ __global__ void __launch_bounds__(kBwdKvThreads, 1) mfa_bwd_dkv_kernel(const __g
       const uint32_t id_s = idesc_f16(BF16 ? 1 : 0, kBwdBM, kBwdBM, 0);  // S^T, dP^T: 128 x 128
       const uint32_t id_o = idesc_f16(BF16 ? 1 : 0, kBwdBM, D, 1);       // dV, dK: B MN-major
       const uint32_t ka = smem_u32(sm.k), va = smem_u32(sm.v);
-      bool ok = mbar_wait(smem_u32(&sm.bar_kv), 0, abort, 1201);
-      for (int u = 0; ok && u < n_steps; ++u) {
-        const int st = u % kBwdStages;
-        if (!(ok = mbar_wait(smem_u32(&sm.bar_full[st]), (u / kBwdStages) & 1, abort, 1202))) break;
-        // P^T / dS^T of step u - 1 live in the S^T / dP^T columns until dV / dK have read them
-        if (u > 0 && !(ok = mbar_wait(smem_u32(&sm.bar_mm), (u - 1) & 1, abort, 1203))) break;
-        tc_fence_after();
-        const uint32_t qa = smem_u32(sm.q[st]), oa = smem_u32(sm.dout[st]);
+      // S^T = K Q^T of the tile in stage st into columns [0, 128); dP^T = V dO^T into [128, 256)
+      auto issue_s = [&](int st) {
+        const uint32_t qa = smem_u32(sm.q[st]);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           tc_mma_ss(tmem + 0, bwd_desc_k(ka, kk), bwd_desc_k(qa, kk), id_s, kk > 0 ? 1u : 0u);
+      };
+      auto issue_dp = [&](int st) {
+        const uint32_t oa = smem_u32(sm.dout[st]);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           tc_mma_ss(tmem + 128, bwd_desc_k(va, kk), bwd_desc_k(oa, kk), id_s, kk > 0 ? 1u : 0u);
+      };
+      // Per step u: dV / dK of step u chunk by chunk; S^T of step u + 1 between the two chunks
+      // when its Q tile has landed (every warp has read S^T of step u by then, and P^T / dS^T of
+      // step u go to the dP^T columns, so the S^T columns are free): it runs while the warps
+      // compute the second chunk; otherwise right after the second chunk's dV / dK. Then, once
+      // dV / dK have read P^T / dS^T, dP^T of step u + 1 and the commit that releases the warps
+      // into step u + 1.
+      bool ok = mbar_wait(smem_u32(&sm.bar_kv), 0, abort, 1201) &&
+                mbar_wait(smem_u32(&sm.bar_full[0]), 0, abort, 1202);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        issue_dp(0);
         tc_commit(smem_u32(&sm.bar_sp));
-        // packed P^T / dS^T of query step kk (16 queries): half kk / 4 at column 64 (kk / 4),
-        // written by chunk (kk / 2) % 2 of that half's warps. The steps of chunk 0 go to the
-        // tensor pipe while the elementwise warps still work on chunk 1 (disjoint columns).
+      }
+      for (int u = 0; ok && u < n_steps; ++u) {
+        const int st = u % kBwdStages;
+        const int st1 = (u + 1) % kBwdStages;
+        const bool more = u + 1 < n_steps;
+        const uint32_t qa = smem_u32(sm.q[st]), oa = smem_u32(sm.dout[st]);
+        const uint32_t ph1 = ((u + 1) / kBwdStages) & 1;
+        bool s_next = false;  // S^T of step u + 1 issued
+        // packed P^T / dS^T of query step kk (16 queries) of half hf = kk / 4, chunk ch =
+        // (kk / 2) % 2: P^T at column 128 + 64 hf + 32 ch + 8 (kk % 2), dS^T 16 columns further
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
           if (!(ok = mbar_wait(smem_u32(&sm.bar_ds[ch]), u & 1, abort, 1204 + ch))) break;
@@ -290,7 +313,7 @@ __global__ void __launch_bounds__(kBwdKvThreads, 1) mfa_bwd_dkv_kernel(const __g
 #pragma unroll
             for (int k2 = 0; k2 < 2; ++k2) {
               const int kk = hf * 4 + ch * 2 + k2;
-              tc_mma_ts(tmem + 256, tmem + (kk >> 2) * 64 + (kk & 3) * 8, bwd_desc_mn(oa, kk),
+              tc_mma_ts(tmem + 256, tmem + 128 + hf * 64 + ch * 32 + k2 * 8, bwd_desc_mn(oa, kk),
                         id_o, (u > 0 || kk > 0) ? 1u : 0u);
             }
 #pragma unroll
@@ -298,13 +321,33 @@ __global__ void __launch_bounds__(kBwdKvThreads, 1) mfa_bwd_dkv_kernel(const __g
 #pragma unroll
             for (int k2 = 0; k2 < 2; ++k2) {
               const int kk = hf * 4 + ch * 2 + k2;
-              tc_mma_ts(tmem + 256 + D, tmem + 128 + (kk >> 2) * 64 + (kk & 3) * 8,
+              tc_mma_ts(tmem + 256 + D, tmem + 128 + hf * 64 + ch * 32 + 16 + k2 * 8,
                         bwd_desc_mn(qa, kk), id_o, (u > 0 || kk > 0) ? 1u : 0u);
             }
+          if (ch == 0 && more && mbar_test_wait(smem_u32(&sm.bar_full[st1]), ph1)) {
+            // (every warp arrived on bar_sfree before its chunk-0 arrival: no real wait)
+            if (!(ok = mbar_wait(smem_u32(&sm.bar_sfree), u & 1, abort, 1206))) break;
+            tc_fence_after();
+            issue_s(st1);
+            s_next = true;
+          }
         }
         if (!ok) break;
         tc_commit(smem_u32(&sm.bar_mm));
         tc_commit(smem_u32(&sm.bar_empty[st]));
+        if (more) {
+          if (!s_next) {
+            if (!(ok = mbar_wait(smem_u32(&sm.bar_full[st1]), ph1, abort, 1202))) break;
+            if (!(ok = mbar_wait(smem_u32(&sm.bar_sfree), u & 1, abort, 1206))) break;
+            tc_fence_after();
+            issue_s(st1);
+          }
+          // dP^T of step u + 1 overwrites the packed P^T / dS^T that dV / dK of step u read
+          if (!(ok = mbar_wait(smem_u32(&sm.bar_mm), u & 1, abort, 1203))) break;
+          tc_fence_after();
+          issue_dp(st1);
+          tc_commit(smem_u32(&sm.bar_sp));  // also covers S^T of step u + 1
+        }
       }
       tc_commit(smem_u32(&sm.bar_final));
       volatile int no_abort = 0;
@@ -335,12 +378,21 @@ __global__ void __launch_bounds__(kBwdKvThreads, 1) mfa_bwd_dkv_kernel(const __g
       const bool interior = __all_sync(0xffffffffu, ilo <= col0 && col0 + 63 <= ihi);
       const float* nlp = &sm.nl[st][half * 64];
       const float* ddp = &sm.dd[st][half * 64];
-#pragma unroll 1
-      for (int ch = 0; ch < 2; ++ch) {  // 32 query columns at a time, read then written in place
-        uint32_t sr[32], dr[32];
-        tmem_ld32(tmem + lane_base + half * 64 + ch * 32, sr);
+      // S^T of both chunks first: once every warp has it, S^T of the next step may be computed
+      // into these columns while the warps work on this one
+      uint32_t sr0[32], sr1[32];
+      tmem_ld32(tmem + lane_base + half * 64, sr0);
+      tmem_ld32(tmem + lane_base + half * 64 + 32, sr1);
+      tmem_wait_ld(sr0, sr1);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.bar_sfree));
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {  // 32 query columns at a time
+        uint32_t(&sr)[32] = ch ? sr1 : sr0;
+        uint32_t dr[32];
         tmem_ld32(tmem + lane_base + 128 + half * 64 + ch * 32, dr);
-        tmem_wait_ld(sr, dr);
+        tmem_wait_ld(dr);
         bool poly = false;
         if (SOFTCAP) {
           float am = 0.f;
@@ -394,10 +446,10 @@ __global__ void __launch_bounds__(kBwdKvThreads, 1) mfa_bwd_dkv_kernel(const __g
         };
         if (interior) chunk(std::true_type{});
         else chunk(std::false_type{});
-        // packed values of columns 64 half + 32 ch .. land on columns 64 half + 16 ch .., which
-        // this warp has already read
-        tmem_st16(tmem + lane_base + half * 64 + ch * 16, pk);
-        tmem_st16(tmem + lane_base + 128 + half * 64 + ch * 16, dk);
+        // P^T and dS^T of the chunk (16 packed columns each) go over the chunk's own 32 dP^T
+        // columns, which this warp has just read
+        tmem_st16(tmem + lane_base + 128 + half * 64 + ch * 32, pk);
+        tmem_st16(tmem + lane_base + 128 + half * 64 + ch * 32 + 16, dk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
