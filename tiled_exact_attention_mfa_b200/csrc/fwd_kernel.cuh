@@ -7,8 +7,9 @@
 // the end O / l and LSE = m + ln l. A tile whose every score of a row is masked leaves that
 // row untouched (the shader's m_new = -inf guard).
 //
-// B200 mapping (one CTA per SM, 384 threads, 2 Q tiles of 128 rows per CTA; setmaxnreg gives
-// the softmax warpgroups 200 registers per thread and the producer / MMA warpgroup 104):
+// B200 mapping, default shape (one CTA per SM, 384 threads, 2 Q tiles of 128 rows per CTA;
+// setmaxnreg gives the softmax warpgroups 200 registers per thread and the producer / MMA
+// warpgroup 104; the single-Q-tile shape used for sliding windows is described at FwdShape):
 //   warp 8      TMA producer: Q tiles once, then K and V tiles through 2-stage rings (128-byte
 //               swizzled smem, 3-D tensor maps so tails are zero-filled per head).
 //   warp 9      TMEM owner and single-thread tcgen05.mma issuer:
@@ -19,8 +20,9 @@
 //               domain (scale * log2 e folded into one FFMA). The running max is only moved when
 //               it grows by more than 2^8 (rescaling is exact for any reference max; a stale one
 //               only bounds P by 2^8), and then O is rescaled in TMEM by the owning warp.
-//   TMEM columns: S_0 [0,128) S_1 [128,256) O_0 [256,256+D) O_1 [256+D, 256+2D);
-//                 P_t (16-bit, 2 per column) overwrites the first 64 columns of S_t.
+//   TMEM columns: S_0 [0,128) S_1 [128,256) O_0 [256,256+D) O_1 [256+D, 256+2D) (one Q tile:
+//                 S [0,128), O [128,128+D)); P_t (16-bit, 2 per column) overwrites the first
+//                 64 columns of S_t.
 // Ordering: QK for tile j+1 of Q tile t overwrites S_t's columns, where PV for tile j reads P_t
 // from. tcgen05 only orders MMAs that share an accumulator, so the MMA thread waits for that PV
 // to complete before issuing the QK (issuing it right behind the PV would rely on an execution
@@ -40,9 +42,35 @@ namespace mfa {
 
 constexpr int kFwdBM = 128;       // query rows per Q tile (= TMEM lanes)
 constexpr int kFwdBN = 128;       // keys per K/V tile
-constexpr int kFwdQT = 2;         // Q tiles per CTA
-constexpr int kFwdStages = 2;     // K ring and V ring depth
-constexpr int kFwdThreads = 384;  // 8 softmax warps + producer + MMA + 2 idle
+// Two CTA shapes. The default holds two Q tiles (384 threads: 8 softmax warps, then a
+// warpgroup of producer + MMA + 2 idle warps; 512 TMEM columns; ~198 KB of shared memory at
+// D = 128; one CTA per SM), whose softmax phases interleave on one tensor core. ONE holds a
+// single Q tile (256 threads: 4 softmax warps, then the same control warpgroup; 256 TMEM
+// columns; at D = 128 one K and one V stage, ~98 KB; two CTAs per SM): the two resident CTAs
+// interleave the same way, and one CTA's start (Q load, first QK) and end (last PV, O store)
+// overlap the other's key tiles, which pays where a CTA has few key tiles (sliding windows).
+// setmaxnreg moves registers from the control warpgroup to the softmax warpgroups; each split
+// adds up to the registers the CTA launches with (threads x launch-bound registers).
+template <bool ONE>
+struct FwdShape {
+  static constexpr int kQT = ONE ? 1 : 2;                // Q tiles per CTA
+  static constexpr int kThreads = ONE ? 256 : 384;
+  static constexpr int kMinBlocks = ONE ? 2 : 1;          // CTAs per SM the launch bounds ask for
+  static constexpr int kProducerWarp = ONE ? 4 : 8;
+  static constexpr int kMmaWarp = ONE ? 5 : 9;
+  static constexpr int kTmemCols = ONE ? 256 : 512;       // S of each Q tile, then O of each
+  static constexpr int kRegsSoftmax = ONE ? 192 : 200;    // per thread after setmaxnreg
+  static constexpr int kRegsControl = ONE ? 64 : 104;
+  static constexpr int kRegsLaunch = ONE ? 128 : 168;     // 65,536 / (threads x CTAs per SM), rounded
+  static_assert(kQT * 128 * kRegsSoftmax + 128 * kRegsControl == kThreads * kRegsLaunch,
+                "the setmaxnreg split must use exactly the CTA's launch registers");
+};
+template <int D, bool ONE>
+__host__ __device__ constexpr int fwd_stages() {  // K ring and V ring depth
+  return (ONE && D == 128) ? 1 : 2;
+}
+constexpr int kFwdQT = 2;         // Q tiles per CTA of the default shape
+constexpr int kFwdThreads = 384;  // threads of the default shape
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kFwdMaxSparseTiles = 2048;  // key tiles a block-sparse row may span (262,144 keys)
 #ifndef MFA_POLY_MASK
@@ -83,19 +111,21 @@ struct FwdParams {
   float lse_mul;    // ln 2
 };
 
-template <int D, bool SPARSE>
+template <int D, bool SPARSE, bool ONE = false>
 struct FwdSmem {
   static constexpr int kTileBytes = kFwdBM * D * 2;  // one 128 x D tile of 16-bit values
   static constexpr int kSlabBytes = 128 * 128;       // 128 rows x 64 columns (128 B) slab
-  uint8_t q[kFwdQT][kTileBytes];
-  uint8_t k[kFwdStages][kTileBytes];
-  uint8_t v[kFwdStages][kTileBytes];
+  static constexpr int kQT = FwdShape<ONE>::kQT;
+  static constexpr int kNS = fwd_stages<D, ONE>();
+  uint8_t q[kQT][kTileBytes];
+  uint8_t k[kNS][kTileBytes];
+  uint8_t v[kNS][kTileBytes];
   uint64_t bar_q;
-  uint64_t bar_k_full[kFwdStages], bar_k_empty[kFwdStages];
-  uint64_t bar_v_full[kFwdStages], bar_v_empty[kFwdStages];
+  uint64_t bar_k_full[kNS], bar_k_empty[kNS];
+  uint64_t bar_v_full[kNS], bar_v_empty[kNS];
   // P of a Q tile becomes ready in two halves (keys 0-63, 64-127), so the first half of PV can
   // run while the second half of the exponentials is computed
-  uint64_t bar_s_full[kFwdQT], bar_p_full[kFwdQT][2], bar_o_done[kFwdQT];
+  uint64_t bar_s_full[kQT], bar_p_full[kQT][2], bar_o_done[kQT];
   uint64_t bar_final;
   uint32_t tmem_base;
   int abort;
@@ -104,9 +134,9 @@ struct FwdSmem {
   uint8_t act_bits[SPARSE ? kFwdMaxSparseTiles : 1];   // ... bit t: Q tile t's block is on
 };
 
-template <int D, bool SPARSE>
+template <int D, bool SPARSE, bool ONE = false>
 constexpr int fwd_smem_bytes() {
-  return (int)sizeof(FwdSmem<D, SPARSE>) + 1024;  // + alignment slack for the 1024-byte swizzle atoms
+  return (int)sizeof(FwdSmem<D, SPARSE, ONE>) + 1024;  // + alignment slack for the 1024-byte swizzle atoms
 }
 
 // Visible key range [lo, hi) of absolute query positions [a0, a1] (inclusive) among Nk keys.
@@ -136,14 +166,22 @@ __device__ __forceinline__ void key_range(const FwdParams& p, int Nk, int a0, in
 // every tile of the CTA's range; chosen for sliding windows, where the two Q tiles' ranges
 // differ by a tile at each end (elsewhere the saving is one diagonal tile per CTA, less than what
 // the extra bookkeeping costs the plain loop).
-template <int D, bool BF16, bool VARLEN, bool SPARSE, bool SOFTCAP, bool PAGED, bool PART = false>
-__global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_constant__ FwdParams p) {
+// ONE: the single-Q-tile CTA shape (FwdShape).
+template <int D, bool BF16, bool VARLEN, bool SPARSE, bool SOFTCAP, bool PAGED, bool PART = false, bool ONE = false>
+__global__ void __launch_bounds__(FwdShape<ONE>::kThreads, FwdShape<ONE>::kMinBlocks)
+    mfa_fwd_kernel(const __grid_constant__ FwdParams p) {
   constexpr bool kRuns = PART && !SPARSE;  // Q tile t takes part in the run [jlo_t, jhi_t)
   constexpr bool kPart = SPARSE || kRuns;  // a Q tile may sit out some visited tiles
+  constexpr int kFwdQT = FwdShape<ONE>::kQT;
+  constexpr int kFwdStages = fwd_stages<D, ONE>();
+  constexpr int kProd = FwdShape<ONE>::kProducerWarp;
+  constexpr int kMma = FwdShape<ONE>::kMmaWarp;
+  constexpr int kOCol = kFwdQT * kFwdBN;  // first TMEM column of O (after the S of each Q tile)
+  using Smem = FwdSmem<D, SPARSE, ONE>;
   static_assert(!(VARLEN && SPARSE), "block masks are defined on the dense layout");
   static_assert(!PAGED || VARLEN, "paged keys come with packed queries");
   extern __shared__ uint8_t smem_raw[];
-  FwdSmem<D, SPARSE>& sm = *reinterpret_cast<FwdSmem<D, SPARSE>*>(
+  Smem& sm = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
   const int warp = threadIdx.x >> 5;
@@ -216,8 +254,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     }
     vlo0 = vlo[0];
     vhi0 = vhi[0];
-    vlo1 = vlo[1];
-    vhi1 = vhi[1];
+    vlo1 = kFwdQT > 1 ? vlo[kFwdQT - 1] : 1;  // (one Q tile: a second that sees nothing)
+    vhi1 = kFwdQT > 1 ? vhi[kFwdQT - 1] : 0;
   }
   // bit t: Q tile t takes part in key tile kt (intersects its visible range)
   auto vis_bits = [&](int kt) -> uint32_t {
@@ -228,7 +266,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
   // ---- setup: the producer thread initialises the barriers and starts the Q load at once, so
   // the copy overlaps the TMEM allocation, the block-sparse tile list and the CTA barrier
   const bool q_early = n_tiles > 0;
-  if (warp == 8 && lane == 0) {
+  if (warp == kProd && lane == 0) {
     mbar_init(smem_u32(&sm.bar_q), 1);
     for (int s = 0; s < kFwdStages; ++s) {
       mbar_init(smem_u32(&sm.bar_k_full[s]), 1);
@@ -248,14 +286,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     if (q_early) {
       tma_prefetch_desc(&p.tm_q);
       const uint32_t bq = smem_u32(&sm.bar_q);
-      mbar_expect_tx(bq, kFwdQT * (uint32_t)FwdSmem<D, SPARSE>::kTileBytes);
+      mbar_expect_tx(bq, kFwdQT * (uint32_t)Smem::kTileBytes);
       for (int t = 0; t < kFwdQT; ++t)
         for (int sl = 0; sl < D / 64; ++sl)
           if constexpr (VARLEN)
-            tma_load_3d(smem_u32(sm.q[t]) + sl * FwdSmem<D, SPARSE>::kSlabBytes, &p.tm_q, bq, sl * 64,
+            tma_load_3d(smem_u32(sm.q[t]) + sl * Smem::kSlabBytes, &p.tm_q, bq, sl * 64,
                         h, rq + q0 + t * kFwdBM);
           else
-            tma_load_3d(smem_u32(sm.q[t]) + sl * FwdSmem<D, SPARSE>::kSlabBytes, &p.tm_q, bq, sl * 64,
+            tma_load_3d(smem_u32(sm.q[t]) + sl * Smem::kSlabBytes, &p.tm_q, bq, sl * 64,
                         q0 + t * kFwdBM, b * p.Hq + h);
     }
   }
@@ -264,7 +302,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     // 32 lanes read 8 tiles each per step (all loads issued before the ballots).
     const int qt0 = q0 / kFwdBM;
     const uint8_t* r0 = p.block_mask + ((size_t)(b * p.Hq + h) * p.nqt + qt0) * p.nkt + kt_lo;
-    const uint8_t* r1 = (qt0 + 1 < p.nqt) ? r0 + p.nkt : nullptr;
+    const uint8_t* r1 = (kFwdQT > 1 && qt0 + 1 < p.nqt) ? r0 + p.nkt : nullptr;
     int count = 0;
     for (int base = 0; base < n_tiles; base += 32 * 8) {
       uint8_t a0[8], a1[8];
@@ -294,11 +332,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       sm.n_act = min(count, kFwdMaxSparseTiles);
     }
   }
-  if (warp == 9) {
-    tmem_alloc(smem_u32(&sm.tmem_base), 512);
+  if (warp == kMma) {
+    tmem_alloc(smem_u32(&sm.tmem_base), FwdShape<ONE>::kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == kProd && lane == 0) {
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_v);
   }
@@ -320,23 +358,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
   auto bits_of = [&](int u) -> uint32_t {  // bit t: Q tile t takes part in visited tile u
     if constexpr (SPARSE) return sm.act_bits[u];
     else if constexpr (kRuns) return ((u >= jlo0 && u < jhi0) ? 1u : 0u) | ((u >= jlo1 && u < jhi1) ? 2u : 0u);
-    else return 3u;
+    else return kFwdQT > 1 ? 3u : 1u;
   };
   if (threadIdx.x == 0 && (p.flags & 2) && n_act > 0)
     atomicAdd(p.tile_counter, (unsigned long long)n_act);
   volatile int* abort = &sm.abort;
 
   constexpr int kSlabs = D / 64;
-  constexpr uint32_t kTileBytes = FwdSmem<D, SPARSE>::kTileBytes;
-  constexpr int kSlab = FwdSmem<D, SPARSE>::kSlabBytes;
+  constexpr uint32_t kTileBytes = Smem::kTileBytes;
+  constexpr int kSlab = Smem::kSlabBytes;
 
-  if (warp >= 8) {
-   regs_control();
-   if (warp == 8) {
+  if (warp >= kProd) {
+   regs_dec<FwdShape<ONE>::kRegsControl>();
+   if (warp == kProd) {
     // ================================================================ TMA producer
     const uint32_t bq = smem_u32(&sm.bar_q);
     if (lane == 0 && n_act > 0) {  // (the Q tiles were requested during setup)
-      int issued_k[kFwdStages] = {0, 0}, issued_v[kFwdStages] = {0, 0};
+      int issued_k[kFwdStages] = {}, issued_v[kFwdStages] = {};
       for (int u = 0; u < n_act; ++u) {
         const int s = u % kFwdStages;
         const int use = u / kFwdStages;
@@ -396,20 +434,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       volatile int no_abort = 0;
       mbar_wait(bq, 0, &no_abort, 803);
     }
-  } else if (warp == 9) {
+  } else if (warp == kMma) {
     // ================================================================ MMA issuer
     if (lane == 0 && n_act > 0) {
       const uint32_t idesc_qk = idesc_f16(BF16 ? 1 : 0, kFwdBM, kFwdBN, 0);
       const uint32_t idesc_pv = idesc_f16(BF16 ? 1 : 0, kFwdBM, D, 1);
       // descriptors of the tiles' first bytes, built once (selected, not indexed, so they stay in
       // registers); each MMA adds a constant offset
-      static_assert(kFwdQT == 2 && kFwdStages == 2, "descriptor selection assumes two of each");
+      static_assert(kFwdQT <= 2 && kFwdStages <= 2, "descriptor selection assumes at most two of each");
       const SmemDesc dq0 = smem_desc_sw128_split(smem_u32(sm.q[0]), 16, 1024);
-      const SmemDesc dq1 = smem_desc_sw128_split(smem_u32(sm.q[1]), 16, 1024);
+      const SmemDesc dq1 = smem_desc_sw128_split(smem_u32(sm.q[kFwdQT - 1]), 16, 1024);
       const SmemDesc dk0 = smem_desc_sw128_split(smem_u32(sm.k[0]), 16, 1024);
-      const SmemDesc dk1 = smem_desc_sw128_split(smem_u32(sm.k[1]), 16, 1024);
+      const SmemDesc dk1 = smem_desc_sw128_split(smem_u32(sm.k[kFwdStages - 1]), 16, 1024);
       const SmemDesc dv0 = smem_desc_sw128_split(smem_u32(sm.v[0]), kSlab, 1024);
-      const SmemDesc dv1 = smem_desc_sw128_split(smem_u32(sm.v[1]), kSlab, 1024);
+      const SmemDesc dv1 = smem_desc_sw128_split(smem_u32(sm.v[kFwdStages - 1]), kSlab, 1024);
       auto issue_qk = [&](int t, int s) {
         const SmemDesc a = t ? dq1 : dq0, bk = s ? dk1 : dk0;
 #pragma unroll
@@ -428,9 +466,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
         for (int kk = h * 4; kk < h * 4 + 4; ++kk) {
           const uint32_t off = (kk * 16 * 128) >> 4;
           if (kk == 0 && !acc)
-            tc_mma_ts_c<0>(tmem + 256 + t * D, tmem + t * kFwdBN + kk * 8, bv.lo + off, bv.hi, idesc_pv);
+            tc_mma_ts_c<0>(tmem + kOCol + t * D, tmem + t * kFwdBN + kk * 8, bv.lo + off, bv.hi, idesc_pv);
           else
-            tc_mma_ts_c<1>(tmem + 256 + t * D, tmem + t * kFwdBN + kk * 8, bv.lo + off, bv.hi, idesc_pv);
+            tc_mma_ts_c<1>(tmem + kOCol + t * D, tmem + t * kFwdBN + kk * 8, bv.lo + off, bv.hi, idesc_pv);
         }
       };
       // Debug flag bit 2 (failure-detection tests): issue no MMA at all, so the softmax warps'
@@ -445,11 +483,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
       uint32_t bits_cur = SPARSE ? sm.act_bits[0] : 0u, bits_next = 0u;
       int j = 0;
       auto act_cur = [&](int t) -> bool {  // Q tile t takes part in tile j
+        if (t >= kFwdQT) return false;
         if constexpr (!kPart) return true;
         else if constexpr (SPARSE) return ((bits_cur >> t) & 1u) != 0;
         else return t ? (j >= jlo1 && j < jhi1) : (j >= jlo0 && j < jhi0);
       };
       auto act_next = [&](int t) -> bool {  // ... in tile j + 1
+        if (t >= kFwdQT) return false;
         if constexpr (!kPart) return true;
         else if constexpr (SPARSE) return ((bits_next >> t) & 1u) != 0;
         else return t ? (j + 1 >= jlo1 && j + 1 < jhi1) : (j + 1 >= jlo0 && j + 1 < jhi0);
@@ -548,7 +588,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     }
    }
   } else {
-    regs_softmax();
+    regs_inc<FwdShape<ONE>::kRegsSoftmax>();
     // ================================================================ softmax warps
     const int t = warp >> 2;                  // Q tile of this warpgroup
     const int quarter = warp & 3;             // TMEM lane quarter of this warp
@@ -559,7 +599,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
     const int a_hi = a_lo + kFwdBM - 1;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t t_s = tmem + lane_base + t * kFwdBN;
-    const uint32_t t_o = tmem + lane_base + 256 + t * D;
+    const uint32_t t_o = tmem + lane_base + kOCol + t * D;
     const float c = p.c_log2;
     float m_run = -INFINITY;  // running max of the stored (scaled, capped) score
     float l_run = 0.f;
@@ -830,10 +870,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) mfa_fwd_kernel(const __grid_co
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMma) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, FwdShape<ONE>::kTmemCols);
   }
 }
 

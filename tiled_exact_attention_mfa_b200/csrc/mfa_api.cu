@@ -254,14 +254,17 @@ struct FwdCall {
   int max_pages, num_pages;
 };
 
-template <int D, bool BF16, bool VARLEN, bool SPARSE, bool SOFTCAP, bool PAGED, bool PART>
+// ONE: the single-Q-tile CTA shape (two CTAs per SM); see mfa::FwdShape.
+template <int D, bool BF16, bool VARLEN, bool SPARSE, bool SOFTCAP, bool PAGED, bool PART, bool ONE = false>
 int launch_fwd(const FwdCall& c, cudaStream_t st) {
   const int B = c.B, Hq = c.Hq, Hkv = c.Hkv, Nq = c.Nq, Nk = c.Nk, dtype = c.dtype;
   const float scale = c.scale, softcap = c.softcap;
+  using Shape = mfa::FwdShape<ONE>;
   static bool smem_done[kMaxDevices] = {};
   static bool regs_ok[kMaxDevices] = {};
-  constexpr int smem = mfa::fwd_smem_bytes<D, SPARSE>();
-  auto kernel = mfa::mfa_fwd_kernel<D, BF16, VARLEN, SPARSE, SOFTCAP, PAGED, PART>;
+  constexpr int smem = mfa::fwd_smem_bytes<D, SPARSE, ONE>();
+  static_assert(!ONE || 2 * (smem + 1024) <= 233472, "two single-Q-tile CTAs must fit one SM");
+  auto kernel = mfa::mfa_fwd_kernel<D, BF16, VARLEN, SPARSE, SOFTCAP, PAGED, PART, ONE>;
   if (!ensure_smem(kernel, smem, smem_done)) return MFA_ERR_CUDA;
   {
     // setmaxnreg redistributes the registers the CTA launched with; refuse to launch if the
@@ -271,7 +274,8 @@ int launch_fwd(const FwdCall& c, cudaStream_t st) {
     if (!regs_ok[dev]) {
       cudaFuncAttributes fa;
       if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return MFA_ERR_CUDA;
-      if (fa.numRegs * mfa::kFwdThreads < 256 * mfa::kRegsSoftmax + 128 * mfa::kRegsControl)
+      if (fa.numRegs * Shape::kThreads <
+          Shape::kQT * 128 * Shape::kRegsSoftmax + 128 * Shape::kRegsControl)
         return MFA_ERR_CUDA;
       regs_ok[dev] = true;
     }
@@ -320,7 +324,7 @@ int launch_fwd(const FwdCall& c, cudaStream_t st) {
   p.causal = c.causal ? 1 : 0;
   p.win_l = c.win_l;
   p.win_r = c.win_r;
-  const int rows_per_cta = mfa::kFwdBM * mfa::kFwdQT;
+  const int rows_per_cta = mfa::kFwdBM * Shape::kQT;
   p.n_qblk = (Nq + rows_per_cta - 1) / rows_per_cta;
   p.flags = g_debug_flags;
   if (p.flags & MFA_DEBUG_COUNT_TILES) {
@@ -344,17 +348,17 @@ int launch_fwd(const FwdCall& c, cudaStream_t st) {
   p.lse_mul = 0.69314718055994531f;
   const long long grid = (long long)p.n_qblk * B * Hq;
   if (grid > 0x7FFFFFFFLL) return MFA_ERR_BAD_SHAPE;
-  kernel<<<(unsigned)grid, mfa::kFwdThreads, smem, st>>>(p);
+  kernel<<<(unsigned)grid, Shape::kThreads, smem, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return MFA_ERR_CUDA;
   mfa_launch_info li = {};
   li.kernel = 1;
   li.grid_x = (int)grid;
   li.grid_y = li.grid_z = 1;
-  li.block_threads = mfa::kFwdThreads;
+  li.block_threads = Shape::kThreads;
   li.smem_bytes = smem;
   li.tile_m = mfa::kFwdBM;
   li.tile_n = mfa::kFwdBN;
-  li.q_tiles_per_cta = mfa::kFwdQT;
+  li.q_tiles_per_cta = Shape::kQT;
   g_last = li;
   return MFA_OK;
 }
@@ -465,21 +469,22 @@ int launch_fill_empty(void* out, float* lse, size_t rows, int D, int dtype, cuda
   return MFA_OK;
 }
 
-template <bool VARLEN, bool SPARSE, bool SOFTCAP, bool PAGED, bool PART>
+template <bool VARLEN, bool SPARSE, bool SOFTCAP, bool PAGED, bool PART, bool ONE>
 int dispatch_fwd_d(const FwdCall& c, int D, cudaStream_t st) {
   const bool bf = c.dtype == MFA_DTYPE_BF16;
   if (D == 128)
-    return bf ? launch_fwd<128, true, VARLEN, SPARSE, SOFTCAP, PAGED, PART>(c, st)
-              : launch_fwd<128, false, VARLEN, SPARSE, SOFTCAP, PAGED, PART>(c, st);
-  return bf ? launch_fwd<64, true, VARLEN, SPARSE, SOFTCAP, PAGED, PART>(c, st)
-            : launch_fwd<64, false, VARLEN, SPARSE, SOFTCAP, PAGED, PART>(c, st);
+    return bf ? launch_fwd<128, true, VARLEN, SPARSE, SOFTCAP, PAGED, PART, ONE>(c, st)
+              : launch_fwd<128, false, VARLEN, SPARSE, SOFTCAP, PAGED, PART, ONE>(c, st);
+  return bf ? launch_fwd<64, true, VARLEN, SPARSE, SOFTCAP, PAGED, PART, ONE>(c, st)
+            : launch_fwd<64, false, VARLEN, SPARSE, SOFTCAP, PAGED, PART, ONE>(c, st);
 }
 
-// PART: each Q tile of a CTA computes only the key tiles its own rows see (dense sliding windows)
-template <bool VARLEN, bool SPARSE, bool PAGED = false, bool PART = false>
+// PART: each Q tile of a CTA computes only the key tiles its own rows see; ONE: one Q tile per
+// CTA, two CTAs per SM (dense sliding windows)
+template <bool VARLEN, bool SPARSE, bool PAGED = false, bool PART = false, bool ONE = false>
 int dispatch_fwd(const FwdCall& c, int D, cudaStream_t st) {
-  return c.softcap > 0.f ? dispatch_fwd_d<VARLEN, SPARSE, true, PAGED, PART>(c, D, st)
-                         : dispatch_fwd_d<VARLEN, SPARSE, false, PAGED, PART>(c, D, st);
+  return c.softcap > 0.f ? dispatch_fwd_d<VARLEN, SPARSE, true, PAGED, PART, ONE>(c, D, st)
+                         : dispatch_fwd_d<VARLEN, SPARSE, false, PAGED, PART, ONE>(c, D, st);
 }
 
 template <int D, bool BF16, bool SOFTCAP>
@@ -559,7 +564,12 @@ int mfa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, 
   clamp_window(win_l, win_r, Nk, Nq);
   FwdCall c = {q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, scale, causal, win_l, win_r, softcap, dtype,
                nullptr, nullptr, 0, 0, nullptr, nullptr, nullptr, 0, 0};
-  if (win_l >= 0 || win_r >= 0) return dispatch_fwd<false, false, false, true>(c, D, st);
+  // Sliding windows: the single-Q-tile shape (two CTAs per SM hide each other's start and end;
+  // with a cap its softmax needs more registers than that shape's split gives, so capped windows
+  // keep two Q tiles, each computing only its own run of key tiles).
+  if (win_l >= 0 || win_r >= 0)
+    return c.softcap > 0.f ? dispatch_fwd_d<false, false, true, false, true, false>(c, D, st)
+                           : dispatch_fwd_d<false, false, false, false, false, true>(c, D, st);
   return dispatch_fwd<false, false>(c, D, st);
 }
 
