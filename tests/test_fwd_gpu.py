@@ -36,6 +36,10 @@ SMALL = [
       2 ** 31 - 1, seed=25),
     P("window_int_max_noncausal_bf16", 1, 2, 1, 200, 333, 128, mi.BF16, False, 2 ** 31 - 1,
       2 ** 31 - 1, seed=26),
+    # windowed launches run one Q tile per CTA (two CTAs per SM): bottom-right alignment with
+    # Nq < Nk under GQA, and Nq > Nk with rows that see no key
+    P("window_nq_lt_nk_gqa2_d64_bf16", 2, 4, 2, 300, 900, 64, mi.BF16, True, 200, 0, seed=27),
+    P("window_nq_gt_nk_empty_rows_fp16", 1, 2, 2, 500, 260, 128, mi.FP16, True, 150, 0, seed=28),
 ]
 
 
