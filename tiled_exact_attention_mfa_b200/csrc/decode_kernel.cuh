@@ -152,8 +152,11 @@ __global__ void __launch_bounds__((kDecMaxHeads<D> + 1) * 32) mfa_decode_phase1_
       __syncwarp();
       if (pid_ok && lane < valid) {
         const size_t src = (((size_t)pid * kDecPage + lane) * p.Hkv + h0) * D;
-        bulk_load(kdst + lane * row_bytes, p.k_pages + src, chunk, bar);
-        bulk_load(vdst + lane * row_bytes, p.v_pages + src, chunk, bar);
+        // K / V are read once: evict them first, so the partials written below stay in L2
+        // for the combine
+        const uint64_t pol = l2_policy_evict_first();
+        bulk_load_hint(kdst + lane * row_bytes, p.k_pages + src, chunk, bar, pol);
+        bulk_load_hint(vdst + lane * row_bytes, p.v_pages + src, chunk, bar, pol);
       }
       issued[s] = use + 1;
     }
@@ -318,13 +321,13 @@ __global__ void __launch_bounds__((kDecMaxHeads<D> + 1) * 32) mfa_decode_phase1_
     if (r >= R) continue;
     const size_t row = (size_t)kvh * p.G * p.Nq + r;  // = (kvh*G + hl) * Nq + t
     float* dst = p.ws_o + (slot + row) * D;
+    // the combine reads these back soon: keep them in L2 ahead of the streamed K / V lines
+    const uint64_t pol = l2_policy_evict_last();
 #pragma unroll
-    for (int n = 0; n < D / 8; ++n)
-      *reinterpret_cast<float2*>(dst + n * 8 + qc) = make_float2(o[n][2 * e], o[n][2 * e + 1]);
-    if ((lane & 3) == 0) {
-      float2 ml = make_float2(m_run[e] == -INFINITY ? -INFINITY : m_run[e] * c, l_run[e]);
-      *reinterpret_cast<float2*>(p.ws_ml + (slot + row) * 2) = ml;
-    }
+    for (int n = 0; n < D / 8; ++n) st_global_f2_hint(dst + n * 8 + qc, o[n][2 * e], o[n][2 * e + 1], pol);
+    if ((lane & 3) == 0)
+      st_global_f2_hint(p.ws_ml + (slot + row) * 2, m_run[e] == -INFINITY ? -INFINITY : m_run[e] * c,
+                        l_run[e], pol);
   }
 }
 
