@@ -19,7 +19,9 @@ pytestmark = pytest.mark.gpu
 MFA_ERR_DEVICE_TIMEOUT = -21
 
 
-def test_wait_runs_out_reports_timeout_and_context_survives(cuda_device):
+# (-1, -1): the two-Q-tile CTA shape; (64, 0): a sliding window, which runs one Q tile per CTA
+@pytest.mark.parametrize("window", [(-1, -1), (64, 0)])
+def test_wait_runs_out_reports_timeout_and_context_survives(cuda_device, window):
     import torch
     import tiled_exact_attention_mfa_b200 as mfa
     case = mi.PrefillCase("one_cta", 1, 1, 1, 128, 128, 64, mi.FP16, True, seed=101)
@@ -29,7 +31,7 @@ def test_wait_runs_out_reports_timeout_and_context_survives(cuda_device):
     old = mfa.mfa_debug_set_flags(mfa.MFA_DEBUG_WITHHOLD_MMA)
     try:
         t0 = time.time()
-        out, lse = mfa.mfa_fwd(qt, kt, vt, scale=case.scale_f32(), causal=True)
+        out, lse = mfa.mfa_fwd(qt, kt, vt, scale=case.scale_f32(), causal=True, window=window)
         torch.cuda.synchronize()
         dt = time.time() - t0
     finally:
@@ -40,9 +42,9 @@ def test_wait_runs_out_reports_timeout_and_context_survives(cuda_device):
     assert 1.5 < dt < 60.0, dt
     assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
     # the context is intact: the same call without the flag matches the oracle
-    out, lse = mfa.mfa_fwd(qt, kt, vt, scale=case.scale_f32(), causal=True)
+    out, lse = mfa.mfa_fwd(qt, kt, vt, scale=case.scale_f32(), causal=True, window=window)
     torch.cuda.synchronize()
     w = lambda x: mi.widen(x, case.dtype)
-    o_ref, l_ref = oracle.attention(w(q), w(k), w(v), case.scale_f32(), True)
+    o_ref, l_ref = oracle.attention(w(q), w(k), w(v), case.scale_f32(), True, *window)
     check_close(from_torch(out), from_torch(lse), o_ref, l_ref, case.dtype, "after timeout")
     assert mfa.mfa_device_status() == (0, 0)
