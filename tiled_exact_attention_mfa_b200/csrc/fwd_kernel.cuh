@@ -69,8 +69,6 @@ template <int D, bool ONE>
 __host__ __device__ constexpr int fwd_stages() {  // K ring and V ring depth
   return (ONE && D == 128) ? 1 : 2;
 }
-constexpr int kFwdQT = 2;         // Q tiles per CTA of the default shape
-constexpr int kFwdThreads = 384;  // threads of the default shape
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kFwdMaxSparseTiles = 2048;  // key tiles a block-sparse row may span (262,144 keys)
 #ifndef MFA_POLY_MASK
@@ -172,7 +170,7 @@ __global__ void __launch_bounds__(FwdShape<ONE>::kThreads, FwdShape<ONE>::kMinBl
     mfa_fwd_kernel(const __grid_constant__ FwdParams p) {
   constexpr bool kRuns = PART && !SPARSE;  // Q tile t takes part in the run [jlo_t, jhi_t)
   constexpr bool kPart = SPARSE || kRuns;  // a Q tile may sit out some visited tiles
-  constexpr int kFwdQT = FwdShape<ONE>::kQT;
+  constexpr int kFwdQT = FwdShape<ONE>::kQT;  // Q tiles of this CTA shape
   constexpr int kFwdStages = fwd_stages<D, ONE>();
   constexpr int kProd = FwdShape<ONE>::kProducerWarp;
   constexpr int kMma = FwdShape<ONE>::kMmaWarp;
