@@ -60,3 +60,25 @@ def test_step_time_spread_is_median_and_deciles():
     assert r == {"ms_median": 5.5, "ms_p10": 1.9, "ms_p90": 9.1}
     assert bench.spread([2.0]) == {"ms_median": 2.0, "ms_p10": 2.0, "ms_p90": 2.0}
     assert bench.spread([]) == {}
+
+
+def test_every_gpu_line_is_timed_at_one_gpu():
+    """The workload loops of the GPU arm (prefill, decode, backward) run at any world size: only
+    the splits-over-GPUs decode line may depend on there being more than one GPU."""
+    import ast
+    src = open(os.path.join(ROOT, "bench.py")).read()
+    tree = ast.parse(src)
+    parents = {}
+    for node in ast.walk(tree):
+        for child in ast.iter_child_nodes(node):
+            parents[child] = node
+    loops = [n for n in ast.walk(tree) if isinstance(n, ast.For) and isinstance(n.iter, ast.Name)
+             and n.iter.id == "BACKWARD_WORKLOADS"]
+    assert loops, "the backward workloads are timed in a loop over BACKWARD_WORKLOADS"
+    for loop in loops:
+        node = loop
+        while node in parents:
+            node = parents[node]
+            if isinstance(node, ast.If):
+                names = {n.id for n in ast.walk(node.test) if isinstance(n, ast.Name)}
+                assert "world" not in names, "the backward lines must not need more than one GPU"
