@@ -662,35 +662,39 @@ __global__ void __launch_bounds__(FwdShape<ONE>::kThreads, FwdShape<ONE>::kMinBl
         for (int i = 0; i < 128; ++i) s[i] = (i < jhi && i >= jlo) ? s[i] : -INFINITY;
       }
       // row max: 8 chains of 3-input max
-      float m8[8];
+      auto row_max = [&]() -> float {
+        float m8[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m8[i] = fmaxf(s[i], s[i + 8]);
+        for (int i = 0; i < 8; ++i) m8[i] = fmaxf(s[i], s[i + 8]);
 #pragma unroll
-      for (int i = 16; i < 128; i += 16)
+        for (int i = 16; i < 128; i += 16)
 #pragma unroll
-        for (int k = 0; k < 8; ++k) m8[k] = max3(m8[k], s[i + k], s[i + 8 + k]);
-      float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-      if (poly && mx > -INFINITY) {
-        const float y = mx * p.cap_in;
-        mx = p.cap_out * (y * tanh_q(y * y));
-      }
-
-      // Lazy rescale: move the reference max only when it grew by more than 2^8 in exp2 terms.
-      const float m_new = fmaxf(m_run, mx);
-      const bool need = (m_new > -INFINITY) && (m_run == -INFINITY || (m_new - m_run) * c > kRescaleLog2);
-      float alpha = 1.f;
-      const bool warp_rescale = __any_sync(0xffffffffu, need);
-      if (warp_rescale) {
-        if (m_new > m_run) {
-          alpha = (m_run == -INFINITY) ? 0.f : fast_exp2((m_run - m_new) * c);
-          m_run = m_new;
+          for (int k = 0; k < 8; ++k) m8[k] = max3(m8[k], s[i + k], s[i + 8 + k]);
+        float mx = max3(max3(m8[0], m8[1], m8[2]), max3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+        if (poly && mx > -INFINITY) {
+          const float y = mx * p.cap_in;
+          mx = p.cap_out * (y * tanh_q(y * y));
         }
-      }
-      const float neg_mc = (m_run == -INFINITY) ? 0.f : -m_run * c;
-
+        return mx;
+      };
+      // Lazy rescale: move the reference max only when it grew by more than 2^8 in exp2 terms.
+      // Returns whether any row of the warp moves it (then alpha and m_run are updated).
+      float alpha = 1.f;
+      auto rescale_decision = [&](float mx) -> bool {
+        const float m_new = fmaxf(m_run, mx);
+        const bool need = (m_new > -INFINITY) && (m_run == -INFINITY || (m_new - m_run) * c > kRescaleLog2);
+        const bool warp_rescale = __any_sync(0xffffffffu, need);
+        if (warp_rescale) {
+          if (m_new > m_run) {
+            alpha = (m_run == -INFINITY) ? 0.f : fast_exp2((m_run - m_new) * c);
+            m_run = m_new;
+          }
+        }
+        return warp_rescale;
+      };
       // O rescale before any PV of this tile reads P (only after the first tile: before it O
       // holds nothing). The previous PV of this Q tile has completed: its commit preceded S.
-      if (warp_rescale && c_t > 0) {
+      auto rescale_o = [&]() {
 #pragma unroll
         for (int cb = 0; cb < D; cb += 32) {
           uint32_t o[32];
@@ -706,9 +710,7 @@ __global__ void __launch_bounds__(FwdShape<ONE>::kThreads, FwdShape<ONE>::kMinBl
           }
           tmem_st32(t_o + cb, o);
         }
-      }
-      // P = exp2(s * c - m * c) on fp32 pairs, packed to the input type and stored to TMEM 16
-      // columns at a time; each half of P is announced as soon as it is stored.
+      };
       if constexpr (PAGED) {
         // the final tile: value rows at or past the length (inside the last page) become 0, by
         // the first Q tile taking part in it (each PV of the tile comes after that one's P)
@@ -728,21 +730,32 @@ __global__ void __launch_bounds__(FwdShape<ONE>::kThreads, FwdShape<ONE>::kMinBl
           fence_proxy_async_smem();  // generic stores, then the tensor core reads them after P
         }
       }
+      // P = exp2(s * c - m * c) on fp32 pairs, packed to the input type and stored to TMEM 16
+      // columns at a time (32 keys per chunk); a half of P (chunks 0-1, 2-3) is announced once it
+      // is stored, when announcements are on.
       const uint64_t c2 = f2_pack(c, c);
-      const uint64_t nm2 = f2_pack(neg_mc, neg_mc);
       uint64_t acc[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[i] = f2_pack(0.f, 0.f);
+      auto announce = [&](int half) {
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.bar_p_full[t][half]));
+      };
       // POLY: the kept value of a pair is tanh(y) * cap / scale with y = s * scale / cap, so
       // x = tanh(y) * (cap log2 e) - m c; a masked score (-inf) gives y = -inf, q = +inf and
       // x = -inf (the polynomial's leading coefficient is positive).
-      auto exponentials = [&](auto poly_tag) {
+      auto exponentials = [&](auto poly_tag, auto ch_lo_tag, auto ch_hi_tag, bool announce_halves,
+                              float neg_mc) {
         constexpr bool kPoly = decltype(poly_tag)::value;
+        constexpr int kChLo = decltype(ch_lo_tag)::value, kChHi = decltype(ch_hi_tag)::value;
         const uint64_t ci2 = f2_pack(p.cap_in, p.cap_in);
         const float cc = p.softcap * 1.4426950408889634f;
         const uint64_t xc2 = kPoly ? f2_pack(cc, cc) : c2;
+        const uint64_t nm2 = f2_pack(neg_mc, neg_mc);
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int ch = kChLo; ch < kChHi; ++ch) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -767,18 +780,43 @@ __global__ void __launch_bounds__(FwdShape<ONE>::kThreads, FwdShape<ONE>::kMinBl
             pk[i] = pack2<BF16>(p0, p1);
           }
           tmem_st16(t_s + ch * 16, pk);
-          if (ch & 1) {
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sm.bar_p_full[t][ch >> 1]));
-          }
+          if ((ch & 1) && announce_halves) announce(ch >> 1);
         }
       };
-      if (SOFTCAP && poly)
-        exponentials(std::integral_constant<bool, true>());
-      else
-        exponentials(std::integral_constant<bool, false>());
+      using I0 = std::integral_constant<int, 0>;
+      using I2 = std::integral_constant<int, 2>;
+      using I4 = std::integral_constant<int, 4>;
+      using PolyOff = std::integral_constant<bool, false>;
+      using PolyOn = std::integral_constant<bool, true>;
+      const float neg_mc_old = (m_run == -INFINITY) ? 0.f : -m_run * c;
+      if (ONE && !SOFTCAP && c_t > 0) {
+        // After the first tile the reference max rarely moves: compute the first half of P
+        // with the current one while the row max of the whole tile is taken alongside, and
+        // announce it unless some row of the warp moves the max, in which case the tile is
+        // redone exactly as the ordinary path below does it (nothing of it was announced).
+        // Bitwise the same results as the ordinary path. (Measured on the single-Q-tile shape:
+        // windows 3-6 % faster; on the two-Q-tile shape it changed nothing beyond noise.)
+        exponentials(PolyOff(), I0(), I2(), false, neg_mc_old);
+        const float mx = row_max();
+        if (!rescale_decision(mx)) {
+          announce(0);
+          exponentials(PolyOff(), I2(), I4(), true, neg_mc_old);
+        } else {
+          rescale_o();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[i] = f2_pack(0.f, 0.f);
+          exponentials(PolyOff(), I0(), I4(), true, (m_run == -INFINITY) ? 0.f : -m_run * c);
+        }
+      } else {
+        const float mx = row_max();
+        const bool warp_rescale = rescale_decision(mx);
+        if (warp_rescale && c_t > 0) rescale_o();
+        const float neg_mc = (m_run == -INFINITY) ? 0.f : -m_run * c;
+        if (SOFTCAP && poly)
+          exponentials(PolyOn(), I0(), I4(), true, neg_mc);
+        else
+          exponentials(PolyOff(), I0(), I4(), true, neg_mc);
+      }
       float sa, sb;
       f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), sa, sb);
       l_run = l_run * alpha + (sa + sb);
