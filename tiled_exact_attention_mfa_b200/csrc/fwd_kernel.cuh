@@ -48,7 +48,8 @@ constexpr int kFwdBN = 128;       // keys per K/V tile
 // single Q tile (256 threads: 4 softmax warps, then the same control warpgroup; 256 TMEM
 // columns; at D = 128 one K and one V stage, ~98 KB; two CTAs per SM): the two resident CTAs
 // interleave the same way, and one CTA's start (Q load, first QK) and end (last PV, O store)
-// overlap the other's key tiles, which pays where a CTA has few key tiles (sliding windows).
+// overlap the other's key tiles. With the speculative reference max below, ONE is the faster
+// shape for uncapped dense calls; capped, packed, block-sparse and paged calls use the default.
 // setmaxnreg moves registers from the control warpgroup to the softmax warpgroups; each split
 // adds up to the registers the CTA launches with (threads x launch-bound registers).
 template <bool ONE>
@@ -795,7 +796,8 @@ __global__ void __launch_bounds__(FwdShape<ONE>::kThreads, FwdShape<ONE>::kMinBl
         // announce it unless some row of the warp moves the max, in which case the tile is
         // redone exactly as the ordinary path below does it (nothing of it was announced).
         // Bitwise the same results as the ordinary path. (Measured on the single-Q-tile shape:
-        // windows 3-6 % faster; on the two-Q-tile shape it changed nothing beyond noise.)
+        // causal N = 4096 6 %, windows 3-6 % faster; on the two-Q-tile shape it changed nothing
+        // beyond noise.)
         exponentials(PolyOff(), I0(), I2(), false, neg_mc_old);
         const float mx = row_max();
         if (!rescale_decision(mx)) {

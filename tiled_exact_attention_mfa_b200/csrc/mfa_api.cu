@@ -564,13 +564,13 @@ int mfa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, 
   clamp_window(win_l, win_r, Nk, Nq);
   FwdCall c = {q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, scale, causal, win_l, win_r, softcap, dtype,
                nullptr, nullptr, 0, 0, nullptr, nullptr, nullptr, 0, 0};
-  // Sliding windows: the single-Q-tile shape (two CTAs per SM hide each other's start and end;
-  // with a cap its softmax needs more registers than that shape's split gives, so capped windows
-  // keep two Q tiles, each computing only its own run of key tiles).
-  if (win_l >= 0 || win_r >= 0)
-    return c.softcap > 0.f ? dispatch_fwd_d<false, false, true, false, true, false>(c, D, st)
-                           : dispatch_fwd_d<false, false, false, false, false, true>(c, D, st);
-  return dispatch_fwd<false, false>(c, D, st);
+  // Uncapped: the single-Q-tile shape (two CTAs per SM, which hide each other's start and end;
+  // measured faster on causal, non-causal and windowed workloads). With a cap its softmax needs
+  // more registers than that shape's split gives, so capped calls keep two Q tiles per CTA (under
+  // a window each computing only its own run of key tiles).
+  if (c.softcap <= 0.f) return dispatch_fwd_d<false, false, false, false, false, true>(c, D, st);
+  if (win_l >= 0 || win_r >= 0) return dispatch_fwd_d<false, false, true, false, true, false>(c, D, st);
+  return dispatch_fwd_d<false, false, true, false, false, false>(c, D, st);
 }
 
 int mfa_fwd_blocksparse(const void* q, const void* k, const void* v, void* out, float* lse,
