@@ -9,7 +9,7 @@
 //
 // B200 mapping, default shape (one CTA per SM, 384 threads, 2 Q tiles of 128 rows per CTA;
 // setmaxnreg gives the softmax warpgroups 200 registers per thread and the producer / MMA
-// warpgroup 104; the single-Q-tile shape used for sliding windows is described at FwdShape):
+// warpgroup 104; the single-Q-tile shape that uncapped dense calls use is described at FwdShape):
 //   warp 8      TMA producer: Q tiles once, then K and V tiles through 2-stage rings (128-byte
 //               swizzled smem, 3-D tensor maps so tails are zero-filled per head).
 //   warp 9      TMEM owner and single-thread tcgen05.mma issuer:
